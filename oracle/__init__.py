@@ -1,0 +1,13 @@
+"""CPU float64 oracle for CLEAR attention. Test infrastructure only: imported by tests/,
+__graft_entry__.smoke() and bench.py's CPU-baseline / reference legs, never by the product path."""
+from .clear_attention import (  # noqa: F401
+    token_coords,
+    clear_mask,
+    clear_attention_forward,
+    clear_attention_rows,
+    clear_attention_backward,
+    window_lattice_count,
+    window_pairs,
+    kept_pairs,
+    useful_flops_fwd,
+)

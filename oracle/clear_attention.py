@@ -1,0 +1,209 @@
+"""Plain, slow CPU float64 oracle for CLEAR attention. TEST INFRASTRUCTURE ONLY.
+
+Only the tests, the smoke check and the bench's CPU-baseline / reference legs may import this
+module. The product path (the CUDA library and its Python binding) never calls it, and this module
+imports nothing from the product package.
+
+What it computes (sources are the pages about arXiv 2412.16112, "CLEAR: Conv-Like Linearization
+Revs Pre-Trained Diffusion Transformers Up"):
+
+* "pith review" = the pith.science machine review of the paper;
+* "atlas summary" = the atlas.scime.ai AI summary of the paper.
+
+1. Mask  [pith review, "Core claim"]: with text tokens first, M_ij = 1 iff i is a text token, or
+   j is a text token, or the Euclidean grid distance of image tokens i and j is below r:
+   dx^2 + dy^2 < r^2.  The review writes the condition 1-based (i <= n_text); here indices are
+   0-based, so "text" means index < n_text.
+2. One softmax over the union of text keys and window keys  [atlas summary, "Approach";
+   pith review, "What carries the argument" (formulation consistency with softmax attention,
+   Eq. 1 in "Assumptions")].
+3. Scale 1/sqrt(c), c = head dim  [pith review, "What carries the argument", the Eq. 7 text].
+4. Backward (dQ, dK, dV): the pages print none; they say only the attention layers are fine-tuned
+   by gradient descent [pith review, "The reading"], so the gradient is the analytic gradient of
+   the forward above (standard softmax-attention calculus, written out in `clear_attention_backward`).
+
+Readings where the pages leave a step open (each listed with its reason in the design notes):
+strict "<" in the radius test; image tokens in row-major order t = n_text + y*W + x; windows are
+clipped at the grid border (border queries see fewer keys); text queries attend to every token
+exactly (no patch-wise approximation); LSE is the natural-log log-sum-exp of the scaled, masked
+scores; r is an integer >= 1.
+
+Everything here is float64 and builds the explicit mask, with no blocking or fusion.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+
+# ----------------------------------------------------------------------------------------------
+# Geometry and mask
+# ----------------------------------------------------------------------------------------------
+
+def token_coords(n_text: int, H: int, W: int):
+    """Grid coordinates (y, x) of every token; text tokens get (-1, -1) and is_text=True.
+
+    Image token (y, x) sits at index n_text + y*W + x (row-major reading of the grid order).
+    """
+    T = n_text + H * W
+    y = np.full(T, -1, dtype=np.int64)
+    x = np.full(T, -1, dtype=np.int64)
+    img = np.arange(H * W, dtype=np.int64)
+    y[n_text:] = img // W
+    x[n_text:] = img % W
+    is_text = np.zeros(T, dtype=bool)
+    is_text[:n_text] = True
+    return y, x, is_text
+
+
+def clear_mask(n_text: int, H: int, W: int, r: int, rows=None) -> np.ndarray:
+    """Boolean CLEAR mask M [len(rows), T] (all T rows if rows is None).
+
+    [pith review, "Core claim"]: M_ij = 1 if i <= n_text or j <= n_text or
+    (d^x_ij)^2 + (d^y_ij)^2 < r^2 (1-based there; 0-based "< n_text" here).
+    """
+    y, x, is_text = token_coords(n_text, H, W)
+    T = y.shape[0]
+    rows = np.arange(T) if rows is None else np.asarray(rows, dtype=np.int64)
+    dy = y[rows][:, None] - y[None, :]
+    dx = x[rows][:, None] - x[None, :]
+    near = dx * dx + dy * dy < r * r
+    return is_text[rows][:, None] | is_text[None, :] | near
+
+
+# ----------------------------------------------------------------------------------------------
+# Forward / backward (explicit mask, float64)
+# ----------------------------------------------------------------------------------------------
+
+def _as_f64(a) -> np.ndarray:
+    if hasattr(a, "detach"):  # a torch tensor: exact upcast (bf16 and fp32 are exact in fp64)
+        a = a.detach().to("cpu").double().numpy()
+    return np.asarray(a, dtype=np.float64)
+
+
+def _masked_softmax_rows(S: np.ndarray, M: np.ndarray):
+    """Row softmax of S restricted to M; returns (P, LSE). Masked entries get probability 0."""
+    S = np.where(M, S, -np.inf)
+    m = S.max(axis=1, keepdims=True)
+    E = np.exp(S - m)
+    l = E.sum(axis=1, keepdims=True)
+    P = E / l
+    lse = (m + np.log(l))[:, 0]
+    return P, lse
+
+
+def clear_attention_forward(q, k, v, n_text: int, H: int, W: int, r: int, scale=None):
+    """O = softmax_M(Q K^T * scale) V and LSE for every (batch, head).
+
+    q, k, v: [B, heads, T, d] (numpy or torch; upcast exactly to float64).
+    Returns O [B, heads, T, d] float64 and LSE [B, heads, T] float64 (natural log).
+    Scale defaults to 1/sqrt(d) [pith review, "What carries the argument", Eq. 7 text].
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    B, Hh, T, d = q.shape
+    assert T == n_text + H * W, "T must equal n_text + H*W"
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    M = clear_mask(n_text, H, W, r)
+    O = np.empty_like(q)
+    LSE = np.empty((B, Hh, T))
+    for b in range(B):
+        for h in range(Hh):
+            S = (q[b, h] @ k[b, h].T) * scale
+            P, lse = _masked_softmax_rows(S, M)
+            O[b, h] = P @ v[b, h]
+            LSE[b, h] = lse
+    return O, LSE
+
+
+def clear_attention_rows(q, k, v, n_text: int, H: int, W: int, r: int, b: int, h: int, rows,
+                         scale=None):
+    """Forward outputs for selected query rows of one (b, h) only; mask rows built explicitly.
+
+    Used where the full T x T mask does not fit (e.g. a 512 x 512 grid, T = 262,656).
+    Returns O_rows [len(rows), d] and LSE_rows [len(rows)] in float64.
+    """
+    qb = _as_f64(q[b, h][rows] if hasattr(q, "detach") else np.asarray(q)[b, h][rows])
+    kb, vb = _as_f64(k[b, h]), _as_f64(v[b, h])
+    d = qb.shape[-1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    M = clear_mask(n_text, H, W, r, rows=rows)
+    S = (qb @ kb.T) * scale
+    P, lse = _masked_softmax_rows(S, M)
+    return P @ vb, lse
+
+
+def clear_attention_backward(q, k, v, dO, n_text: int, H: int, W: int, r: int, scale=None):
+    """Analytic gradient of the forward above with respect to q, k and v, given dO.
+
+    With S = scale * Q K^T, P = softmax_M(S) row-wise and O = P V:
+        dV = P^T dO
+        dP = dO V^T
+        D_i = sum_j P_ij dP_ij  (= rowsum(dO o O))
+        dS = P o (dP - D)
+        dQ = scale * dS K
+        dK = scale * dS^T Q
+    Masked entries have P = 0, so they carry no gradient.
+    """
+    q, k, v, dO = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(dO)
+    B, Hh, T, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    M = clear_mask(n_text, H, W, r)
+    dq = np.empty_like(q)
+    dk = np.empty_like(k)
+    dv = np.empty_like(v)
+    for b in range(B):
+        for h in range(Hh):
+            S = (q[b, h] @ k[b, h].T) * scale
+            P, _ = _masked_softmax_rows(S, M)
+            O = P @ v[b, h]
+            dv[b, h] = P.T @ dO[b, h]
+            dP = dO[b, h] @ v[b, h].T
+            D = (dO[b, h] * O).sum(axis=1, keepdims=True)
+            dS = P * (dP - D)
+            dq[b, h] = scale * (dS @ k[b, h])
+            dk[b, h] = scale * (dS.T @ q[b, h])
+    return dq, dk, dv
+
+
+# ----------------------------------------------------------------------------------------------
+# Counting: window size, kept pairs, useful FLOPs
+# ----------------------------------------------------------------------------------------------
+
+def window_lattice_count(r: int) -> int:
+    """Keys in an interior query's window: #{(dx, dy) in Z^2 : dx^2 + dy^2 < r^2}.
+
+    [pith review, "What carries the argument"]: the window's key count is constant in the
+    resolution and is about pi/4 of the square window's.
+    """
+    n = 0
+    for dy in range(-r, r + 1):
+        rem = r * r - dy * dy
+        if rem <= 0:
+            continue
+        w = math.isqrt(rem - 1)  # largest dx with dx^2 < rem
+        n += 2 * w + 1
+    return n
+
+
+def window_pairs(H: int, W: int, r: int) -> int:
+    """Kept image-image pairs P(r) with border clipping: sum over offsets of the overlap area."""
+    total = 0
+    for dy in range(-(r - 1), r):
+        rem = r * r - dy * dy
+        w = math.isqrt(rem - 1)
+        for dx in range(-w, w + 1):
+            total += max(0, H - abs(dy)) * max(0, W - abs(dx))
+    return total
+
+
+def kept_pairs(n_text: int, H: int, W: int, r: int) -> int:
+    """Number of ones in M: text rows (all T keys) + image rows x text keys + window pairs."""
+    N = H * W
+    T = n_text + N
+    return n_text * T + N * n_text + window_pairs(H, W, r)
+
+
+def useful_flops_fwd(B: int, heads: int, n_text: int, H: int, W: int, r: int, d: int) -> int:
+    """Forward FLOPs on kept pairs only: 2*d for q.k plus 2*d for p*v, per kept (q, k) pair."""
+    return 4 * d * B * heads * kept_pairs(n_text, H, W, r)
