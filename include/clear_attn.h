@@ -1,0 +1,144 @@
+/*
+ * clear_attn.h — C ABI of the B200 (sm_100a) CLEAR attention library (libclear_attn.so).
+ *
+ * CLEAR ("CLEAR: Conv-Like Linearization Revs Pre-Trained Diffusion Transformers Up",
+ * arXiv 2412.16112) replaces full attention in a diffusion transformer by a mask that keeps a
+ * (query i, key j) pair iff i is a text token, or j is a text token, or image tokens i and j lie at
+ * squared Euclidean grid distance dx^2 + dy^2 < r^2 (pith.science review, "Core claim"; atlas.scime.ai
+ * summary, "Approach"). Each query row takes one softmax over its kept keys, with scores scaled by
+ * 1/sqrt(d) (pith.science review, "What carries the argument", Eq. 7 text).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Tensors are dense, row-major, on the current CUDA device, with shape [B, heads, T, d] where
+ * T = n_text + H*W: the n_text text tokens come first, then the image tokens of an H x W grid in
+ * row-major order (token n_text + y*W + x is grid position (y, x)). Element type is bf16 for
+ * q, k, v, o, dO, dq, dk, dv; lse is fp32 [B, heads, T], natural log of the softmax denominator
+ * of the scaled, masked scores. Every pointer must be 16-byte aligned.
+ *
+ * Windows are clipped at the grid border (border queries see fewer keys). Text query rows attend
+ * to all T keys exactly. r is an integer >= 1; any r whose square exceeds the grid diagonal's
+ * square keeps every pair (full attention). Supported head dims: d = 64 and d = 128.
+ *
+ * Ownership: the caller owns every buffer and the stream. The library allocates no device memory
+ * in these calls; scratch space comes from the caller's workspace (size from the *_workspace_size
+ * queries). Outputs are written in full; inputs are never written.
+ *
+ * Asynchrony and errors: calls enqueue kernels on `stream` (a cudaStream_t passed as void*;
+ * NULL = legacy default stream) and return without synchronising. Argument errors are detected on
+ * the host before anything is launched: the call returns the error status and leaves every output
+ * untouched. A kernel whose internal bounded wait expired records a device error word instead of
+ * hanging; clear_attn_check() synchronises the stream and reports it as CLEAR_ERR_DEVICE_TIMEOUT.
+ * Calls are thread-safe (no mutable global state besides the device error word).
+ */
+#ifndef CLEAR_ATTN_H_
+#define CLEAR_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(CLEAR_BUILD_SO) && defined(__GNUC__)
+#define CLEAR_API __attribute__((visibility("default")))
+#else
+#define CLEAR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CLEAR_OK = 0,
+  CLEAR_ERR_INVALID_ARG = 1,      /* null/misaligned pointer, non-positive size, r < 1, overflow */
+  CLEAR_ERR_UNSUPPORTED = 2,      /* d not in {64, 128}, or no sm_100 device */
+  CLEAR_ERR_WORKSPACE = 3,        /* workspace missing or smaller than the queried size */
+  CLEAR_ERR_CUDA = 4,             /* a CUDA runtime/driver call failed (launch, tensor map) */
+  CLEAR_ERR_DEVICE_TIMEOUT = 5    /* a kernel's bounded wait expired (reported by clear_attn_check) */
+} clear_status_t;
+
+/* Problem description. All fields are plain element counts. */
+typedef struct {
+  int B;        /* batch size, >= 1 */
+  int heads;    /* attention heads, >= 1 */
+  int n_text;   /* text tokens placed before the image tokens, >= 0 */
+  int H, W;     /* image token grid, >= 1 each */
+  int d;        /* head dim: 64 or 128 */
+  int r;        /* window radius in grid units (strict: dx^2 + dy^2 < r^2), >= 1 */
+} clear_attn_params_t;
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+CLEAR_API int clear_attn_version(void);
+
+/* Human-readable name of a status code (static storage). */
+CLEAR_API const char* clear_status_string(clear_status_t status);
+
+/* Bytes of caller-provided device workspace clear_attn_fwd needs (0 when n_text == 0).
+ * Returns 0 and sets *status (if non-NULL) on invalid params. */
+CLEAR_API size_t clear_attn_fwd_workspace_size(const clear_attn_params_t* params, clear_status_t* status);
+
+/* Bytes of caller-provided device workspace clear_attn_bwd needs. */
+CLEAR_API size_t clear_attn_bwd_workspace_size(const clear_attn_params_t* params, clear_status_t* status);
+
+/*
+ * Forward: o = softmax_M(q k^T / sqrt(d)) v, lse = log sum_j exp(q_i.k_j / sqrt(d)) over kept j.
+ *   q, k, v   in : bf16 [B, heads, T, d]
+ *   o         out: bf16 [B, heads, T, d]
+ *   lse       out: fp32 [B, heads, T]
+ *   workspace in/out scratch: device memory of at least clear_attn_fwd_workspace_size() bytes
+ *             (may be NULL when that size is 0); contents are undefined on return.
+ *   stream    cudaStream_t (as void*).
+ */
+CLEAR_API clear_status_t clear_attn_fwd(const clear_attn_params_t* params, const void* q, const void* k,
+                              const void* v, void* o, float* lse, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/*
+ * Backward of clear_attn_fwd with respect to q, k and v, given the upstream gradient dO and the
+ * forward's o and lse (analytic softmax-attention gradient restricted to the mask):
+ *   dV = P^T dO;  dP = dO V^T;  D = rowsum(dO o O);  dS = P o (dP - D);
+ *   dQ = dS K / sqrt(d);  dK = dS^T Q / sqrt(d).
+ *   q, k, v, o, dO  in : bf16 [B, heads, T, d];  lse in: fp32 [B, heads, T]
+ *   dq, dk, dv      out: bf16 [B, heads, T, d]
+ *   workspace       scratch of at least clear_attn_bwd_workspace_size() bytes.
+ */
+CLEAR_API clear_status_t clear_attn_bwd(const clear_attn_params_t* params, const void* q, const void* k,
+                              const void* v, const void* o, const float* lse, const void* dO,
+                              void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/* Synchronises `stream`, then reads and clears the device error word of the current device.
+ * Returns CLEAR_OK, CLEAR_ERR_DEVICE_TIMEOUT (a kernel gave up a bounded wait; its outputs are
+ * invalid) or CLEAR_ERR_CUDA (the stream reported a CUDA error). */
+CLEAR_API clear_status_t clear_attn_check(void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Host-only scheduler queries (no GPU needed). They expose the tile enumeration the kernels use,
+ * so its coverage can be checked against a brute-force mask on the CPU.
+ * --------------------------------------------------------------------------------------------- */
+
+/* Work-list shape of the forward: numbers of text (split) items and image items, the text split
+ * count S and 128-key chunks per split. Any output pointer may be NULL. */
+CLEAR_API clear_status_t clear_sched_forward_shape(const clear_attn_params_t* params, long long* n_text_items,
+                                         long long* n_image_items, int* splits,
+                                         int* chunks_per_split);
+
+/* Key tiles visited by forward work item `item` (0 <= item < n_text_items + n_image_items), in
+ * order. Each tile is 4 ints: kind (0 = linear chunk, 1 = image rectangle), a, b, flags
+ * (1 = every pair kept, no mask needed). Linear: tokens [a, a + 128), first b of them real.
+ * Rectangle: grid rows [a, a + 8) x columns [b, b + 16). Also returns the item's query tile:
+ * q_info = {is_text, bh, q0 (first token, or first grid row), x0 (first grid column)}.
+ * Writes at most max_tiles tiles; returns the item's total tile count via *n_tiles. */
+CLEAR_API clear_status_t clear_sched_item_tiles(const clear_attn_params_t* params, long long item,
+                                      int* q_info, int* tiles, int max_tiles, int* n_tiles);
+
+/* Useful (kept-pair) and executed (padded-tile) multiply-add pair counts of one forward call,
+ * summed over B and heads: useful = number of ones in the mask; executed = 128 x 128 per visited
+ * tile pair. FLOPs are 4 * d times these. */
+CLEAR_API clear_status_t clear_sched_pair_counts(const clear_attn_params_t* params, long long* useful_pairs,
+                                       long long* executed_pairs);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CLEAR_ATTN_H_ */

@@ -1,0 +1,202 @@
+"""ctypes binding of libclear_attn.so (argument marshalling only: every step runs in the library).
+
+The library must have been built (``python -m local_circular_window_b200.build`` or
+``__graft_entry__.build()``); importing this module without it raises ImportError. There is no
+fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libclear_attn.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "clear_attn.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m local_circular_window_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+CLEAR_OK = 0
+STATUS_NAMES = {0: "CLEAR_OK", 1: "CLEAR_ERR_INVALID_ARG", 2: "CLEAR_ERR_UNSUPPORTED", 3: "CLEAR_ERR_WORKSPACE",
+                4: "CLEAR_ERR_CUDA", 5: "CLEAR_ERR_DEVICE_TIMEOUT"}
+
+
+class ClearParams(ctypes.Structure):
+    """Mirror of clear_attn_params_t."""
+    _fields_ = [("B", ctypes.c_int), ("heads", ctypes.c_int), ("n_text", ctypes.c_int), ("H", ctypes.c_int),
+                ("W", ctypes.c_int), ("d", ctypes.c_int), ("r", ctypes.c_int)]
+
+
+class ClearError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+_P = ctypes.POINTER(ClearParams)
+_vp = ctypes.c_void_p
+_ll = ctypes.c_longlong
+_i = ctypes.c_int
+
+_lib.clear_attn_version.restype = _i
+_lib.clear_status_string.restype = ctypes.c_char_p
+_lib.clear_status_string.argtypes = [_i]
+_lib.clear_attn_fwd_workspace_size.restype = ctypes.c_size_t
+_lib.clear_attn_fwd_workspace_size.argtypes = [_P, ctypes.POINTER(_i)]
+_lib.clear_attn_bwd_workspace_size.restype = ctypes.c_size_t
+_lib.clear_attn_bwd_workspace_size.argtypes = [_P, ctypes.POINTER(_i)]
+_lib.clear_attn_fwd.restype = _i
+_lib.clear_attn_fwd.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+_lib.clear_attn_bwd.restype = _i
+_lib.clear_attn_bwd.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+_lib.clear_attn_check.restype = _i
+_lib.clear_attn_check.argtypes = [_vp]
+_lib.clear_sched_forward_shape.restype = _i
+_lib.clear_sched_forward_shape.argtypes = [_P, ctypes.POINTER(_ll), ctypes.POINTER(_ll), ctypes.POINTER(_i),
+                                           ctypes.POINTER(_i)]
+_lib.clear_sched_item_tiles.restype = _i
+_lib.clear_sched_item_tiles.argtypes = [_P, _ll, ctypes.POINTER(_i), ctypes.POINTER(_i), _i, ctypes.POINTER(_i)]
+_lib.clear_sched_pair_counts.restype = _i
+_lib.clear_sched_pair_counts.argtypes = [_P, ctypes.POINTER(_ll), ctypes.POINTER(_ll)]
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/clear_attn.h declares."""
+    text = open(HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(clear_[a-z_]+)\s*\(", text)))
+
+
+def make_params(B: int, heads: int, n_text: int, H: int, W: int, d: int, r: int) -> ClearParams:
+    return ClearParams(B, heads, n_text, H, W, d, r)
+
+
+def version() -> int:
+    return _lib.clear_attn_version()
+
+
+def status_string(status: int) -> str:
+    return _lib.clear_status_string(status).decode()
+
+
+def fwd_workspace_size(p: ClearParams) -> int:
+    st = _i(0)
+    n = _lib.clear_attn_fwd_workspace_size(ctypes.byref(p), ctypes.byref(st))
+    if st.value != CLEAR_OK:
+        raise ClearError(st.value, "clear_attn_fwd_workspace_size")
+    return n
+
+
+def bwd_workspace_size(p: ClearParams) -> int:
+    st = _i(0)
+    n = _lib.clear_attn_bwd_workspace_size(ctypes.byref(p), ctypes.byref(st))
+    if st.value != CLEAR_OK:
+        raise ClearError(st.value, "clear_attn_bwd_workspace_size")
+    return n
+
+
+def forward_shape(p: ClearParams):
+    nt, ni, s, c = _ll(0), _ll(0), _i(0), _i(0)
+    st = _lib.clear_sched_forward_shape(ctypes.byref(p), ctypes.byref(nt), ctypes.byref(ni), ctypes.byref(s),
+                                        ctypes.byref(c))
+    if st != CLEAR_OK:
+        raise ClearError(st, "clear_sched_forward_shape")
+    return nt.value, ni.value, s.value, c.value
+
+
+def item_tiles(p: ClearParams, item: int):
+    """(q_info, tiles) of one forward work item; tiles is a list of (kind, a, b, flags)."""
+    q = (_i * 4)()
+    n = _i(0)
+    st = _lib.clear_sched_item_tiles(ctypes.byref(p), item, q, None, 0, ctypes.byref(n))
+    if st != CLEAR_OK:
+        raise ClearError(st, "clear_sched_item_tiles")
+    buf = (_i * (4 * max(1, n.value)))()
+    st = _lib.clear_sched_item_tiles(ctypes.byref(p), item, q, buf, n.value, ctypes.byref(n))
+    if st != CLEAR_OK:
+        raise ClearError(st, "clear_sched_item_tiles")
+    tiles = [tuple(buf[4 * i:4 * i + 4]) for i in range(n.value)]
+    return tuple(q), tiles
+
+
+def pair_counts(p: ClearParams):
+    u, e = _ll(0), _ll(0)
+    st = _lib.clear_sched_pair_counts(ctypes.byref(p), ctypes.byref(u), ctypes.byref(e))
+    if st != CLEAR_OK:
+        raise ClearError(st, "clear_sched_pair_counts")
+    return u.value, e.value
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_qkv(name, t, shape):
+    if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous() and tuple(t.shape) == tuple(shape)):
+        raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {tuple(shape)}")
+
+
+def clear_attn_fwd(q, k, v, n_text: int, H: int, W: int, r: int, o=None, lse=None, workspace=None, stream=None):
+    """CLEAR attention forward through the C ABI. Returns (o, lse); raises ClearError on failure."""
+    B, heads, T, d = q.shape
+    if T != n_text + H * W:
+        raise ValueError("T must equal n_text + H * W")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_qkv(name, t, q.shape)
+    p = make_params(B, heads, n_text, H, W, d, r)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, heads, T), dtype=torch.float32, device=q.device)
+    ws_bytes = fwd_workspace_size(p)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    st = _lib.clear_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(workspace),
+                             0 if workspace is None else workspace.numel() * workspace.element_size(),
+                             _stream_ptr(stream))
+    if st != CLEAR_OK:
+        raise ClearError(st, "clear_attn_fwd")
+    return o, lse
+
+
+def clear_attn_bwd(q, k, v, o, lse, dO, n_text: int, H: int, W: int, r: int, dq=None, dk=None, dv=None,
+                   workspace=None, stream=None):
+    """CLEAR attention backward through the C ABI. Returns (dq, dk, dv)."""
+    B, heads, T, d = q.shape
+    if T != n_text + H * W:
+        raise ValueError("T must equal n_text + H * W")
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dO", dO)):
+        _check_qkv(name, t, q.shape)
+    p = make_params(B, heads, n_text, H, W, d, r)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    ws_bytes = bwd_workspace_size(p)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    st = _lib.clear_attn_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq),
+                             _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                             _stream_ptr(stream))
+    if st != CLEAR_OK:
+        raise ClearError(st, "clear_attn_bwd")
+    return dq, dk, dv
+
+
+def clear_attn_check(stream=None) -> int:
+    """Synchronise the stream and return the device status (CLEAR_OK or an error code)."""
+    return _lib.clear_attn_check(_stream_ptr(stream))

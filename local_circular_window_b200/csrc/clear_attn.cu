@@ -1,0 +1,354 @@
+// Host side of libclear_attn.so: argument validation, TMA tensor-map encoding, kernel launches and
+// the host-only scheduler queries. The C ABI is declared in include/clear_attn.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "clear_attn.h"
+#include "clear_bwd.cuh"
+#include "clear_fwd.cuh"
+#include "clear_sched.cuh"
+
+using namespace clear;
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+// ------------------------------------------------------------------------------------------------
+// Validation
+// ------------------------------------------------------------------------------------------------
+struct Checked {
+  clear_status_t st;
+  Geom g;
+};
+
+// Radius beyond which every pair of the grid is kept; larger radii are clamped to it.
+int full_radius(int H, int W) {
+  long long d2 = (long long)(H - 1) * (H - 1) + (long long)(W - 1) * (W - 1);
+  long long r = (long long)std::sqrt((double)d2);
+  while (r * r > d2) --r;
+  while ((r + 1) * (r + 1) <= d2) ++r;
+  return (int)(r + 1);  // (r+1)^2 > d2
+}
+
+Checked check_params(const clear_attn_params_t* p) {
+  Checked c{};
+  c.st = CLEAR_ERR_INVALID_ARG;
+  if (!p) return c;
+  if (p->B < 1 || p->heads < 1 || p->n_text < 0 || p->H < 1 || p->W < 1 || p->r < 1) return c;
+  if (p->d != 64 && p->d != 128) {
+    c.st = CLEAR_ERR_UNSUPPORTED;
+    return c;
+  }
+  const long long N = (long long)p->H * p->W;
+  const long long T = N + p->n_text;
+  const long long BH = (long long)p->B * p->heads;
+  if (N > (1ll << 28) || p->n_text > (1 << 24) || T > (1ll << 30) || BH > (1ll << 20)) return c;
+  if (BH * T * p->d >= (1ll << 40)) return c;
+  const int r = p->r < full_radius(p->H, p->W) ? p->r : full_radius(p->H, p->W);
+  c.g = make_geom(p->B, p->heads, p->n_text, p->H, p->W, p->d, r);
+  c.st = CLEAR_OK;
+  return c;
+}
+
+bool aligned16(const void* ptr) { return ptr && (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct FwdWorkspace {
+  size_t opart_off, ml_off, total;
+};
+
+FwdWorkspace fwd_workspace_layout(const Geom& g) {
+  FwdWorkspace w{};
+  if (g.n_text == 0) return w;
+  const size_t rows = (size_t)g.S * g.BH * g.n_text;
+  w.opart_off = 0;
+  w.ml_off = align256(rows * g.d * sizeof(float));
+  w.total = align256(w.ml_off + rows * sizeof(float2));
+  return w;
+}
+
+// ------------------------------------------------------------------------------------------------
+// Device checks and TMA descriptors
+// ------------------------------------------------------------------------------------------------
+clear_status_t check_device(int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CLEAR_ERR_CUDA;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return CLEAR_ERR_CUDA;
+  if (major != 10) return CLEAR_ERR_UNSUPPORTED;
+  if (cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return CLEAR_ERR_CUDA;
+  return CLEAR_OK;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// [BH, T, d] viewed as a 3D tensor (d, T, BH); box = 64 x 128 x 1, 128-byte swizzle.
+bool make_linear_map(CUtensorMap* m, const void* base, const Geom& g) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)g.d, (cuuint64_t)g.T, (cuuint64_t)g.BH};
+  cuuint64_t strides[2] = {(cuuint64_t)g.d * 2, (cuuint64_t)g.T * g.d * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)kTile, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Image part of [BH, T, d] viewed as a 4D tensor (d, W, H, BH) starting at token n_text;
+// box = 64 x 16 x 8 x 1 (an 8 x 16 grid rectangle), 128-byte swizzle, zero fill outside the grid.
+bool make_image_map(CUtensorMap* m, const void* base, const Geom& g) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const char* img = static_cast<const char*>(base) + (size_t)g.n_text * g.d * 2;
+  cuuint64_t dims[4] = {(cuuint64_t)g.d, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.BH};
+  cuuint64_t strides[3] = {(cuuint64_t)g.d * 2, (cuuint64_t)g.W * g.d * 2, (cuuint64_t)g.T * g.d * 2};
+  cuuint32_t box[4] = {64, (cuuint32_t)kKW, (cuuint32_t)kKH, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<char*>(img), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct QKVMaps {
+  CUtensorMap q_lin, q_img, k_lin, k_img, v_lin, v_img;
+};
+
+bool make_qkv_maps(QKVMaps* m, const void* q, const void* k, const void* v, const Geom& g) {
+  return make_linear_map(&m->q_lin, q, g) && make_image_map(&m->q_img, q, g) &&
+         make_linear_map(&m->k_lin, k, g) && make_image_map(&m->k_img, k, g) &&
+         make_linear_map(&m->v_lin, v, g) && make_image_map(&m->v_img, v, g);
+}
+
+template <int D>
+clear_status_t launch_fwd(const Geom& g, const QKVMaps& m, void* o, float* lse, void* ws,
+                          int num_sms, cudaStream_t stream) {
+  using L = FwdLayout<D>;
+  FwdParams p{};
+  p.g = g;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  const FwdWorkspace wl = fwd_workspace_layout(g);
+  p.opart = g.n_text ? reinterpret_cast<float*>(static_cast<char*>(ws) + wl.opart_off) : nullptr;
+  p.ml = g.n_text ? reinterpret_cast<float2*>(static_cast<char*>(ws) + wl.ml_off) : nullptr;
+  p.n_work = g.n_txt_items + g.n_img_items;
+  if (cudaFuncSetAttribute(clear_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           L::kAlloc) != cudaSuccess)
+    return CLEAR_ERR_CUDA;
+  const long long grid = p.n_work < num_sms ? p.n_work : num_sms;
+  clear_fwd_kernel<D><<<(unsigned)grid, kFwdThreads, L::kAlloc, stream>>>(
+      m.q_lin, m.q_img, m.k_lin, m.k_img, m.v_lin, m.v_img, p);
+  if (cudaGetLastError() != cudaSuccess) return CLEAR_ERR_CUDA;
+  if (g.n_text > 0) {
+    const long long rows = (long long)g.BH * g.n_text;
+    const int wpb = 8;
+    clear_fwd_combine_kernel<D><<<(unsigned)((rows + wpb - 1) / wpb), wpb * 32, 0, stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return CLEAR_ERR_CUDA;
+  }
+  return CLEAR_OK;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------------------------------------
+// C ABI
+// ------------------------------------------------------------------------------------------------
+extern "C" {
+
+int clear_attn_version(void) { return kVersion; }
+
+const char* clear_status_string(clear_status_t s) {
+  switch (s) {
+    case CLEAR_OK: return "CLEAR_OK";
+    case CLEAR_ERR_INVALID_ARG: return "CLEAR_ERR_INVALID_ARG";
+    case CLEAR_ERR_UNSUPPORTED: return "CLEAR_ERR_UNSUPPORTED";
+    case CLEAR_ERR_WORKSPACE: return "CLEAR_ERR_WORKSPACE";
+    case CLEAR_ERR_CUDA: return "CLEAR_ERR_CUDA";
+    case CLEAR_ERR_DEVICE_TIMEOUT: return "CLEAR_ERR_DEVICE_TIMEOUT";
+  }
+  return "CLEAR_ERR_UNKNOWN";
+}
+
+size_t clear_attn_fwd_workspace_size(const clear_attn_params_t* params, clear_status_t* status) {
+  const Checked c = check_params(params);
+  if (status) *status = c.st;
+  if (c.st != CLEAR_OK) return 0;
+  return fwd_workspace_layout(c.g).total;
+}
+
+size_t clear_attn_bwd_workspace_size(const clear_attn_params_t* params, clear_status_t* status) {
+  const Checked c = check_params(params);
+  if (status) *status = c.st;
+  if (c.st != CLEAR_OK) return 0;
+  return bwd_workspace_layout(c.g).total;
+}
+
+clear_status_t clear_attn_fwd(const clear_attn_params_t* params, const void* q, const void* k,
+                              const void* v, void* o, float* lse, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  const Checked c = check_params(params);
+  if (c.st != CLEAR_OK) return c.st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return CLEAR_ERR_INVALID_ARG;
+  const size_t need = fwd_workspace_layout(c.g).total;
+  if (need > 0 && (workspace_bytes < need || !aligned16(workspace))) return CLEAR_ERR_WORKSPACE;
+  int num_sms = 0;
+  clear_status_t st = check_device(&num_sms);
+  if (st != CLEAR_OK) return st;
+  QKVMaps maps;
+  if (!make_qkv_maps(&maps, q, k, v, c.g)) return CLEAR_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return c.g.d == 128 ? launch_fwd<128>(c.g, maps, o, lse, workspace, num_sms, s)
+                      : launch_fwd<64>(c.g, maps, o, lse, workspace, num_sms, s);
+}
+
+clear_status_t clear_attn_bwd(const clear_attn_params_t* params, const void* q, const void* k,
+                              const void* v, const void* o, const float* lse, const void* dO,
+                              void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  const Checked c = check_params(params);
+  if (c.st != CLEAR_OK) return c.st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      !aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return CLEAR_ERR_INVALID_ARG;
+  const BwdWorkspace wl = bwd_workspace_layout(c.g);
+  if (workspace_bytes < wl.total || !aligned16(workspace)) return CLEAR_ERR_WORKSPACE;
+  int num_sms = 0;
+  clear_status_t st = check_device(&num_sms);
+  if (st != CLEAR_OK) return st;
+  QKVMaps maps;
+  if (!make_qkv_maps(&maps, q, k, v, c.g)) return CLEAR_ERR_CUDA;
+  CUtensorMap do_lin, do_img;
+  if (!make_linear_map(&do_lin, dO, c.g) || !make_image_map(&do_img, dO, c.g)) return CLEAR_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  BwdArgs a{};
+  a.g = c.g;
+  a.o = static_cast<const __nv_bfloat16*>(o);
+  a.dO = static_cast<const __nv_bfloat16*>(dO);
+  a.lse = lse;
+  a.dq = static_cast<__nv_bfloat16*>(dq);
+  a.dk = static_cast<__nv_bfloat16*>(dk);
+  a.dv = static_cast<__nv_bfloat16*>(dv);
+  a.ws = static_cast<char*>(workspace);
+  a.wl = wl;
+  return c.g.d == 128 ? launch_bwd<128>(a, maps.q_lin, maps.q_img, maps.k_lin, maps.k_img, maps.v_lin,
+                                        maps.v_img, do_lin, do_img, num_sms, s)
+                      : launch_bwd<64>(a, maps.q_lin, maps.q_img, maps.k_lin, maps.k_img, maps.v_lin,
+                                       maps.v_img, do_lin, do_img, num_sms, s);
+}
+
+clear_status_t clear_attn_check(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return CLEAR_ERR_CUDA;
+  int err = 0;
+  if (cudaMemcpyFromSymbol(&err, clear::g_clear_device_error, sizeof(int)) != cudaSuccess)
+    return CLEAR_ERR_CUDA;
+  if (err != 0) {
+    const int zero = 0;
+    cudaMemcpyToSymbol(clear::g_clear_device_error, &zero, sizeof(int));
+    return CLEAR_ERR_DEVICE_TIMEOUT;
+  }
+  return CLEAR_OK;
+}
+
+clear_status_t clear_sched_forward_shape(const clear_attn_params_t* params, long long* n_text_items,
+                                         long long* n_image_items, int* splits,
+                                         int* chunks_per_split) {
+  const Checked c = check_params(params);
+  if (c.st != CLEAR_OK) return c.st;
+  if (n_text_items) *n_text_items = c.g.n_txt_items;
+  if (n_image_items) *n_image_items = c.g.n_img_items;
+  if (splits) *splits = c.g.S;
+  if (chunks_per_split) *chunks_per_split = c.g.cps;
+  return CLEAR_OK;
+}
+
+clear_status_t clear_sched_item_tiles(const clear_attn_params_t* params, long long item, int* q_info,
+                                      int* tiles, int max_tiles, int* n_tiles) {
+  const Checked c = check_params(params);
+  if (c.st != CLEAR_OK) return c.st;
+  if (item < 0 || item >= c.g.n_txt_items + c.g.n_img_items || max_tiles < 0) return CLEAR_ERR_INVALID_ARG;
+  const WorkItem it = decode_work(c.g, item);
+  if (q_info) {
+    q_info[0] = it.is_text;
+    q_info[1] = it.bh;
+    q_info[2] = it.q0;
+    q_info[3] = it.x0;
+  }
+  KeyIter ki;
+  ki.init(c.g, it);
+  KeyTile t;
+  int n = 0;
+  while (ki.next(&t)) {
+    if (tiles && n < max_tiles) {
+      tiles[4 * n + 0] = t.kind;
+      tiles[4 * n + 1] = t.a;
+      tiles[4 * n + 2] = t.b;
+      tiles[4 * n + 3] = t.flags;
+    }
+    ++n;
+  }
+  if (n_tiles) *n_tiles = n;
+  return CLEAR_OK;
+}
+
+clear_status_t clear_sched_pair_counts(const clear_attn_params_t* params, long long* useful_pairs,
+                                       long long* executed_pairs) {
+  const Checked c = check_params(params);
+  if (c.st != CLEAR_OK) return c.st;
+  const Geom& g = c.g;
+  // Kept pairs: text rows see all T keys, image rows see all text keys plus their clipped disc.
+  long long win = 0;
+  for (int dy = -(g.r - 1); dy <= g.r - 1; ++dy) {
+    const int w = half_width(g.r, dy < 0 ? -dy : dy);
+    if (w < 0) continue;
+    const long long rows = g.H - (dy < 0 ? -dy : dy);
+    if (rows <= 0) continue;
+    for (int dx = -w; dx <= w; ++dx) {
+      const long long cols = g.W - (dx < 0 ? -dx : dx);
+      if (cols > 0) win += rows * cols;
+    }
+  }
+  const long long N = (long long)g.H * g.W;
+  const long long per_head = (long long)g.n_text * g.T + N * g.n_text + win;
+  if (useful_pairs) *useful_pairs = per_head * g.BH;
+  if (executed_pairs) {
+    long long tiles = 0;
+    WorkItem it{};
+    for (int qt = 0; qt < g.nQ; ++qt) {  // image items of one (b, h)
+      it = decode_work(g, g.n_txt_items + qt);
+      tiles += count_key_tiles(g, it);
+    }
+    tiles += (long long)g.nTq * g.nC;  // text rows: every chunk once per text query tile
+    *executed_pairs = tiles * (long long)kTile * kTile * g.BH;
+  }
+  return CLEAR_OK;
+}
+
+}  // extern "C"

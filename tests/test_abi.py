@@ -1,0 +1,109 @@
+"""C ABI checks that need no GPU: the library loads, exports every declared symbol, validates its
+arguments on the host and reports sizes. Error paths never launch anything, so they are safe to run
+with host buffers standing in for device pointers (the canaries prove nothing was written)."""
+import ctypes
+
+import numpy as np
+import pytest
+
+import local_circular_window_b200 as L
+from local_circular_window_b200 import _binding as Bd
+
+
+def test_library_exports_every_declared_function():
+    names = L.header_functions()
+    assert len(names) >= 10
+    missing = [n for n in names if not hasattr(L.lib(), n)]
+    assert missing == []
+
+
+def test_version_and_status_strings():
+    assert L.version() >= 100
+    for code, name in Bd.STATUS_NAMES.items():
+        assert L.status_string(code) == name
+    assert L.status_string(99) == "CLEAR_ERR_UNKNOWN"
+
+
+@pytest.mark.parametrize("fields,expected", [
+    (dict(r=0), 1), (dict(B=0), 1), (dict(heads=0), 1), (dict(H=0), 1), (dict(W=-3), 1), (dict(n_text=-1), 1),
+    (dict(d=96), 2), (dict(d=256), 2), (dict(H=1 << 15, W=1 << 15), 1), (dict(n_text=1 << 25), 1),
+])
+def test_invalid_params_statuses(fields, expected):
+    base = dict(B=1, heads=2, n_text=16, H=16, W=16, d=64, r=4)
+    base.update(fields)
+    p = L.make_params(**base)
+    st = ctypes.c_int(0)
+    assert L.lib().clear_attn_fwd_workspace_size(ctypes.byref(p), ctypes.byref(st)) == 0
+    assert st.value == expected
+    assert L.lib().clear_attn_bwd_workspace_size(ctypes.byref(p), ctypes.byref(st)) == 0
+    assert st.value == expected
+
+
+def _canary(n=4096):
+    a = np.full(n, 0x5A, dtype=np.uint8)
+    return a, ctypes.c_void_p(a.ctypes.data)
+
+
+def test_forward_argument_errors_launch_nothing():
+    p = L.make_params(1, 2, 16, 16, 16, 64, 4)
+    bufs = [_canary() for _ in range(6)]
+    q, k, v, o, lse, ws = (b[1] for b in bufs)
+    wsz = L.fwd_workspace_size(p)
+    f = L.lib().clear_attn_fwd
+    # null pointers
+    assert f(ctypes.byref(p), None, k, v, o, lse, ws, wsz, None) == 1
+    assert f(ctypes.byref(p), q, k, v, None, lse, ws, wsz, None) == 1
+    # misaligned pointer
+    assert f(ctypes.byref(p), ctypes.c_void_p(q.value + 2), k, v, o, lse, ws, wsz, None) == 1
+    # workspace too small / missing
+    assert f(ctypes.byref(p), q, k, v, o, lse, ws, wsz - 1, None) == 3
+    assert f(ctypes.byref(p), q, k, v, o, lse, None, wsz, None) == 3
+    # bad params
+    bad = L.make_params(1, 2, 16, 16, 16, 96, 4)
+    assert f(ctypes.byref(bad), q, k, v, o, lse, ws, wsz, None) == 2
+    for a, _ in bufs:
+        assert (a == 0x5A).all()
+
+
+def test_backward_argument_errors_launch_nothing():
+    p = L.make_params(2, 3, 7, 9, 11, 128, 3)
+    bufs = [_canary() for _ in range(10)]
+    q, k, v, o, lse, dO, dq, dk, dv, ws = (b[1] for b in bufs)
+    wsz = L.bwd_workspace_size(p)
+    f = L.lib().clear_attn_bwd
+    assert f(ctypes.byref(p), q, k, v, o, lse, None, dq, dk, dv, ws, wsz, None) == 1
+    assert f(ctypes.byref(p), q, k, v, o, lse, dO, dq, ctypes.c_void_p(dk.value + 8), dv, ws, wsz, None) == 1
+    assert f(ctypes.byref(p), q, k, v, o, lse, dO, dq, dk, dv, ws, wsz - 256, None) == 3
+    zero_r = L.make_params(2, 3, 7, 9, 11, 128, 0)
+    assert f(ctypes.byref(zero_r), q, k, v, o, lse, dO, dq, dk, dv, ws, wsz, None) == 1
+    for a, _ in bufs:
+        assert (a == 0x5A).all()
+
+
+def test_workspace_sizes():
+    # Forward scratch holds the split partials of the text rows: S * BH * n_text rows of d fp32 plus
+    # (max, sum) pairs; none without text.
+    p = L.make_params(1, 24, 512, 64, 64, 128, 8)
+    nt, ni, S, cps = L.forward_shape(p)
+    rows = S * 24 * 512
+    need = rows * 128 * 4 + rows * 8
+    got = L.fwd_workspace_size(p)
+    assert need <= got <= need + 512
+    assert L.fwd_workspace_size(L.make_params(1, 2, 0, 8, 8, 64, 2)) == 0
+    # Backward scratch: D and LSE*log2(e) per row, and three sets of text-row split partials.
+    b = L.bwd_workspace_size(p)
+    assert b >= 2 * 24 * 4608 * 4 + 3 * rows * 128 * 4
+
+
+def test_no_fallback_without_library(monkeypatch, tmp_path):
+    # The binding refuses to import when the shared library is absent (no CPU fallback path).
+    import importlib.util
+    import os
+    src = os.path.join(os.path.dirname(Bd.__file__), "_binding.py")
+    code = open(src).read().replace('LIB_PATH = os.path.join(_PKG, "libclear_attn.so")',
+                                    f'LIB_PATH = {str(tmp_path / "missing.so")!r}')
+    mod_path = tmp_path / "binding_copy.py"
+    mod_path.write_text(code)
+    spec = importlib.util.spec_from_file_location("binding_copy", mod_path)
+    with pytest.raises(ImportError):
+        spec.loader.exec_module(importlib.util.module_from_spec(spec))

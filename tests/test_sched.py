@@ -1,0 +1,110 @@
+"""The tile scheduler (the enumeration the kernels run, exposed by the host-only ABI queries) must
+cover every kept (query, key) pair of the CLEAR mask exactly once and visit no useless tile. The
+truth is the oracle's explicit mask."""
+import itertools
+
+import numpy as np
+import pytest
+
+import local_circular_window_b200 as L
+import oracle
+
+KQH, KQW, KKH, KKW, TILE = 8, 16, 8, 16, 128
+
+
+def _keys_of_tile(tile, n_text, H, W, T):
+    kind, a, b, flags = tile
+    if kind == 0:
+        return list(range(a, a + b))
+    keys = []
+    for y in range(a, a + KKH):
+        for x in range(b, b + KKW):
+            if 0 <= y < H and 0 <= x < W:
+                keys.append(n_text + y * W + x)
+    return keys
+
+
+def _raw_keys_of_tile(tile, n_text, H, W):
+    """All 128 slots of a tile, None where the slot is outside the grid / past the valid count."""
+    kind, a, b, flags = tile
+    if kind == 0:
+        return [a + c if c < b else None for c in range(TILE)]
+    out = []
+    for y in range(a, a + KKH):
+        for x in range(b, b + KKW):
+            out.append(n_text + y * W + x if (0 <= y < H and 0 <= x < W) else None)
+    return out
+
+
+def _queries_of_item(q_info, n_text, H, W, T):
+    is_text, bh, q0, x0 = q_info
+    if is_text:
+        return [t for t in range(q0, q0 + TILE) if t < n_text]
+    return [n_text + y * W + x for y in range(q0, q0 + KQH) for x in range(x0, x0 + KQW) if y < H and x < W]
+
+
+CASES = [(16, 16, 16, 4), (0, 19, 21, 3), (5, 24, 40, 5), (3, 9, 17, 1), (200, 13, 50, 7), (1, 8, 8, 30),
+         (0, 33, 47, 9), (7, 70, 18, 12), (130, 96, 96, 6)]
+
+
+@pytest.mark.parametrize("n_text,H,W,r", CASES)
+def test_tiles_cover_mask_exactly(n_text, H, W, r):
+    p = L.make_params(1, 1, n_text, H, W, 64, r)
+    T = n_text + H * W
+    n_txt_items, n_img_items, S, cps = L.forward_shape(p)
+    M = oracle.clear_mask(n_text, H, W, r) if T <= 4000 else None
+    text_cover = {}
+    for item in range(n_txt_items + n_img_items):
+        q_info, tiles = L.item_tiles(p, item)
+        assert (item < n_txt_items) == bool(q_info[0])
+        queries = _queries_of_item(q_info, n_text, H, W, T)
+        keys = [k for t in tiles for k in _keys_of_tile(t, n_text, H, W, T)]
+        assert len(keys) == len(set(keys)), "a key is visited twice by one item"
+        if q_info[0]:
+            text_cover.setdefault(q_info[2], []).extend(keys)
+            assert all(t[0] == 0 for t in tiles)
+            continue
+        rows = M[queries] if M is not None else oracle.clear_mask(n_text, H, W, r, rows=queries)
+        need = set(np.nonzero(rows.any(axis=0))[0].tolist())
+        assert need <= set(keys), "a kept pair is not covered"
+        for t in tiles:
+            slots = _raw_keys_of_tile(t, n_text, H, W)
+            real = [s for s in slots if s is not None]
+            assert real, "tile with no real key"
+            if t[0] == 1:
+                kept = rows[:, real]
+                assert kept.any(), "rectangle tile with no kept pair"
+                full = all(s is not None for s in slots) and kept.all()
+                assert bool(t[3]) == full, ("full flag wrong", t)
+            else:
+                assert bool(t[3]) == (t[2] == TILE)
+    # Text query tiles: splits of one tile cover every token exactly once.
+    for q0, keys in text_cover.items():
+        assert sorted(keys) == list(range(T))
+
+
+@pytest.mark.parametrize("n_text,H,W,r", CASES[:6])
+def test_pair_counts(n_text, H, W, r):
+    p = L.make_params(2, 3, n_text, H, W, 64, r)
+    useful, executed = L.pair_counts(p)
+    assert useful == 6 * oracle.kept_pairs(n_text, H, W, r)
+    assert executed >= useful
+    n_txt_items, n_img_items, S, cps = L.forward_shape(p)
+    tiles = sum(len(L.item_tiles(p, i)[1]) for i in range(n_txt_items + n_img_items))
+    assert executed == tiles * TILE * TILE
+
+
+def test_radius_beyond_diagonal_is_clamped_to_full_attention():
+    # r larger than the grid diagonal keeps every pair; the scheduler clamps it and visits every key.
+    p = L.make_params(1, 1, 16, 16, 16, 64, 1000)
+    useful, executed = L.pair_counts(p)
+    T = 16 + 256
+    assert useful == T * T
+
+
+def test_split_shape_at_8k():
+    p = L.make_params(1, 24, 512, 512, 512, 128, 8)
+    n_txt_items, n_img_items, S, cps = L.forward_shape(p)
+    assert n_img_items == 24 * (512 // 8) * (512 // 16)
+    assert S * cps >= (512 + 512 * 512 + 127) // 128 and S <= 32
+    assert n_txt_items == 24 * 4 * S
