@@ -1,0 +1,370 @@
+"""Benchmark of CLEAR attention on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 8k_r8] [--impl clear|reference]
+
+A step is one forward call (clear_attn_fwd: scheduler enumeration, image-row and text-row kernels,
+split combine) on the workload the metric is quoted on: B=1, 24 heads, d=128, 512 text tokens,
+512 x 512 image grid (8192^2 pixels), r=8, bf16 inputs. The backward (dQ/dK/dV) is measured in the
+same run on the distillation shape and reported under "bwd".
+
+value = useful (kept-pair) TFLOP/s over all ranks; each rank runs its own independent call (weak
+scaling, no collective on the data path). Inputs (4.8 GB) are far larger than L2.
+With --impl reference the float64 CPU oracle is timed instead, on sampled rows extrapolated to a
+full call.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from clear_inputs import WORKLOADS, Workload, make_inputs  # noqa: E402
+
+METRIC = "CLEAR attn useful TFLOP/s & ms/call (bf16, 512² grid, r=8); % of TC peak"
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), \
+            float(d.get("hbm_gbs", 0.0)), "measured"
+    return FALLBACK_BF16_TFLOPS, 1400.0, 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def _max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _flops(L, wl: Workload):
+    p = L.make_params(wl.B, wl.heads, wl.n_text, wl.H, wl.W, wl.d, wl.r)
+    useful, executed = L.pair_counts(p)
+    return 4.0 * wl.d * useful, 4.0 * wl.d * executed
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle timing (bounded sample, extrapolated to one call)
+# ------------------------------------------------------------------------------------------------
+_ORACLE_INPUTS = {}
+
+
+def oracle_call_seconds(wl: Workload, budget_s: float, seed: int = 0):
+    """Time the float64 oracle on sampled text and image query rows of one head and extrapolate to
+    a full call (B * heads heads, n_text text rows + H*W image rows each)."""
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    if wl.name not in _ORACLE_INPUTS:  # one head's inputs, drawn once (not timed)
+        _ORACLE_INPUTS[wl.name] = make_inputs(Workload(wl.name, 1, 1, wl.n_text, wl.H, wl.W, wl.d, wl.r), seed=0)
+    q, k, v = _ORACLE_INPUTS[wl.name]
+    rng = np.random.default_rng(seed)
+    per_kind = {}
+    for kind in ("text", "image"):
+        if kind == "text" and wl.n_text == 0:
+            per_kind[kind] = (0.0, 0)
+            continue
+        n_rows, spent = 0, 0.0
+        while spent < budget_s / 2 and n_rows < 4096:
+            if kind == "text":
+                rows = sorted(rng.choice(wl.n_text, size=min(4, wl.n_text), replace=False).tolist())
+            else:
+                rows = sorted((wl.n_text + rng.choice(wl.H * wl.W, size=8, replace=False)).tolist())
+            t0 = time.perf_counter()
+            oracle.clear_attention_rows(q, k, v, wl.n_text, wl.H, wl.W, wl.r, 0, 0, rows)
+            spent += time.perf_counter() - t0
+            n_rows += len(rows)
+        per_kind[kind] = (spent / max(1, n_rows), n_rows)
+    per_head = per_kind["text"][0] * wl.n_text + per_kind["image"][0] * wl.H * wl.W
+    total = per_head * wl.B * wl.heads
+    sample = (f"oracle rows of head 0: {per_kind['text'][1]} text + {per_kind['image'][1]} image rows "
+              f"({sum(v[0] * v[1] for v in per_kind.values()):.1f} s), extrapolated per row to "
+              f"{wl.B * wl.heads} heads x ({wl.n_text} text + {wl.H * wl.W} image) rows")
+    return total, cores, sample
+
+
+# ------------------------------------------------------------------------------------------------
+def run_reference(args):
+    world, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.config]
+    import oracle
+    useful = 4.0 * wl.d * wl.B * wl.heads * oracle.kept_pairs(wl.n_text, wl.H, wl.W, wl.r)
+    per_step_budget = max(0.5, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    times = []
+    for i in range(args.warmup + args.steps):
+        t, cores, sample = oracle_call_seconds(wl, per_step_budget, seed=i)
+        if i >= args.warmup:
+            times.append(t)
+    sec = statistics.mean(times)
+    value = useful / sec / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, **{k: getattr(wl, k) for k in ("B", "heads", "n_text", "H", "W", "d", "r")}},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample + f"; {args.steps} timed samples"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _time_calls(fn, steps, stream):
+    """CUDA-event time of each call on `stream`; returns per-call ms list and total ms."""
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    evs[0].record(stream)
+    for i in range(steps):
+        fn()
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize()
+    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(steps)]
+    return per, evs[0].elapsed_time(evs[-1])
+
+
+def run_clear(args):
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    import local_circular_window_b200 as L
+    wl = WORKLOADS[args.config]
+    peak, peak_sus, hbm, peak_kind = _peaks()
+    useful, executed = _flops(L, wl)
+    stream = torch.cuda.current_stream()
+
+    q, k, v = make_inputs(wl, seed=1000 + rank, device="cuda")
+    o = torch.empty_like(q)
+    lse = torch.empty((wl.B, wl.heads, wl.T), dtype=torch.float32, device="cuda")
+    p = L.make_params(wl.B, wl.heads, wl.n_text, wl.H, wl.W, wl.d, wl.r)
+    ws = torch.empty(max(16, L.fwd_workspace_size(p)), dtype=torch.uint8, device="cuda")
+
+    def call():
+        L.clear_attn_fwd(q, k, v, wl.n_text, wl.H, wl.W, wl.r, o=o, lse=lse, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        call()
+    if L.clear_attn_check() != 0:
+        raise RuntimeError("device error during warm-up")
+    torch.cuda.synchronize()
+    _barrier(world)
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        _barrier(world)
+        per, total_ms = _time_calls(call, args.steps, stream)
+        _barrier(world)
+    if L.clear_attn_check() != 0:
+        raise RuntimeError("device error during timing")
+    total_ms = _max_over_ranks(total_ms, world)
+    ms = total_ms / args.steps
+    value = useful * world / (ms * 1e-3) / 1e12
+    kernel_ms = statistics.mean(per)
+    achieved = useful / (kernel_ms * 1e-3) / 1e12
+
+    # End to end through the public API: pinned host inputs -> device, forward, outputs -> host.
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        dq_, dk_, dv_ = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+        def e2e_call():
+            dq_.copy_(hq, non_blocking=True)
+            dk_.copy_(hk, non_blocking=True)
+            dv_.copy_(hv, non_blocking=True)
+            L.clear_attn_fwd(dq_, dk_, dv_, wl.n_text, wl.H, wl.W, wl.r, o=o, lse=lse, workspace=ws, stream=stream)
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        e2e_call()
+        torch.cuda.synchronize()
+        k_e2e = max(1, min(args.steps, 5))
+        _barrier(world)
+        _, e2e_ms = _time_calls(e2e_call, k_e2e, stream)
+        e2e_ms = _max_over_ranks(e2e_ms, world) / k_e2e
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+        d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+        e2e = {"value": useful * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+               "steps": k_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        del hq, hk, hv, ho, hl, dq_, dk_, dv_
+    del q, k, v, o, lse, ws
+    torch.cuda.empty_cache()
+
+    # Backward rows of the hot path, on the distillation shape.
+    bwd = None
+    if not args.no_bwd:
+        bwl = WORKLOADS["bwd_flux1024_r32"]
+        bq, bk, bv, bdo = make_inputs(bwl, seed=2000 + rank, device="cuda", with_grad_out=True)
+        bo, blse = L.clear_attn_fwd(bq, bk, bv, bwl.n_text, bwl.H, bwl.W, bwl.r)
+        bp = L.make_params(bwl.B, bwl.heads, bwl.n_text, bwl.H, bwl.W, bwl.d, bwl.r)
+        bws = torch.empty(L.bwd_workspace_size(bp), dtype=torch.uint8, device="cuda")
+        gq, gk, gv = torch.empty_like(bq), torch.empty_like(bk), torch.empty_like(bv)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+        def bcall():
+            flush.zero_()  # the 280 MB working set is near L2 size: flush L2 between calls
+            L.clear_attn_bwd(bq, bk, bv, bo, blse, bdo, bwl.n_text, bwl.H, bwl.W, bwl.r, dq=gq, dk=gk, dv=gv,
+                             workspace=bws, stream=stream)
+
+        def flush_only():
+            flush.zero_()
+
+        for _ in range(3):
+            bcall()
+        torch.cuda.synchronize()
+        nb = max(3, min(args.steps, 20))
+        per_b, _ = _time_calls(bcall, nb, stream)
+        per_f, _ = _time_calls(flush_only, nb, stream)
+        bms = max(1e-6, statistics.median(per_b) - statistics.median(per_f))
+        bu, be = _flops(L, bwl)
+        if L.clear_attn_check() != 0:
+            raise RuntimeError("device error in backward timing")
+        bwd = {"workload": bwl.name, "ms_per_call": bms, "useful_tflops": 2.5 * bu / (bms * 1e-3) / 1e12,
+               "flop_convention": "backward = 2.5 x forward useful FLOPs (5 vs 2 matmuls)",
+               "l2": "flushed between calls (256 MiB write, its time subtracted)"}
+        del bq, bk, bv, bdo, bo, blse, bws, gq, gk, gv, flush
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sec, cores, sample = oracle_call_seconds(wl, args.cpu_budget)
+        cpu = {"value": useful / sec / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": sample}
+
+    clocks = clk.summary()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "heads": wl.heads, "n_text": wl.n_text, "H": wl.H,
+                       "W": wl.W, "d": wl.d, "r": wl.r, "T": wl.T,
+                       "l2": "inputs (3 x %.2f GB) larger than L2" % (q_bytes(wl) / 1e9),
+                       "parallelism": f"independent call per GPU x{world}"},
+            "pct_of_tc_peak": 100.0 * achieved / peak,
+            "padded_tflops": executed / (kernel_ms * 1e-3) / 1e12,
+            "useful_gflop_per_call": useful / 1e9, "executed_gflop_per_call": executed / 1e9,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_source": f"{peak_kind} bf16 dense (burst; kernel timed alone)",
+                         "kernel": "clear_fwd_kernel + clear_fwd_combine_kernel (one call, CUDA events)"},
+            "e2e": e2e, "cpu_baseline": cpu, "bwd": bwd, "clocks": clocks,
+            "gpu_launches": 2 * args.steps,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def q_bytes(wl):
+    return wl.B * wl.heads * wl.T * wl.d * 2
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="clear", choices=["clear", "reference"])
+    ap.add_argument("--config", default="8k_r8", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-bwd", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU work for cpu_baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_clear(args)
+
+
+if __name__ == "__main__":
+    main()
