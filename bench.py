@@ -213,6 +213,8 @@ def run_clear(args):
     torch.cuda.set_device(local)
     import local_circular_window_b200 as L
     wl = WORKLOADS[args.config]
+    if args.heads:  # sized-down copy of the same shape (profiling captures only)
+        wl = Workload(f"{wl.name}_h{args.heads}", wl.B, args.heads, wl.n_text, wl.H, wl.W, wl.d, wl.r)
     peak, peak_sus, hbm, peak_kind = _peaks()
     useful, executed = _flops(L, wl)
     stream = torch.cuda.current_stream()
@@ -353,6 +355,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="clear", choices=["clear", "reference"])
     ap.add_argument("--config", default="8k_r8", choices=sorted(WORKLOADS))
+    ap.add_argument("--heads", type=int, default=0, help="override the head count (sized-down profiling runs)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -116,24 +116,27 @@ CLEAR_API clear_status_t clear_attn_check(void* stream);
  * so its coverage can be checked against a brute-force mask on the CPU.
  * --------------------------------------------------------------------------------------------- */
 
-/* Work-list shape of the forward: numbers of text (split) items and image items, the text split
- * count S and 128-key chunks per split. Any output pointer may be NULL. */
+/* Work-list shape of the forward. The forward works on pairs of 128-row query tiles that share
+ * their key tiles: pairs of consecutive text tiles (split over key ranges) and 16 x 16 image
+ * blocks (upper and lower 8 x 16 halves). Returns the numbers of text pairs (all splits) and image
+ * pairs, the text split count S and the 128-key chunks per split. Any output may be NULL. */
 CLEAR_API clear_status_t clear_sched_forward_shape(const clear_attn_params_t* params, long long* n_text_items,
                                          long long* n_image_items, int* splits,
                                          int* chunks_per_split);
 
-/* Key tiles visited by forward work item `item` (0 <= item < n_text_items + n_image_items), in
- * order. Each tile is 4 ints: kind (0 = linear chunk, 1 = image rectangle), a, b, flags
- * (1 = every pair kept, no mask needed). Linear: tokens [a, a + 128), first b of them real.
- * Rectangle: grid rows [a, a + 8) x columns [b, b + 16). Also returns the item's query tile:
- * q_info = {is_text, bh, q0 (first token, or first grid row), x0 (first grid column)}.
- * Writes at most max_tiles tiles; returns the item's total tile count via *n_tiles. */
+/* Union key tiles visited by forward pair `item` (0 <= item < n_text_items + n_image_items), in
+ * order. Each tile is 4 ints: kind (0 = linear chunk, 1 = image rectangle), a, b, flags.
+ * Linear: tokens [a, a + 128), first b of them real. Rectangle: grid rows [a, a + 8) x columns
+ * [b, b + 16). flags: bit 0 / bit 1 = half A / half B needs the tile (some kept pair), bit 2 /
+ * bit 3 = every pair of half A / half B with the tile is kept (no mask). q_info = {is_text, bh,
+ * q0 (first token of half A, or first grid row of the block), x0 (first grid column), half B
+ * holds real queries}. Writes at most max_tiles tiles; the total count goes to *n_tiles. */
 CLEAR_API clear_status_t clear_sched_item_tiles(const clear_attn_params_t* params, long long item,
                                       int* q_info, int* tiles, int max_tiles, int* n_tiles);
 
 /* Useful (kept-pair) and executed (padded-tile) multiply-add pair counts of one forward call,
- * summed over B and heads: useful = number of ones in the mask; executed = 128 x 128 per visited
- * tile pair. FLOPs are 4 * d times these. */
+ * summed over B and heads: useful = number of ones in the mask; executed = 128 x 128 per tile
+ * product the forward issues (a half times a key tile it needs). FLOPs are 4 * d times these. */
 CLEAR_API clear_status_t clear_sched_pair_counts(const clear_attn_params_t* params, long long* useful_pairs,
                                        long long* executed_pairs);
 

@@ -115,7 +115,7 @@ def forward_shape(p: ClearParams):
 
 def item_tiles(p: ClearParams, item: int):
     """(q_info, tiles) of one forward work item; tiles is a list of (kind, a, b, flags)."""
-    q = (_i * 4)()
+    q = (_i * 5)()
     n = _i(0)
     st = _lib.clear_sched_item_tiles(ctypes.byref(p), item, q, None, 0, ctypes.byref(n))
     if st != CLEAR_OK:

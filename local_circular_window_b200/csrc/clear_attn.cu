@@ -52,6 +52,10 @@ Checked check_params(const clear_attn_params_t* p) {
   if (N > (1ll << 28) || p->n_text > (1 << 24) || T > (1ll << 30) || BH > (1ll << 20)) return c;
   if (BH * T * p->d >= (1ll << 40)) return c;
   const int r = p->r < full_radius(p->H, p->W) ? p->r : full_radius(p->H, p->W);
+  if (hw_table_size(r, p->H) > kMaxHwTable) {  // half-width table must fit in shared memory
+    c.st = CLEAR_ERR_UNSUPPORTED;
+    return c;
+  }
   c.g = make_geom(p->B, p->heads, p->n_text, p->H, p->W, p->d, r);
   c.st = CLEAR_OK;
   return c;
@@ -150,6 +154,8 @@ template <int D>
 clear_status_t launch_fwd(const Geom& g, const QKVMaps& m, void* o, float* lse, void* ws,
                           int num_sms, cudaStream_t stream) {
   using L = FwdLayout<D>;
+  const int smem_bytes = L::alloc_bytes(hw_table_size(g.r, g.H));
+  if (smem_bytes > 232448) return CLEAR_ERR_UNSUPPORTED;  // guarded by check_params
   FwdParams p{};
   p.g = g;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
@@ -158,12 +164,12 @@ clear_status_t launch_fwd(const Geom& g, const QKVMaps& m, void* o, float* lse, 
   const FwdWorkspace wl = fwd_workspace_layout(g);
   p.opart = g.n_text ? reinterpret_cast<float*>(static_cast<char*>(ws) + wl.opart_off) : nullptr;
   p.ml = g.n_text ? reinterpret_cast<float2*>(static_cast<char*>(ws) + wl.ml_off) : nullptr;
-  p.n_work = g.n_txt_items + g.n_img_items;
+  p.n_work = g.n_txt_pairs + g.n_img_pairs;
   if (cudaFuncSetAttribute(clear_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           L::kAlloc) != cudaSuccess)
+                           smem_bytes) != cudaSuccess)
     return CLEAR_ERR_CUDA;
   const long long grid = p.n_work < num_sms ? p.n_work : num_sms;
-  clear_fwd_kernel<D><<<(unsigned)grid, kFwdThreads, L::kAlloc, stream>>>(
+  clear_fwd_kernel<D><<<(unsigned)grid, kFwdThreads, smem_bytes, stream>>>(
       m.q_lin, m.q_img, m.k_lin, m.k_img, m.v_lin, m.v_img, p);
   if (cudaGetLastError() != cudaSuccess) return CLEAR_ERR_CUDA;
   if (g.n_text > 0) {
@@ -282,8 +288,8 @@ clear_status_t clear_sched_forward_shape(const clear_attn_params_t* params, long
                                          int* chunks_per_split) {
   const Checked c = check_params(params);
   if (c.st != CLEAR_OK) return c.st;
-  if (n_text_items) *n_text_items = c.g.n_txt_items;
-  if (n_image_items) *n_image_items = c.g.n_img_items;
+  if (n_text_items) *n_text_items = c.g.n_txt_pairs;
+  if (n_image_items) *n_image_items = c.g.n_img_pairs;
   if (splits) *splits = c.g.S;
   if (chunks_per_split) *chunks_per_split = c.g.cps;
   return CLEAR_OK;
@@ -293,15 +299,16 @@ clear_status_t clear_sched_item_tiles(const clear_attn_params_t* params, long lo
                                       int* tiles, int max_tiles, int* n_tiles) {
   const Checked c = check_params(params);
   if (c.st != CLEAR_OK) return c.st;
-  if (item < 0 || item >= c.g.n_txt_items + c.g.n_img_items || max_tiles < 0) return CLEAR_ERR_INVALID_ARG;
-  const WorkItem it = decode_work(c.g, item);
+  if (item < 0 || item >= c.g.n_txt_pairs + c.g.n_img_pairs || max_tiles < 0) return CLEAR_ERR_INVALID_ARG;
+  const PairItem it = decode_pair(c.g, item);
   if (q_info) {
     q_info[0] = it.is_text;
     q_info[1] = it.bh;
     q_info[2] = it.q0;
     q_info[3] = it.x0;
+    q_info[4] = it.validB;
   }
-  KeyIter ki;
+  PairKeyIter ki;
   ki.init(c.g, it);
   KeyTile t;
   int n = 0;
@@ -339,13 +346,21 @@ clear_status_t clear_sched_pair_counts(const clear_attn_params_t* params, long l
   const long long per_head = (long long)g.n_text * g.T + N * g.n_text + win;
   if (useful_pairs) *useful_pairs = per_head * g.BH;
   if (executed_pairs) {
+    // Tile products actually issued by the forward: each half of a pair multiplies the union key
+    // tiles it needs (image blocks of one (b, h), then the text tile pairs over all splits).
     long long tiles = 0;
-    WorkItem it{};
-    for (int qt = 0; qt < g.nQ; ++qt) {  // image items of one (b, h)
-      it = decode_work(g, g.n_txt_items + qt);
-      tiles += count_key_tiles(g, it);
+    for (int blk = 0; blk < g.nQ2; ++blk) {
+      const PairItem it = decode_pair(g, g.n_txt_pairs + blk);
+      int nu, na, nb;
+      count_pair_tiles(g, it, nullptr, 0, &nu, &na, &nb);
+      tiles += na + nb;
     }
-    tiles += (long long)g.nTq * g.nC;  // text rows: every chunk once per text query tile
+    for (long long w = 0; w < (long long)g.nTq2 * g.S; ++w) {
+      const PairItem it = decode_pair(g, w);
+      int nu, na, nb;
+      count_pair_tiles(g, it, nullptr, 0, &nu, &na, &nb);
+      tiles += na + nb;
+    }
     *executed_pairs = tiles * (long long)kTile * kTile * g.BH;
   }
   return CLEAR_OK;

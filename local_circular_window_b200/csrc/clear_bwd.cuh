@@ -21,7 +21,7 @@
 #pragma once
 #include <cuda_bf16.h>
 
-#include "clear_fwd.cuh"
+#include "clear_common.cuh"
 #include "clear_sched.cuh"
 #include "sm100_ptx.cuh"
 

@@ -63,6 +63,11 @@ struct Geom {
   int S;             // splits of a text query tile's key range
   int cps;           // chunks per split
   long long n_txt_items, n_img_items;
+  // Forward pairs: two query tiles share every key tile they visit (a 16 x 16 image block, or
+  // two consecutive 128-row text tiles).
+  int nqy2, nQ2;     // image blocks per (b, h): ceil(H/16) x ceil(W/16)
+  int nTq2;          // text tile pairs: ceil(nTq / 2)
+  long long n_txt_pairs, n_img_pairs;
 };
 
 CLEAR_HD int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -113,6 +118,11 @@ CLEAR_HD Geom make_geom(int B, int heads, int n_text, int H, int W, int d, int r
   choose_splits(g.nC, kSplitTargetChunks, kMaxSplits, &g.S, &g.cps);
   g.n_txt_items = (long long)g.BH * g.nTq * g.S;
   g.n_img_items = (long long)g.BH * g.nQ;
+  g.nqy2 = cdiv(H, 2 * kQH);
+  g.nQ2 = g.nqy2 * g.nqx;
+  g.nTq2 = cdiv(g.nTq, 2);
+  g.n_txt_pairs = (long long)g.BH * g.nTq2 * g.S;
+  g.n_img_pairs = (long long)g.BH * g.nQ2;
   return g;
 }
 
@@ -157,6 +167,8 @@ CLEAR_HD WorkItem decode_work(const Geom& g, long long w) {
 // Enumerates the key tiles of one work item, in visiting order.
 struct KeyIter {
   // fixed per item
+  const int* wtab;        // optional half-width table (device shared memory), entries [0, wtab_n)
+  int wtab_n;
   int is_text, r, H, W, n_text, T;
   int y0, yl, x0, xl;     // image query tile, clipped to the grid (rows y0..yl, cols x0..xl)
   int ky_begin, ky_end;   // key rows that any query of the tile can reach
@@ -165,7 +177,9 @@ struct KeyIter {
   int band_ky;            // current band's first key row
   int kx, kx_end;         // next rectangle column and the band's last needed column
 
-  CLEAR_HD void init(const Geom& g, const WorkItem& it) {
+  CLEAR_HD void init(const Geom& g, const WorkItem& it, const int* table = nullptr, int table_n = 0) {
+    wtab = table;
+    wtab_n = table_n;
     is_text = it.is_text; r = g.r; H = g.H; W = g.W; n_text = g.n_text; T = g.T;
     if (is_text) {
       lin_next = it.c_begin;
@@ -193,7 +207,7 @@ struct KeyIter {
       if (band_ky > ky_end) return false;
       int band_last = imin(band_ky + kKH - 1, H - 1);
       int dmin = imax(0, imax(y0 - band_last, band_ky - yl));
-      int w = half_width(r, dmin);
+      int w = (dmin < wtab_n) ? wtab[dmin] : half_width(r, dmin);
       if (w < 0) continue;
       kx = imax(0, x0 - w);
       kx_end = imin(W - 1, xl + w);
@@ -230,13 +244,169 @@ struct KeyIter {
 };
 
 // Number of key tiles an item visits (host-side cost estimates and tests).
-CLEAR_HD int count_key_tiles(const Geom& g, const WorkItem& it) {
+CLEAR_HD int count_key_tiles(const Geom& g, const WorkItem& it, const int* table = nullptr, int table_n = 0) {
   KeyIter ki;
-  ki.init(g, it);
+  ki.init(g, it, table, table_n);
   KeyTile t;
   int n = 0;
   while (ki.next(&t)) ++n;
   return n;
+}
+
+// ------------------------------------------------------------------------------------------------
+// Pair work items for the forward: half A and half B of a pair share the key tiles.
+// ------------------------------------------------------------------------------------------------
+enum PairFlags : int { kNeedA = 1, kNeedB = 2, kFullA = 4, kFullB = 8 };
+
+struct PairItem {
+  int is_text;
+  int bh;
+  int q0;        // text: first token of half A (half B starts 128 later); image: block row y0
+  int x0;        // image: block column x0
+  int validB;    // half B holds at least one real query row
+  int split, c_begin, c_end;  // text: split index and linear chunk range
+};
+
+CLEAR_HD PairItem decode_pair(const Geom& g, long long w) {
+  PairItem it;
+  if (w < g.n_txt_pairs) {
+    int s = (int)(w % g.S);
+    long long t = w / g.S;
+    int qp = (int)(t % g.nTq2);
+    it.is_text = 1;
+    it.bh = (int)(t / g.nTq2);
+    it.q0 = qp * 2 * kTile;
+    it.x0 = 0;
+    it.validB = (it.q0 + kTile) < g.n_text;
+    it.split = s;
+    it.c_begin = s * g.cps;
+    it.c_end = imin(g.nC, (s + 1) * g.cps);
+  } else {
+    long long u = w - g.n_txt_pairs;
+    int blk = (int)(u % g.nQ2);
+    it.is_text = 0;
+    it.bh = (int)(u / g.nQ2);
+    it.q0 = (blk / g.nqx) * (2 * kQH);
+    it.x0 = (blk % g.nqx) * kQW;
+    it.validB = (it.q0 + kQH) < g.H;
+    it.split = 0;
+    it.c_begin = 0;
+    it.c_end = 0;
+  }
+  return it;
+}
+
+// Union key tiles of a pair, with per-half need / full flags. Image blocks visit the text chunks,
+// then band by band the 16-column rectangles covering the union of both halves' windows; a
+// rectangle is needed by a half iff some (query of that half, key of the rectangle) pair is kept.
+struct PairKeyIter {
+  const int* wtab;
+  int wtab_n;
+  int is_text, r, H, W, n_text, T, validB;
+  int y0, x0, xl;             // block origin, last column
+  int yA0, yAl, yB0, yBl;     // half rows (clipped); B rows only if validB
+  int ky_begin, ky_end;
+  int lin_next, lin_end;
+  int band_ky, kx, kx_end;
+
+  CLEAR_HD void init(const Geom& g, const PairItem& it, const int* table = nullptr, int table_n = 0) {
+    wtab = table;
+    wtab_n = table_n;
+    is_text = it.is_text; r = g.r; H = g.H; W = g.W; n_text = g.n_text; T = g.T; validB = it.validB;
+    if (is_text) {
+      lin_next = it.c_begin;
+      lin_end = it.c_end;
+      band_ky = 1; ky_end = 0; kx = 1; kx_end = 0;
+      y0 = x0 = xl = yA0 = yAl = yB0 = yBl = 0; ky_begin = 0;
+      return;
+    }
+    lin_next = 0;
+    lin_end = g.nTk;
+    y0 = it.q0; x0 = it.x0;
+    xl = imin(x0 + kQW - 1, W - 1);
+    yA0 = y0; yAl = imin(y0 + kQH - 1, H - 1);
+    yB0 = y0 + kQH; yBl = imin(y0 + 2 * kQH - 1, H - 1);
+    const int ylast = validB ? yBl : yAl;
+    ky_begin = imax(0, y0 - (r - 1));
+    ky_end = imin(H - 1, ylast + (r - 1));
+    band_ky = ky_begin - kKH;
+    kx = 1; kx_end = 0;
+  }
+
+  CLEAR_HD int hw(int dy) const { return (dy < wtab_n) ? wtab[dy] : half_width(r, dy); }
+
+  CLEAR_HD bool advance_band() {
+    const int ylast = validB ? yBl : yAl;
+    while (true) {
+      band_ky += kKH;
+      if (band_ky > ky_end) return false;
+      const int band_last = imin(band_ky + kKH - 1, H - 1);
+      const int dmin = imax(0, imax(y0 - band_last, band_ky - ylast));
+      const int w = hw(dmin);
+      if (w < 0) continue;
+      kx = imax(0, x0 - w);
+      kx_end = imin(W - 1, xl + w);
+      if (kx <= kx_end) return true;
+    }
+  }
+
+  // need / full of rectangle [ky, ky+8) x [kx, kx+16) for query rows [qa, qb], columns [x0, xl].
+  CLEAR_HD int half_flags(int ky, int kxx, int qa, int qb, int need_bit, int full_bit) const {
+    const int kyl = imin(ky + kKH - 1, H - 1);
+    const int kxl = imin(kxx + kKW - 1, W - 1);
+    const int dy = imax(0, imax(qa - kyl, ky - qb));
+    const int dx = imax(0, imax(x0 - kxl, kxx - xl));
+    if (dy * dy + dx * dx >= r * r) return 0;
+    const bool inside = (ky + kKH - 1 <= H - 1) && (kxx + kKW - 1 <= W - 1);
+    const int mdy = imax(ky + kKH - 1 - qa, qb - ky);
+    const int mdx = imax(kxx + kKW - 1 - x0, xl - kxx);
+    return need_bit | ((inside && mdy * mdy + mdx * mdx < r * r) ? full_bit : 0);
+  }
+
+  CLEAR_HD bool next(KeyTile* t) {
+    if (lin_next < lin_end) {
+      const int a = lin_next * kTile;
+      const int lim = is_text ? T : n_text;
+      t->kind = kLinear;
+      t->a = a;
+      t->b = imin(kTile, lim - a);
+      const int full = (t->b == kTile);
+      t->flags = kNeedA | (full ? kFullA : 0) | (validB ? (kNeedB | (full ? kFullB : 0)) : 0);
+      ++lin_next;
+      return true;
+    }
+    if (is_text) return false;
+    while (true) {
+      if (kx > kx_end) {
+        if (!advance_band()) return false;
+      }
+      const int f = half_flags(band_ky, kx, yA0, yAl, kNeedA, kFullA) |
+                    (validB ? half_flags(band_ky, kx, yB0, yBl, kNeedB, kFullB) : 0);
+      t->kind = kRect;
+      t->a = band_ky;
+      t->b = kx;
+      t->flags = f;
+      kx += kKW;
+      if (f & (kNeedA | kNeedB)) return true;  // rectangles neither half reaches are skipped
+    }
+  }
+};
+
+// Needed tiles of one half (half = 0: A, 1: B) in a pair, and the union tile count.
+CLEAR_HD void count_pair_tiles(const Geom& g, const PairItem& it, const int* table, int table_n, int* n_union,
+                               int* n_a, int* n_b) {
+  PairKeyIter ki;
+  ki.init(g, it, table, table_n);
+  KeyTile t;
+  int nu = 0, na = 0, nb = 0;
+  while (ki.next(&t)) {
+    ++nu;
+    na += (t.flags & kNeedA) ? 1 : 0;
+    nb += (t.flags & kNeedB) ? 1 : 0;
+  }
+  *n_union = nu;
+  *n_a = na;
+  *n_b = nb;
 }
 
 }  // namespace clear

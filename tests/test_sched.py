@@ -36,15 +36,21 @@ def _raw_keys_of_tile(tile, n_text, H, W):
     return out
 
 
-def _queries_of_item(q_info, n_text, H, W, T):
-    is_text, bh, q0, x0 = q_info
+def _queries_of_half(q_info, half, n_text, H, W):
+    is_text, bh, q0, x0, valid_b = q_info
+    if half == 1 and not valid_b:
+        return []
     if is_text:
-        return [t for t in range(q0, q0 + TILE) if t < n_text]
-    return [n_text + y * W + x for y in range(q0, q0 + KQH) for x in range(x0, x0 + KQW) if y < H and x < W]
+        start = q0 + half * TILE
+        return [t for t in range(start, start + TILE) if t < n_text]
+    y0 = q0 + half * KQH
+    return [n_text + y * W + x for y in range(y0, y0 + KQH) for x in range(x0, x0 + KQW) if y < H and x < W]
 
 
 CASES = [(16, 16, 16, 4), (0, 19, 21, 3), (5, 24, 40, 5), (3, 9, 17, 1), (200, 13, 50, 7), (1, 8, 8, 30),
-         (0, 33, 47, 9), (7, 70, 18, 12), (130, 96, 96, 6)]
+         (0, 33, 47, 9), (7, 70, 18, 12), (130, 96, 96, 6), (300, 20, 20, 3)]
+NEED = (1, 2)
+FULL = (4, 8)
 
 
 @pytest.mark.parametrize("n_text,H,W,r", CASES)
@@ -57,28 +63,32 @@ def test_tiles_cover_mask_exactly(n_text, H, W, r):
     for item in range(n_txt_items + n_img_items):
         q_info, tiles = L.item_tiles(p, item)
         assert (item < n_txt_items) == bool(q_info[0])
-        queries = _queries_of_item(q_info, n_text, H, W, T)
         keys = [k for t in tiles for k in _keys_of_tile(t, n_text, H, W, T)]
-        assert len(keys) == len(set(keys)), "a key is visited twice by one item"
+        assert len(keys) == len(set(keys)), "a key is visited twice by one pair"
+        for t in tiles:
+            assert t[3] & 3, "union tile that neither half needs"
         if q_info[0]:
             text_cover.setdefault(q_info[2], []).extend(keys)
             assert all(t[0] == 0 for t in tiles)
-            continue
-        rows = M[queries] if M is not None else oracle.clear_mask(n_text, H, W, r, rows=queries)
-        need = set(np.nonzero(rows.any(axis=0))[0].tolist())
-        assert need <= set(keys), "a kept pair is not covered"
-        for t in tiles:
-            slots = _raw_keys_of_tile(t, n_text, H, W)
-            real = [s for s in slots if s is not None]
-            assert real, "tile with no real key"
-            if t[0] == 1:
+        for half in (0, 1):
+            queries = _queries_of_half(q_info, half, n_text, H, W)
+            if not queries:
+                assert not any(t[3] & NEED[half] for t in tiles)
+                continue
+            rows = M[queries] if M is not None else oracle.clear_mask(n_text, H, W, r, rows=queries)
+            need = set(np.nonzero(rows.any(axis=0))[0].tolist())
+            covered = set(k for t in tiles if t[3] & NEED[half] for k in _keys_of_tile(t, n_text, H, W, T))
+            if not q_info[0]:  # a text split covers its own key range only (checked across splits below)
+                assert need <= covered, "a kept pair of this half is not covered"
+            for t in tiles:
+                slots = _raw_keys_of_tile(t, n_text, H, W)
+                real = [s_ for s_ in slots if s_ is not None]
                 kept = rows[:, real]
-                assert kept.any(), "rectangle tile with no kept pair"
-                full = all(s is not None for s in slots) and kept.all()
-                assert bool(t[3]) == full, ("full flag wrong", t)
-            else:
-                assert bool(t[3]) == (t[2] == TILE)
-    # Text query tiles: splits of one tile cover every token exactly once.
+                assert bool(t[3] & NEED[half]) == bool(kept.any()), ("need flag wrong", half, t)
+                full = all(s_ is not None for s_ in slots) and kept.all()
+                if t[3] & NEED[half]:
+                    assert bool(t[3] & FULL[half]) == full, ("full flag wrong", half, t)
+    # Text query pairs: the splits of one pair cover every token exactly once.
     for q0, keys in text_cover.items():
         assert sorted(keys) == list(range(T))
 
@@ -90,8 +100,10 @@ def test_pair_counts(n_text, H, W, r):
     assert useful == 6 * oracle.kept_pairs(n_text, H, W, r)
     assert executed >= useful
     n_txt_items, n_img_items, S, cps = L.forward_shape(p)
-    tiles = sum(len(L.item_tiles(p, i)[1]) for i in range(n_txt_items + n_img_items))
-    assert executed == tiles * TILE * TILE
+    products = 0
+    for i in range(n_txt_items + n_img_items):
+        products += sum(((t[3] & 1) != 0) + ((t[3] & 2) != 0) for t in L.item_tiles(p, i)[1])
+    assert executed == products * TILE * TILE
 
 
 def test_radius_beyond_diagonal_is_clamped_to_full_attention():
@@ -105,6 +117,6 @@ def test_radius_beyond_diagonal_is_clamped_to_full_attention():
 def test_split_shape_at_8k():
     p = L.make_params(1, 24, 512, 512, 512, 128, 8)
     n_txt_items, n_img_items, S, cps = L.forward_shape(p)
-    assert n_img_items == 24 * (512 // 8) * (512 // 16)
+    assert n_img_items == 24 * (512 // 16) * (512 // 16)
     assert S * cps >= (512 + 512 * 512 + 127) // 128 and S <= 32
-    assert n_txt_items == 24 * 4 * S
+    assert n_txt_items == 24 * 2 * S
