@@ -42,6 +42,7 @@ constexpr uint32_t kRegsLow = 72;
 constexpr uint32_t kRegsHigh = 216;
 static_assert(2 * 128 * kRegsHigh + 128 * kRegsLow <= 384 * 168, "register split exceeds the launch allocation");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kLastTile = 16;              // mailbox flag: last needed tile of the half in this pair
 
 struct FwdParams {
   Geom g;
@@ -69,8 +70,10 @@ struct FwdLayout {
   static constexpr int bSFull = bVEmpty + kVStages;      // + half
   static constexpr int bPFull = bSFull + 2;              // + half
   static constexpr int bODone = bPFull + 2;              // + half
-  static constexpr int kNumBars = bODone + 2;
-  static constexpr int kMisc = kBars + kNumBars * 8;
+  static constexpr int bInfo = bODone + 2;               // + half: tile descriptor mailbox full
+  static constexpr int kNumBars = bInfo + 2;
+  static constexpr int kInfo = kBars + kNumBars * 8;     // int4[2]: {kind, a, b, flags | kLastTile}
+  static constexpr int kMisc = kInfo + 32;
   static constexpr int kWTab = kMisc + 16;               // int[kMaxRTable] (tile enumeration)
   static constexpr int kHwTab = kWTab + kMaxRTable * 4;  // int16[hw_table_size(r, H)] (masks)
   static constexpr int kFixed = kHwTab + 1024;           // + slack for 1024-byte alignment
@@ -94,6 +97,7 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   int* wtab = reinterpret_cast<int*>(smem + L::kWTab);
   int16_t* hwtab = reinterpret_cast<int16_t*>(smem + L::kHwTab);
+  int4* info = reinterpret_cast<int4*>(smem + L::kInfo);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -114,6 +118,7 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
       mbar_init(&bars[L::bSFull + h], 1);
       mbar_init(&bars[L::bPFull + h], 128);
       mbar_init(&bars[L::bODone + h], 1);
+      mbar_init(&bars[L::bInfo + h], 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -241,6 +246,10 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
             mbar_arrive(&bars[L::bVEmpty + vs]);
             continue;
           }
+          // Hand the tile to this half's softmax (its previous descriptor was consumed before it
+          // signalled the previous P, which this thread has waited for).
+          info[h] = make_int4(t.kind, t.a, t.b, t.flags | (j == n - 1 ? kLastTile : 0));
+          mbar_arrive(&bars[L::bInfo + h]);
           if (j == 0 && !mbar_wait(&bars[L::bQFull], items & 1, abort_flag, kDevTimeoutMma)) goto mma_done;
           if (!mbar_wait(&bars[L::bKFull + ks], kph, abort_flag, kDevTimeoutMma)) goto mma_done;
           tc_fence_after();
@@ -282,7 +291,6 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t s_tm = tmem + lane_base + L::s_col(half);
     const uint32_t o_tm = tmem + lane_base + L::o_col(half);
-    const int need_bit = half == 0 ? kNeedA : kNeedB;
     const int full_bit = half == 0 ? kFullA : kFullB;
     uint32_t nq = 0, n_out = 0;
     const float sl2 = p.scale_log2;
@@ -301,12 +309,17 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
       }
       float m_used = -INFINITY;  // running max, scaled log2 units
       float l = 0.f;
-      PairKeyIter ki;
-      ki.init(g, it, wtab, wtn);
-      KeyTile t;
       int j = 0;
-      while (ki.next(&t)) {
-        if (!(t.flags & need_bit)) continue;
+      bool last = false;
+      while (!last) {
+        if (!mbar_wait(&bars[L::bInfo + half], nq & 1, abort_flag, kDevTimeoutSoftmax)) goto softmax_done;
+        const int4 ti = info[half];
+        KeyTile t;
+        t.kind = ti.x;
+        t.a = ti.y;
+        t.b = ti.z;
+        t.flags = ti.w;
+        last = (ti.w & kLastTile) != 0;
         if (!mbar_wait(&bars[L::bSFull + half], nq & 1, abort_flag, kDevTimeoutSoftmax)) goto softmax_done;
         tc_fence_after();
         float s[kTile];
@@ -327,20 +340,19 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
             #pragma unroll
             for (int c = 0; c < kTile; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
           } else {
-            int lo[kKH];
-            unsigned span[kKH];
+            // keep bits: word q holds key rows 2q (bits 0-15) and 2q+1 (bits 16-31)
+            uint32_t keep[kKH / 2];
             #pragma unroll
-            for (int kr = 0; kr < kKH; ++kr) {
-              int hi;
-              row_range_tab(g, hwtab, hwn, yq, xq, t.a + kr, t.b, &lo[kr], &hi);
-              span[kr] = (unsigned)(hi - lo[kr]);
+            for (int q = 0; q < kKH / 2; ++q) {
+              int lo0, hi0, lo1, hi1;
+              row_range_tab(g, hwtab, hwn, yq, xq, t.a + 2 * q, t.b, &lo0, &hi0);
+              row_range_tab(g, hwtab, hwn, yq, xq, t.a + 2 * q + 1, t.b, &lo1, &hi1);
+              const int n0 = imax(hi0 - lo0 + 1, 0), n1 = imax(hi1 - lo1 + 1, 0);
+              keep[q] = (((1u << n0) - 1u) << (lo0 & 15)) | ((((1u << n1) - 1u) << (lo1 & 15)) << 16);
             }
             #pragma unroll
-            for (int kr = 0; kr < kKH; ++kr) {
-              #pragma unroll
-              for (int c = 0; c < kKW; ++c)
-                s[kr * kKW + c] = ((unsigned)(c - lo[kr]) <= span[kr]) ? s[kr * kKW + c] : -INFINITY;
-            }
+            for (int c = 0; c < kTile; ++c)
+              s[c] = (keep[c >> 5] & (1u << (c & 31))) ? s[c] : -INFINITY;
           }
         }
         // ---- tile max (8 independent chains of 3-input maxima)
