@@ -111,22 +111,28 @@ CLEAR_API clear_status_t clear_attn_bwd(const clear_attn_params_t* params, const
  * invalid) or CLEAR_ERR_CUDA (the stream reported a CUDA error). */
 CLEAR_API clear_status_t clear_attn_check(void* stream);
 
+/* Context of the expired wait behind the last CLEAR_ERR_DEVICE_TIMEOUT that clear_attn_check()
+ * returned on this host thread (zeros if none): {code (1 producer, 3 MMA, 4 softmax), wait site,
+ * CTA index, thread index, phase parity (-1 for a polling loop), three site-specific counters}.
+ * For diagnosis only; the layout may change between versions. */
+CLEAR_API void clear_attn_device_diag(int* out8);
+
 /* ---------------------------------------------------------------------------------------------
  * Host-only scheduler queries (no GPU needed). They expose the tile enumeration the kernels use,
  * so its coverage can be checked against a brute-force mask on the CPU.
  * --------------------------------------------------------------------------------------------- */
 
 /* Work-list shape of the forward. The forward works on pairs of 128-row query tiles that share
- * their key tiles: pairs of consecutive text tiles (split over key ranges) and 16 x 16 image
+ * their 64-key tiles: pairs of consecutive text tiles (split over key ranges) and 16 x 16 image
  * blocks (upper and lower 8 x 16 halves). Returns the numbers of text pairs (all splits) and image
- * pairs, the text split count S and the 128-key chunks per split. Any output may be NULL. */
+ * pairs, the text split count S and the 64-key chunks per split. Any output may be NULL. */
 CLEAR_API clear_status_t clear_sched_forward_shape(const clear_attn_params_t* params, long long* n_text_items,
                                          long long* n_image_items, int* splits,
                                          int* chunks_per_split);
 
 /* Union key tiles visited by forward pair `item` (0 <= item < n_text_items + n_image_items), in
  * order. Each tile is 4 ints: kind (0 = linear chunk, 1 = image rectangle), a, b, flags.
- * Linear: tokens [a, a + 128), first b of them real. Rectangle: grid rows [a, a + 8) x columns
+ * Linear: tokens [a, a + 64), first b of them real. Rectangle: grid rows [a, a + 4) x columns
  * [b, b + 16). flags: bit 0 / bit 1 = half A / half B needs the tile (some kept pair), bit 2 /
  * bit 3 = every pair of half A / half B with the tile is kept (no mask). q_info = {is_text, bh,
  * q0 (first token of half A, or first grid row of the block), x0 (first grid column), half B
@@ -135,7 +141,7 @@ CLEAR_API clear_status_t clear_sched_item_tiles(const clear_attn_params_t* param
                                       int* q_info, int* tiles, int max_tiles, int* n_tiles);
 
 /* Useful (kept-pair) and executed (padded-tile) multiply-add pair counts of one forward call,
- * summed over B and heads: useful = number of ones in the mask; executed = 128 x 128 per tile
+ * summed over B and heads: useful = number of ones in the mask; executed = 128 x 64 per tile
  * product the forward issues (a half times a key tile it needs). FLOPs are 4 * d times these. */
 CLEAR_API clear_status_t clear_sched_pair_counts(const clear_attn_params_t* params, long long* useful_pairs,
                                        long long* executed_pairs);

@@ -56,6 +56,8 @@ _lib.clear_attn_bwd.restype = _i
 _lib.clear_attn_bwd.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 _lib.clear_attn_check.restype = _i
 _lib.clear_attn_check.argtypes = [_vp]
+_lib.clear_attn_device_diag.restype = None
+_lib.clear_attn_device_diag.argtypes = [ctypes.POINTER(_i)]
 _lib.clear_sched_forward_shape.restype = _i
 _lib.clear_sched_forward_shape.argtypes = [_P, ctypes.POINTER(_ll), ctypes.POINTER(_ll), ctypes.POINTER(_i),
                                            ctypes.POINTER(_i)]
@@ -200,3 +202,10 @@ def clear_attn_bwd(q, k, v, o, lse, dO, n_text: int, H: int, W: int, r: int, dq=
 def clear_attn_check(stream=None) -> int:
     """Synchronise the stream and return the device status (CLEAR_OK or an error code)."""
     return _lib.clear_attn_check(_stream_ptr(stream))
+
+
+def device_diag() -> list:
+    """Context of the wait behind the last device timeout reported to this thread (diagnosis)."""
+    out = (_i * 8)()
+    _lib.clear_attn_device_diag(out)
+    return list(out)

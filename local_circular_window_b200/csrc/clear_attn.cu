@@ -72,7 +72,7 @@ struct FwdWorkspace {
 FwdWorkspace fwd_workspace_layout(const Geom& g) {
   FwdWorkspace w{};
   if (g.n_text == 0) return w;
-  const size_t rows = (size_t)g.S * g.BH * g.n_text;
+  const size_t rows = (size_t)g.fS * g.BH * g.n_text;
   w.opart_off = 0;
   w.ml_off = align256(rows * g.d * sizeof(float));
   w.total = align256(w.ml_off + rows * sizeof(float2));
@@ -112,13 +112,13 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// [BH, T, d] viewed as a 3D tensor (d, T, BH); box = 64 x 128 x 1, 128-byte swizzle.
-bool make_linear_map(CUtensorMap* m, const void* base, const Geom& g) {
+// [BH, T, d] viewed as a 3D tensor (d, T, BH); box = 64 x rows x 1, 128-byte swizzle.
+bool make_linear_map(CUtensorMap* m, const void* base, const Geom& g, int rows = kTile) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)g.d, (cuuint64_t)g.T, (cuuint64_t)g.BH};
   cuuint64_t strides[2] = {(cuuint64_t)g.d * 2, (cuuint64_t)g.T * g.d * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)kTile, 1};
+  cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -126,14 +126,15 @@ bool make_linear_map(CUtensorMap* m, const void* base, const Geom& g) {
 }
 
 // Image part of [BH, T, d] viewed as a 4D tensor (d, W, H, BH) starting at token n_text;
-// box = 64 x 16 x 8 x 1 (an 8 x 16 grid rectangle), 128-byte swizzle, zero fill outside the grid.
-bool make_image_map(CUtensorMap* m, const void* base, const Geom& g) {
+// box = 64 x 16 x rows x 1 (a rows x 16 grid rectangle), 128-byte swizzle, zero fill outside
+// the grid.
+bool make_image_map(CUtensorMap* m, const void* base, const Geom& g, int rows = kKH) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   const char* img = static_cast<const char*>(base) + (size_t)g.n_text * g.d * 2;
   cuuint64_t dims[4] = {(cuuint64_t)g.d, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.BH};
   cuuint64_t strides[3] = {(cuuint64_t)g.d * 2, (cuuint64_t)g.W * g.d * 2, (cuuint64_t)g.T * g.d * 2};
-  cuuint32_t box[4] = {64, (cuuint32_t)kKW, (cuuint32_t)kKH, 1};
+  cuuint32_t box[4] = {64, (cuuint32_t)kKW, (cuuint32_t)rows, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<char*>(img), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -148,6 +149,13 @@ bool make_qkv_maps(QKVMaps* m, const void* q, const void* k, const void* v, cons
   return make_linear_map(&m->q_lin, q, g) && make_image_map(&m->q_img, q, g) &&
          make_linear_map(&m->k_lin, k, g) && make_image_map(&m->k_img, k, g) &&
          make_linear_map(&m->v_lin, v, g) && make_image_map(&m->v_img, v, g);
+}
+
+// Forward maps: 128-row query tiles, 64-key K/V tiles (64-token chunks and 4 x 16 rectangles).
+bool make_fwd_maps(QKVMaps* m, const void* q, const void* k, const void* v, const Geom& g) {
+  return make_linear_map(&m->q_lin, q, g) && make_image_map(&m->q_img, q, g) &&
+         make_linear_map(&m->k_lin, k, g, kFChunk) && make_image_map(&m->k_img, k, g, kFKH) &&
+         make_linear_map(&m->v_lin, v, g, kFChunk) && make_image_map(&m->v_img, v, g, kFKH);
 }
 
 template <int D>
@@ -229,7 +237,7 @@ clear_status_t clear_attn_fwd(const clear_attn_params_t* params, const void* q, 
   clear_status_t st = check_device(&num_sms);
   if (st != CLEAR_OK) return st;
   QKVMaps maps;
-  if (!make_qkv_maps(&maps, q, k, v, c.g)) return CLEAR_ERR_CUDA;
+  if (!make_fwd_maps(&maps, q, k, v, c.g)) return CLEAR_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return c.g.d == 128 ? launch_fwd<128>(c.g, maps, o, lse, workspace, num_sms, s)
                       : launch_fwd<64>(c.g, maps, o, lse, workspace, num_sms, s);
@@ -270,17 +278,26 @@ clear_status_t clear_attn_bwd(const clear_attn_params_t* params, const void* q, 
                                        maps.v_img, do_lin, do_img, num_sms, s);
 }
 
+static thread_local int t_last_diag[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+
 clear_status_t clear_attn_check(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return CLEAR_ERR_CUDA;
   int err = 0;
   if (cudaMemcpyFromSymbol(&err, clear::g_clear_device_error, sizeof(int)) != cudaSuccess)
     return CLEAR_ERR_CUDA;
   if (err != 0) {
+    if (cudaMemcpyFromSymbol(t_last_diag, clear::g_clear_device_diag, sizeof(t_last_diag)) != cudaSuccess)
+      return CLEAR_ERR_CUDA;
     const int zero = 0;
     cudaMemcpyToSymbol(clear::g_clear_device_error, &zero, sizeof(int));
     return CLEAR_ERR_DEVICE_TIMEOUT;
   }
   return CLEAR_OK;
+}
+
+void clear_attn_device_diag(int* out8) {
+  if (!out8) return;
+  for (int i = 0; i < 8; ++i) out8[i] = t_last_diag[i];
 }
 
 clear_status_t clear_sched_forward_shape(const clear_attn_params_t* params, long long* n_text_items,
@@ -290,8 +307,8 @@ clear_status_t clear_sched_forward_shape(const clear_attn_params_t* params, long
   if (c.st != CLEAR_OK) return c.st;
   if (n_text_items) *n_text_items = c.g.n_txt_pairs;
   if (n_image_items) *n_image_items = c.g.n_img_pairs;
-  if (splits) *splits = c.g.S;
-  if (chunks_per_split) *chunks_per_split = c.g.cps;
+  if (splits) *splits = c.g.fS;
+  if (chunks_per_split) *chunks_per_split = c.g.fcps;
   return CLEAR_OK;
 }
 
@@ -355,13 +372,13 @@ clear_status_t clear_sched_pair_counts(const clear_attn_params_t* params, long l
       count_pair_tiles(g, it, nullptr, 0, &nu, &na, &nb);
       tiles += na + nb;
     }
-    for (long long w = 0; w < (long long)g.nTq2 * g.S; ++w) {
+    for (long long w = 0; w < (long long)g.nTq2 * g.fS; ++w) {
       const PairItem it = decode_pair(g, w);
       int nu, na, nb;
       count_pair_tiles(g, it, nullptr, 0, &nu, &na, &nb);
       tiles += na + nb;
     }
-    *executed_pairs = tiles * (long long)kTile * kTile * g.BH;
+    *executed_pairs = tiles * (long long)kTile * kFChunk * g.BH;
   }
   return CLEAR_OK;
 }

@@ -8,19 +8,21 @@
 //
 // One CTA per SM, persistent over a static list of pair items (clear_sched.cuh). A pair is two
 // 128-row query tiles ("halves" A and B: the upper and lower 8 x 16 rectangles of a 16 x 16 image
-// block, or two consecutive text tiles) that share every key tile: each K/V tile is loaded once
+// block, or two consecutive text tiles) that share every 64-key tile: each K/V tile is loaded once
 // and multiplied by whichever halves reach it.
-//   warps 0-3  softmax / epilogue of half A (thread t owns query row t = TMEM lane t);
-//   warps 4-7  softmax / epilogue of half B;
-//   warp 8     TMA producer: Q of both halves once per pair, K tiles into a 2-slot ring, V tiles
-//              into a 2-slot ring; it polls the three streams and issues whatever has room;
-//   warps 9/10 MMA issuers, one per half: S = Q K^T (TMEM), then, once the softmax has written P
-//              over S (bf16, in TMEM), O += P V (A operand from TMEM). The two halves run
-//              independently, so one half's products overlap the other half's softmax. A K/V slot
-//              is released when both halves are done with it (barriers with two arrivals: a half
-//              that skips a tile arrives once the tile has landed, keeping arrivals in phase);
-//   warp 11    idle (it completes the third warpgroup, whose registers go to the softmax).
-// TMEM columns: S_A [0,128), O_A [128,256), S_B [256,384), O_B [384,512).
+//   warps 0-3   softmax / epilogue of half A (thread t owns query row t = TMEM lane t);
+//   warps 4-7   softmax / epilogue of half B;
+//   warp 8      TMA producer: Q of both halves once per pair, K and V tiles into 4-slot rings;
+//   warps 9/10  MMA issuers, one per half. Each polls two walks over the pair's union tiles: the
+//               QK walk issues S_j = Q K_j^T into one of two 64-column TMEM buffers (up to one
+//               needed tile ahead of P V); the PV walk issues O += P_j V_j once the softmax has
+//               written P_j over S_j (bf16, in TMEM; A operand from TMEM). Tiles a half does not
+//               need are still observed (their "full" phase) and released by that half, so each
+//               half sees every phase of every ring slot in order, which is what makes the
+//               parity-based barrier waits exact. Polling (instead of blocking) keeps either walk
+//               from holding up the other, so every wait depends only on earlier tiles;
+//   warp 11     idle (it completes the third warpgroup, whose registers go to the softmax).
+// TMEM columns of half h: S buffers [256h, 256h+64) and [256h+64, 256h+128), O [256h+128, 256h+256).
 // The running max is rescaled lazily: O and l are only rescaled when a row's max grows by more
 // than 2^8, which leaves the result exact up to rounding (the final division uses the same max).
 #pragma once
@@ -32,12 +34,12 @@
 
 namespace clear {
 
-constexpr int kKStages = 2;   // K ring slots (a slot is freed once every Q K^T reading it is done)
-constexpr int kVStages = 2;   // V ring slots (freed once every P V reading it is done)
+constexpr int kKStages = 4;   // K ring slots
+constexpr int kVStages = 4;   // V ring slots
 constexpr int kFwdThreads = 384;           // 3 warpgroups: softmax A, softmax B, producer + MMA
 // Launched at 168 registers per thread (65536 / 384, rounded to 8). The producer / MMA warpgroup
 // drops to kRegsLow and the two softmax warpgroups grow to kRegsHigh:
-// 2 * 128 * kRegsHigh + 128 * kRegsLow = 384 * 168.
+// 2 * 128 * kRegsHigh + 128 * kRegsLow <= 384 * 168.
 constexpr uint32_t kRegsLow = 72;
 constexpr uint32_t kRegsHigh = 216;
 static_assert(2 * 128 * kRegsHigh + 128 * kRegsLow <= 384 * 168, "register split exceeds the launch allocation");
@@ -49,39 +51,57 @@ struct FwdParams {
   float scale_log2;           // (1/sqrt(d)) * log2(e)
   __nv_bfloat16* o;           // [BH, T, d]
   float* lse;                 // [BH, T]
-  float* opart;               // [S, BH, n_text, d] unnormalised partial O of text rows
-  float2* ml;                 // [S, BH, n_text] (running max in scaled log2 units, sum)
+  float* opart;               // [fS, BH, n_text, d] unnormalised partial O of text rows
+  float2* ml;                 // [fS, BH, n_text] (running max in scaled log2 units, sum)
   long long n_work;           // pair items
 };
 
 template <int D>
 struct FwdLayout {
-  static constexpr int kTileBytes = kTile * D * 2;       // one 128-row bf16 tile
+  static constexpr int kQTileBytes = kTile * D * 2;      // one 128-row bf16 query tile
+  static constexpr int kKVTileBytes = kFChunk * D * 2;   // one 64-key bf16 tile
+  static constexpr int kKVBlock = kFChunk * 128;         // 64 rows x 64 elements (128B-swizzled)
   static constexpr int kQ = 0;                           // Q_A, Q_B
-  static constexpr int kK = kQ + 2 * kTileBytes;
-  static constexpr int kV = kK + kKStages * kTileBytes;
-  static constexpr int kBars = kV + kVStages * kTileBytes;
+  static constexpr int kK = kQ + 2 * kQTileBytes;
+  static constexpr int kV = kK + kKStages * kKVTileBytes;
+  static constexpr int kBars = kV + kVStages * kKVTileBytes;
   // barrier indices
   static constexpr int bQFull = 0, bQEmpty = 1;
   static constexpr int bKFull = 2;                       // + slot
   static constexpr int bKEmpty = bKFull + kKStages;      // + slot
   static constexpr int bVFull = bKEmpty + kKStages;      // + slot
   static constexpr int bVEmpty = bVFull + kVStages;      // + slot
-  static constexpr int bSFull = bVEmpty + kVStages;      // + half
-  static constexpr int bPFull = bSFull + 2;              // + half
-  static constexpr int bODone = bPFull + 2;              // + half
-  static constexpr int bInfo = bODone + 2;               // + half: tile descriptor mailbox full
-  static constexpr int kNumBars = bInfo + 2;
-  static constexpr int kInfo = kBars + kNumBars * 8;     // int4[2]: {kind, a, b, flags | kLastTile}
-  static constexpr int kMisc = kInfo + 32;
+  static constexpr int bSFull = bVEmpty + kVStages;      // + 2 * half + buffer
+  static constexpr int bPFull = bSFull + 4;              // + 2 * half + buffer
+  static constexpr int bInfo = bPFull + 4;               // + 2 * half + buffer
+  static constexpr int bODone = bInfo + 4;               // + half: last P V of the half's pair done
+  static constexpr int bOReady = bODone + 2;             // + half: every P V done (one phase per tile)
+  static constexpr int kNumBars = bOReady + 2;
+  static constexpr int kInfo = kBars + kNumBars * 8;     // int4[2][2]: {kind, a, b, flags | kLastTile}
+  static constexpr int kMisc = kInfo + 64;
   static constexpr int kWTab = kMisc + 16;               // int[kMaxRTable] (tile enumeration)
   static constexpr int kHwTab = kWTab + kMaxRTable * 4;  // int16[hw_table_size(r, H)] (masks)
   static constexpr int kFixed = kHwTab + 1024;           // + slack for 1024-byte alignment
   static __host__ __device__ constexpr int alloc_bytes(int hw_entries) { return kFixed + ((hw_entries * 2 + 15) & ~15); }
   static constexpr uint32_t kTmemCols = 512;
-  static __host__ __device__ constexpr uint32_t s_col(int half) { return half * 256; }
+  static __host__ __device__ constexpr uint32_t s_col(int half, int buf) { return half * 256 + buf * 64; }
   static __host__ __device__ constexpr uint32_t o_col(int half) { return half * 256 + 128; }
 };
+
+// Loads one 64-key tile (all 64-element column blocks) of k or v: a 64-token chunk (kind kLinear,
+// first token a) or a 4 x 16 grid rectangle (kind kRect, rows from a, columns from b).
+template <int D>
+__device__ __forceinline__ void load_kv64(uint8_t* dst, const CUtensorMap* lin, const CUtensorMap* img, uint64_t* bar,
+                                          int kind, int a, int b, int bh) {
+  #pragma unroll
+  for (int h = 0; h < D / 64; ++h) {
+    uint8_t* d = dst + h * FwdLayout<D>::kKVBlock;
+    if (kind == kLinear)
+      tma_load_3d(d, lin, bar, h * 64, a, bh);
+    else
+      tma_load_4d(d, img, bar, h * 64, b, a, bh);
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1)
@@ -114,16 +134,20 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
       mbar_init(&bars[L::bVFull + s], 1);
       mbar_init(&bars[L::bVEmpty + s], 2);
     }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&bars[L::bSFull + i], 1);
+      mbar_init(&bars[L::bPFull + i], 128);
+      mbar_init(&bars[L::bInfo + i], 1);
+    }
     for (int h = 0; h < 2; ++h) {
-      mbar_init(&bars[L::bSFull + h], 1);
-      mbar_init(&bars[L::bPFull + h], 128);
       mbar_init(&bars[L::bODone + h], 1);
-      mbar_init(&bars[L::bInfo + h], 1);
+      mbar_init(&bars[L::bOReady + h], 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
   }
-  // Half-width table: wtab[dy] = largest dx with dx^2 + dy^2 < r^2 (or -1).
+  // Half-width tables: wtab[dy] (tile enumeration, first kMaxRTable rows) and the int16 table
+  // hwtab[dy] for every |dy| < min(r, H) (masks).
   for (int i = threadIdx.x; i < kMaxRTable; i += blockDim.x) wtab[i] = half_width(g.r, i);
   const int hwn = hw_table_size(g.r, g.H);
   for (int i = threadIdx.x; i < hwn; i += blockDim.x) hwtab[i] = (int16_t)half_width(g.r, i);
@@ -137,6 +161,7 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
   const uint32_t tmem = *tmem_slot;
   const int wtn = imin(g.r, kMaxRTable);
   const long long stride = gridDim.x;
+
   if (warp == 8) {
     // ------------------------------------------------------------------ TMA producer
     regs_dec<kRegsLow>();
@@ -159,16 +184,16 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
         bool prog = false;
         if (wq < p.n_work && (q_loads == 0 || mbar_test(&bars[L::bQEmpty], (q_loads - 1) & 1))) {
           const PairItem it = decode_pair(g, wq);
-          mbar_arrive_expect_tx(&bars[L::bQFull], (it.validB ? 2 : 1) * L::kTileBytes);
+          mbar_arrive_expect_tx(&bars[L::bQFull], (it.validB ? 2 : 1) * L::kQTileBytes);
           if (it.is_text) {
             load_tile<D>(smem + L::kQ, &tm_q_lin, &tm_q_img, &bars[L::bQFull], kLinear, it.q0, 0, it.bh);
             if (it.validB)
-              load_tile<D>(smem + L::kQ + L::kTileBytes, &tm_q_lin, &tm_q_img, &bars[L::bQFull], kLinear,
+              load_tile<D>(smem + L::kQ + L::kQTileBytes, &tm_q_lin, &tm_q_img, &bars[L::bQFull], kLinear,
                            it.q0 + kTile, 0, it.bh);
           } else {
             load_tile<D>(smem + L::kQ, &tm_q_lin, &tm_q_img, &bars[L::bQFull], kRect, it.q0, it.x0, it.bh);
             if (it.validB)
-              load_tile<D>(smem + L::kQ + L::kTileBytes, &tm_q_lin, &tm_q_img, &bars[L::bQFull], kRect,
+              load_tile<D>(smem + L::kQ + L::kQTileBytes, &tm_q_lin, &tm_q_img, &bars[L::bQFull], kRect,
                            it.q0 + kQH, it.x0, it.bh);
           }
           ++q_loads;
@@ -178,8 +203,8 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
         if (kval) {
           const uint32_t ks = Gk % kKStages;
           if (mbar_test(&bars[L::bKEmpty + ks], ((Gk / kKStages) & 1) ^ 1)) {
-            mbar_arrive_expect_tx(&bars[L::bKFull + ks], L::kTileBytes);
-            load_tile<D>(smem + L::kK + ks * L::kTileBytes, &tm_k_lin, &tm_k_img, &bars[L::bKFull + ks], tk.kind,
+            mbar_arrive_expect_tx(&bars[L::bKFull + ks], L::kKVTileBytes);
+            load_kv64<D>(smem + L::kK + ks * L::kKVTileBytes, &tm_k_lin, &tm_k_img, &bars[L::bKFull + ks], tk.kind,
                          tk.a, tk.b, itk.bh);
             ++Gk;
             if (!kik.next(&tk)) {
@@ -193,8 +218,8 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
         if (vval && Gv < Gk) {
           const uint32_t vs = Gv % kVStages;
           if (mbar_test(&bars[L::bVEmpty + vs], ((Gv / kVStages) & 1) ^ 1)) {
-            mbar_arrive_expect_tx(&bars[L::bVFull + vs], L::kTileBytes);
-            load_tile<D>(smem + L::kV + vs * L::kTileBytes, &tm_v_lin, &tm_v_img, &bars[L::bVFull + vs], tv.kind,
+            mbar_arrive_expect_tx(&bars[L::bVFull + vs], L::kKVTileBytes);
+            load_kv64<D>(smem + L::kV + vs * L::kKVTileBytes, &tm_v_lin, &tm_v_img, &bars[L::bVFull + vs], tv.kind,
                          tv.a, tv.b, itv.bh);
             ++Gv;
             if (!kiv.next(&tv)) {
@@ -205,7 +230,7 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
             prog = true;
           }
         }
-        if (!wd.tick(prog, abort_flag, kDevTimeoutTmaEmpty)) break;
+        if (!wd.tick(prog, abort_flag, kDevTimeoutTmaEmpty, 1, (int)Gk, (int)Gv, (int)q_loads)) break;
       }
     }
     __syncwarp();
@@ -213,72 +238,132 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
     // ------------------------------------------------------------------ MMA issuers (one per half)
     regs_dec<kRegsLow>();
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kFChunk, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
       const int h = warp - 9;
       const int need_bit = h == 0 ? kNeedA : kNeedB;
-      const uint32_t q_addr = smem_u32(smem + L::kQ + h * L::kTileBytes);
-      const uint32_t s_tm = tmem + L::s_col(h);
+      const uint32_t q_addr = smem_u32(smem + L::kQ + h * L::kQTileBytes);
       const uint32_t o_tm = tmem + L::o_col(h);
-      uint32_t G = 0, nq = 0, items = 0;
-      for (long long w = blockIdx.x; w < p.n_work; w += stride, ++items) {
-        const PairItem it = decode_pair(g, w);
-        int nu, na, nb;
-        count_pair_tiles(g, it, wtab, wtn, &nu, &na, &nb);
-        const int n = h == 0 ? na : nb;
-        if (n == 0) {  // this half has no queries in the pair: release Q once it has landed
-          if (!mbar_wait(&bars[L::bQFull], items & 1, abort_flag, kDevTimeoutMma)) goto mma_done;
-          mbar_arrive(&bars[L::bQEmpty]);
-        }
-        PairKeyIter ki;
-        ki.init(g, it, wtab, wtn);
-        KeyTile t;
-        int j = 0;
-        for (; ki.next(&t); ++G) {
-          const uint32_t ks = G % kKStages, kph = (G / kKStages) & 1;
-          const uint32_t vs = G % kVStages, vph = (G / kVStages) & 1;
-          if (!(t.flags & need_bit)) {
-            // Skipped tile: arrive on its empty barriers once it has landed (so the arrival
-            // belongs to this use of the slot).
-            if (!mbar_wait(&bars[L::bKFull + ks], kph, abort_flag, kDevTimeoutMma)) goto mma_done;
-            mbar_arrive(&bars[L::bKEmpty + ks]);
-            if (!mbar_wait(&bars[L::bVFull + vs], vph, abort_flag, kDevTimeoutMma)) goto mma_done;
-            mbar_arrive(&bars[L::bVEmpty + vs]);
-            continue;
+      // QK walk over the union tiles (union index Gq, needed-tile counter nqk).
+      long long wq = blockIdx.x;
+      uint32_t items = 0, Gq = 0, nqk = 0;
+      PairKeyIter ki;
+      KeyTile t{};
+      bool in_item = false, q_seen = false, have = false, done = false;
+      int jq = 0, nitem = 0;
+      // PV walk: union index Gp; up to two needed tiles whose Q K^T is issued and P V is not.
+      uint32_t Gp = 0, npv = 0;
+      uint32_t pend_G[2] = {0, 0};
+      int pend_fl[2] = {0, 0};  // bit 0: first of item, bit 1: last of item
+      int pend = 0;
+      PollWatchdog wd;
+      wd.start();
+      while (!done || Gp < Gq) {
+        bool prog = false;
+        // ---- QK walk step
+        if (!done && !in_item) {
+          if (wq >= p.n_work) {
+            done = true;
+          } else {
+            const PairItem it = decode_pair(g, wq);
+            int nu, na, nb;
+            count_pair_tiles(g, it, wtab, wtn, &nu, &na, &nb);
+            nitem = h == 0 ? na : nb;
+            jq = 0;
+            ki.init(g, it, wtab, wtn);
+            in_item = true;
+            q_seen = false;
+            have = false;
           }
-          // Hand the tile to this half's softmax (its previous descriptor was consumed before it
-          // signalled the previous P, which this thread has waited for).
-          info[h] = make_int4(t.kind, t.a, t.b, t.flags | (j == n - 1 ? kLastTile : 0));
-          mbar_arrive(&bars[L::bInfo + h]);
-          if (j == 0 && !mbar_wait(&bars[L::bQFull], items & 1, abort_flag, kDevTimeoutMma)) goto mma_done;
-          if (!mbar_wait(&bars[L::bKFull + ks], kph, abort_flag, kDevTimeoutMma)) goto mma_done;
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(smem + L::kK + ks * L::kTileBytes);
-          #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-            umma_ss(s_tm, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
-                    idesc_qk, kk > 0);
-          }
-          umma_commit(&bars[L::bSFull + h]);
-          umma_commit(&bars[L::bKEmpty + ks]);
-          if (j == n - 1) umma_commit(&bars[L::bQEmpty]);
-          // O += P V once the softmax has written P over S
-          if (!mbar_wait(&bars[L::bPFull + h], nq & 1, abort_flag, kDevTimeoutMma)) goto mma_done;
-          if (!mbar_wait(&bars[L::bVFull + vs], vph, abort_flag, kDevTimeoutMma)) goto mma_done;
-          tc_fence_after();
-          const uint32_t v_addr = smem_u32(smem + L::kV + vs * L::kTileBytes);
-          #pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk)
-            umma_ts(o_tm, s_tm + kk * 8, smem_desc_sw128(v_addr + kk * 2048, kHalfBytes, 1024), idesc_pv,
-                    (j > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&bars[L::bVEmpty + vs]);
-          if (j == n - 1) umma_commit(&bars[L::bODone + h]);
-          ++nq;
-          ++j;
         }
+        if (in_item && !q_seen && mbar_test(&bars[L::bQFull], items & 1)) {
+          q_seen = true;  // every half observes every Q phase; a half without queries here
+          if (nitem == 0) mbar_arrive(&bars[L::bQEmpty]);  // releases Q at once
+          prog = true;
+        }
+        if (in_item && q_seen && !have) {
+          if (ki.next(&t)) {
+            have = true;
+          } else {
+            in_item = false;
+            ++items;
+            wq += stride;
+            prog = true;
+          }
+        }
+        if (have) {
+          const uint32_t ks = Gq % kKStages;
+          const bool needed = (t.flags & need_bit) != 0;
+          if ((!needed || pend < 2) && mbar_test(&bars[L::bKFull + ks], (Gq / kKStages) & 1)) {
+            if (!needed) {
+              mbar_arrive(&bars[L::bKEmpty + ks]);  // observed and released
+            } else {
+              const bool last = (jq == nitem - 1);
+              const uint32_t b = nqk & 1;
+              // Hand the tile to this half's softmax. Slot b was last used by needed tile nqk - 2,
+              // whose P has been consumed (its P V is issued before this Q K^T can be).
+              info[2 * h + b] = make_int4(t.kind, t.a, t.b, t.flags | (last ? kLastTile : 0));
+              mbar_arrive(&bars[L::bInfo + 2 * h + b]);
+              tc_fence_after();
+              const uint32_t k_addr = smem_u32(smem + L::kK + ks * L::kKVTileBytes);
+              #pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t qoff = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+                const uint32_t koff = (kk >> 2) * L::kKVBlock + (kk & 3) * 32;
+                umma_ss(tmem + L::s_col(h, b), smem_desc_sw128(q_addr + qoff, 16, 1024),
+                        smem_desc_sw128(k_addr + koff, 16, 1024), idesc_qk, kk > 0);
+              }
+              umma_commit(&bars[L::bSFull + 2 * h + b]);
+              umma_commit(&bars[L::bKEmpty + ks]);
+              if (last) umma_commit(&bars[L::bQEmpty]);
+              const int slot = (npv + pend) & 1;
+              pend_G[slot] = Gq;
+              pend_fl[slot] = (jq == 0 ? 1 : 0) | (last ? 2 : 0);
+              ++pend;
+              ++nqk;
+              ++jq;
+            }
+            ++Gq;
+            have = false;
+            prog = true;
+          }
+        }
+        // ---- PV walk step (tiles the QK walk has passed, in order)
+        if (Gp < Gq) {
+          const uint32_t vs = Gp % kVStages;
+          const int slot = npv & 1;
+          const bool needed = pend > 0 && pend_G[slot] == Gp;
+          if (!needed) {
+            if (mbar_test(&bars[L::bVFull + vs], (Gp / kVStages) & 1)) {
+              mbar_arrive(&bars[L::bVEmpty + vs]);  // observed and released
+              ++Gp;
+              prog = true;
+            }
+          } else {
+            const uint32_t b = npv & 1;
+            if (mbar_test(&bars[L::bPFull + 2 * h + b], (npv >> 1) & 1) &&
+                mbar_test(&bars[L::bVFull + vs], (Gp / kVStages) & 1)) {
+              tc_fence_after();
+              const uint32_t v_addr = smem_u32(smem + L::kV + vs * L::kKVTileBytes);
+              const uint32_t s_tm = tmem + L::s_col(h, b);
+              const bool first = pend_fl[slot] & 1;
+              #pragma unroll
+              for (int kk = 0; kk < kFChunk / 16; ++kk)
+                umma_ts(o_tm, s_tm + kk * 8, smem_desc_sw128(v_addr + kk * 2048, L::kKVBlock, 1024), idesc_pv,
+                        (!first || kk > 0) ? 1u : 0u);
+              umma_commit(&bars[L::bVEmpty + vs]);
+              umma_commit(&bars[L::bOReady + h]);
+              if (pend_fl[slot] & 2) umma_commit(&bars[L::bODone + h]);
+              ++npv;
+              --pend;
+              ++Gp;
+              prog = true;
+            }
+          }
+        }
+        if (!wd.tick(prog, abort_flag, kDevTimeoutMma, 2 + h, (int)Gq, (int)(Gp | (npv << 16)),
+                     pend | (have ? 4 : 0) | (done ? 8 : 0) | (q_seen ? 16 : 0) | ((int)items << 8))) break;
       }
-    mma_done:;
     }
     __syncwarp();
   } else if (warp == 11) {
@@ -289,7 +374,6 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
     const int half = warp >> 2;              // 0: A, 1: B
     const int row = threadIdx.x & 127;       // TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t s_tm = tmem + lane_base + L::s_col(half);
     const uint32_t o_tm = tmem + lane_base + L::o_col(half);
     const int full_bit = half == 0 ? kFullA : kFullB;
     uint32_t nq = 0, n_out = 0;
@@ -312,38 +396,40 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
       int j = 0;
       bool last = false;
       while (!last) {
-        if (!mbar_wait(&bars[L::bInfo + half], nq & 1, abort_flag, kDevTimeoutSoftmax)) goto softmax_done;
-        const int4 ti = info[half];
+        const uint32_t b = nq & 1, ph = (nq >> 1) & 1;
+        if (!mbar_wait(&bars[L::bInfo + 2 * half + b], ph, abort_flag, kDevTimeoutSoftmax, 10 + half, (int)nq, j))
+          goto softmax_done;
+        const int4 ti = info[2 * half + b];
         KeyTile t;
         t.kind = ti.x;
         t.a = ti.y;
         t.b = ti.z;
         t.flags = ti.w;
         last = (ti.w & kLastTile) != 0;
-        if (!mbar_wait(&bars[L::bSFull + half], nq & 1, abort_flag, kDevTimeoutSoftmax)) goto softmax_done;
+        if (!mbar_wait(&bars[L::bSFull + 2 * half + b], ph, abort_flag, kDevTimeoutSoftmax, 12 + half, (int)nq, j))
+          goto softmax_done;
         tc_fence_after();
-        float s[kTile];
+        const uint32_t s_tm = tmem + lane_base + L::s_col(half, b);
+        float s[kFChunk];
         {
-          uint32_t sr[4][32];
+          uint32_t sr[2][32];
           tmem_ld32(s_tm + 0, sr[0]);
           tmem_ld32(s_tm + 32, sr[1]);
-          tmem_ld32(s_tm + 64, sr[2]);
-          tmem_ld32(s_tm + 96, sr[3]);
           tmem_wait_ld();
           #pragma unroll
-          for (int c = 0; c < kTile; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
+          for (int c = 0; c < kFChunk; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
         }
         // ---- mask (branch-free selects; full tiles skip it)
         if (!(t.flags & full_bit)) {
           if (t.kind == kLinear) {
             const int lim = t.b;
             #pragma unroll
-            for (int c = 0; c < kTile; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
+            for (int c = 0; c < kFChunk; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
           } else {
             // keep bits: word q holds key rows 2q (bits 0-15) and 2q+1 (bits 16-31)
-            uint32_t keep[kKH / 2];
+            uint32_t keep[kFKH / 2];
             #pragma unroll
-            for (int q = 0; q < kKH / 2; ++q) {
+            for (int q = 0; q < kFKH / 2; ++q) {
               int lo0, hi0, lo1, hi1;
               row_range_tab(g, hwtab, hwn, yq, xq, t.a + 2 * q, t.b, &lo0, &hi0);
               row_range_tab(g, hwtab, hwn, yq, xq, t.a + 2 * q + 1, t.b, &lo1, &hi1);
@@ -351,7 +437,7 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
               keep[q] = (((1u << n0) - 1u) << (lo0 & 15)) | ((((1u << n1) - 1u) << (lo1 & 15)) << 16);
             }
             #pragma unroll
-            for (int c = 0; c < kTile; ++c)
+            for (int c = 0; c < kFChunk; ++c)
               s[c] = (keep[c >> 5] & (1u << (c & 31))) ? s[c] : -INFINITY;
           }
         }
@@ -360,16 +446,13 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
         #pragma unroll
         for (int u = 0; u < 8; ++u) mx[u] = fmax3(s[u], s[u + 8], s[u + 16]);
         #pragma unroll
-        for (int c = 24; c < kTile - 8; c += 16) {
-          #pragma unroll
-          for (int u = 0; u < 8; ++u) mx[u] = fmax3(mx[u], s[c + u], s[c + 8 + u]);
-        }
+        for (int u = 0; u < 8; ++u) mx[u] = fmax3(mx[u], s[u + 24], s[u + 32]);
         #pragma unroll
-        for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], s[kTile - 8 + u]);
+        for (int u = 0; u < 8; ++u) mx[u] = fmax3(mx[u], s[u + 40], s[u + 48]);
+        #pragma unroll
+        for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], s[u + 56]);
         const float mt = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(fmax3(mx[3], mx[4], mx[5]), mx[6], mx[7]));
         const float mt_scaled = mt * sl2;
-        // S_j being ready means every earlier product of this CTA has completed, including this
-        // half's P V of tile j-1: O may be rescaled in place.
         float alpha = 1.f;
         bool need_rescale = false;
         if (m_used == -INFINITY) {
@@ -381,6 +464,11 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
           need_rescale = true;
         }
         if (j > 0 && __any_sync(0xffffffffu, need_rescale)) {
+          // O holds P V up to tile j-1: wait for that product (the one for tile j cannot start
+          // before this tile's P is signalled), then rescale O in place.
+          if (!mbar_wait(&bars[L::bOReady + half], (nq - 1) & 1, abort_flag, kDevTimeoutSoftmax, 14 + half, (int)nq, j))
+            goto softmax_done;
+          tc_fence_after();
           #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t ov[32];
@@ -394,30 +482,26 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
         // ---- P = 2^(s * scale_log2 - m), row sum, bf16 pairs written over S in TMEM
         const float base = (m_used == -INFINITY) ? 0.f : m_used;
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        uint32_t pw[32];
         #pragma unroll
-        for (int hc = 0; hc < 2; ++hc) {
-          uint32_t pw[32];
-          #pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            const int c = hc * 64 + 2 * q;
-            const float e0 = ex2_approx(fmaf(s[c], sl2, -base));
-            const float e1 = ex2_approx(fmaf(s[c + 1], sl2, -base));
-            acc[(2 * q) & 7] += e0;
-            acc[(2 * q + 1) & 7] += e1;
-            pw[q] = pack_bf16x2(e0, e1);
-          }
-          tmem_st32(s_tm + hc * 32, pw);
+        for (int q = 0; q < 32; ++q) {
+          const float e0 = ex2_approx(fmaf(s[2 * q], sl2, -base));
+          const float e1 = ex2_approx(fmaf(s[2 * q + 1], sl2, -base));
+          acc[(2 * q) & 7] += e0;
+          acc[(2 * q + 1) & 7] += e1;
+          pw[q] = pack_bf16x2(e0, e1);
         }
+        tmem_st32(s_tm, pw);
         l += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars[L::bPFull + half]);
+        mbar_arrive(&bars[L::bPFull + 2 * half + b]);
         ++nq;
         ++j;
       }
       // ---- epilogue: wait for this half's last P V, then write O / l (or the split partial)
-      if (j == 0) continue;
-      if (!mbar_wait(&bars[L::bODone + half], n_out & 1, abort_flag, kDevTimeoutSoftmax)) goto softmax_done;
+      if (!mbar_wait(&bars[L::bODone + half], n_out & 1, abort_flag, kDevTimeoutSoftmax, 16 + half, (int)nq, (int)n_out))
+        goto softmax_done;
       ++n_out;
       tc_fence_after();
       if (it.is_text) {
@@ -487,7 +571,7 @@ __global__ void clear_fwd_combine_kernel(const FwdParams p) {
   const int bh = (int)(row_id / g.n_text);
   const int tq = (int)(row_id % g.n_text);
   float m = -INFINITY;
-  for (int s = 0; s < g.S; ++s) {
+  for (int s = 0; s < g.fS; ++s) {
     const float2 v = p.ml[((size_t)s * g.BH + bh) * g.n_text + tq];
     if (v.y > 0.f) m = fmaxf(m, v.x);
   }
@@ -496,7 +580,7 @@ __global__ void clear_fwd_combine_kernel(const FwdParams p) {
   #pragma unroll
   for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
   float l = 0.f;
-  for (int s = 0; s < g.S; ++s) {
+  for (int s = 0; s < g.fS; ++s) {
     const size_t prow = ((size_t)s * g.BH + bh) * g.n_text + tq;
     const float2 v = p.ml[prow];
     if (!(v.y > 0.f)) continue;

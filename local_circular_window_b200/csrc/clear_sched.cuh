@@ -42,6 +42,10 @@ constexpr int kQW = 16;     // image query tile columns
 constexpr int kKH = 8;      // image key tile rows
 constexpr int kKW = 16;     // image key tile columns
 constexpr int kTile = 128;  // rows per query tile, keys per key tile
+// The forward pairs two query tiles and visits 64-key tiles: 4 x 16 grid rectangles or 64-token
+// chunks (half-size key tiles let each half double-buffer S in tensor memory).
+constexpr int kFKH = 4;       // forward key rectangle rows
+constexpr int kFChunk = 64;   // forward keys per tile
 
 enum KeyKind : int { kLinear = 0, kRect = 1 };
 enum KeyFlags : int { kNeedsMask = 0, kFull = 1 };
@@ -64,9 +68,12 @@ struct Geom {
   int cps;           // chunks per split
   long long n_txt_items, n_img_items;
   // Forward pairs: two query tiles share every key tile they visit (a 16 x 16 image block, or
-  // two consecutive 128-row text tiles).
+  // two consecutive 128-row text tiles); key tiles are 64 keys.
   int nqy2, nQ2;     // image blocks per (b, h): ceil(H/16) x ceil(W/16)
   int nTq2;          // text tile pairs: ceil(nTq / 2)
+  int fnC;           // 64-key chunks over all T tokens
+  int fnTk;          // 64-key chunks over the text tokens
+  int fS, fcps;      // forward text splits and 64-key chunks per split
   long long n_txt_pairs, n_img_pairs;
 };
 
@@ -121,7 +128,10 @@ CLEAR_HD Geom make_geom(int B, int heads, int n_text, int H, int W, int d, int r
   g.nqy2 = cdiv(H, 2 * kQH);
   g.nQ2 = g.nqy2 * g.nqx;
   g.nTq2 = cdiv(g.nTq, 2);
-  g.n_txt_pairs = (long long)g.BH * g.nTq2 * g.S;
+  g.fnC = cdiv(g.T, kFChunk);
+  g.fnTk = cdiv(n_text, kFChunk);
+  choose_splits(g.fnC, 2 * kSplitTargetChunks, kMaxSplits, &g.fS, &g.fcps);
+  g.n_txt_pairs = (long long)g.BH * g.nTq2 * g.fS;
   g.n_img_pairs = (long long)g.BH * g.nQ2;
   return g;
 }
@@ -270,8 +280,8 @@ struct PairItem {
 CLEAR_HD PairItem decode_pair(const Geom& g, long long w) {
   PairItem it;
   if (w < g.n_txt_pairs) {
-    int s = (int)(w % g.S);
-    long long t = w / g.S;
+    int s = (int)(w % g.fS);
+    long long t = w / g.fS;
     int qp = (int)(t % g.nTq2);
     it.is_text = 1;
     it.bh = (int)(t / g.nTq2);
@@ -279,8 +289,8 @@ CLEAR_HD PairItem decode_pair(const Geom& g, long long w) {
     it.x0 = 0;
     it.validB = (it.q0 + kTile) < g.n_text;
     it.split = s;
-    it.c_begin = s * g.cps;
-    it.c_end = imin(g.nC, (s + 1) * g.cps);
+    it.c_begin = s * g.fcps;
+    it.c_end = imin(g.fnC, (s + 1) * g.fcps);
   } else {
     long long u = w - g.n_txt_pairs;
     int blk = (int)(u % g.nQ2);
@@ -296,9 +306,10 @@ CLEAR_HD PairItem decode_pair(const Geom& g, long long w) {
   return it;
 }
 
-// Union key tiles of a pair, with per-half need / full flags. Image blocks visit the text chunks,
-// then band by band the 16-column rectangles covering the union of both halves' windows; a
-// rectangle is needed by a half iff some (query of that half, key of the rectangle) pair is kept.
+// Union key tiles of a pair (64 keys each), with per-half need / full flags. Image blocks visit the
+// 64-token text chunks, then band by band (4 key rows) the 16-column rectangles covering the union
+// of both halves' windows; a tile is needed by a half iff some (query of that half, key of the
+// tile) pair is kept.
 struct PairKeyIter {
   const int* wtab;
   int wtab_n;
@@ -321,7 +332,7 @@ struct PairKeyIter {
       return;
     }
     lin_next = 0;
-    lin_end = g.nTk;
+    lin_end = g.fnTk;
     y0 = it.q0; x0 = it.x0;
     xl = imin(x0 + kQW - 1, W - 1);
     yA0 = y0; yAl = imin(y0 + kQH - 1, H - 1);
@@ -329,7 +340,7 @@ struct PairKeyIter {
     const int ylast = validB ? yBl : yAl;
     ky_begin = imax(0, y0 - (r - 1));
     ky_end = imin(H - 1, ylast + (r - 1));
-    band_ky = ky_begin - kKH;
+    band_ky = ky_begin - kFKH;
     kx = 1; kx_end = 0;
   }
 
@@ -338,9 +349,9 @@ struct PairKeyIter {
   CLEAR_HD bool advance_band() {
     const int ylast = validB ? yBl : yAl;
     while (true) {
-      band_ky += kKH;
+      band_ky += kFKH;
       if (band_ky > ky_end) return false;
-      const int band_last = imin(band_ky + kKH - 1, H - 1);
+      const int band_last = imin(band_ky + kFKH - 1, H - 1);
       const int dmin = imax(0, imax(y0 - band_last, band_ky - ylast));
       const int w = hw(dmin);
       if (w < 0) continue;
@@ -350,27 +361,27 @@ struct PairKeyIter {
     }
   }
 
-  // need / full of rectangle [ky, ky+8) x [kx, kx+16) for query rows [qa, qb], columns [x0, xl].
+  // need / full of rectangle [ky, ky+4) x [kx, kx+16) for query rows [qa, qb], columns [x0, xl].
   CLEAR_HD int half_flags(int ky, int kxx, int qa, int qb, int need_bit, int full_bit) const {
-    const int kyl = imin(ky + kKH - 1, H - 1);
+    const int kyl = imin(ky + kFKH - 1, H - 1);
     const int kxl = imin(kxx + kKW - 1, W - 1);
     const int dy = imax(0, imax(qa - kyl, ky - qb));
     const int dx = imax(0, imax(x0 - kxl, kxx - xl));
     if (dy * dy + dx * dx >= r * r) return 0;
-    const bool inside = (ky + kKH - 1 <= H - 1) && (kxx + kKW - 1 <= W - 1);
-    const int mdy = imax(ky + kKH - 1 - qa, qb - ky);
+    const bool inside = (ky + kFKH - 1 <= H - 1) && (kxx + kKW - 1 <= W - 1);
+    const int mdy = imax(ky + kFKH - 1 - qa, qb - ky);
     const int mdx = imax(kxx + kKW - 1 - x0, xl - kxx);
     return need_bit | ((inside && mdy * mdy + mdx * mdx < r * r) ? full_bit : 0);
   }
 
   CLEAR_HD bool next(KeyTile* t) {
     if (lin_next < lin_end) {
-      const int a = lin_next * kTile;
+      const int a = lin_next * kFChunk;
       const int lim = is_text ? T : n_text;
       t->kind = kLinear;
       t->a = a;
-      t->b = imin(kTile, lim - a);
-      const int full = (t->b == kTile);
+      t->b = imin(kFChunk, lim - a);
+      const int full = (t->b == kFChunk);
       t->flags = kNeedA | (full ? kFullA : 0) | (validB ? (kNeedB | (full ? kFullB : 0)) : 0);
       ++lin_next;
       return true;

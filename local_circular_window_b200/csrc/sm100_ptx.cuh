@@ -22,6 +22,37 @@ enum DeviceError : int {
 
 // Defined once per library (single translation unit).
 __device__ int g_clear_device_error = 0;
+// Context of the first expired wait: {code, site, block, thread, parity, ctx0, ctx1, ctx2}.
+__device__ int g_clear_device_diag[8];
+// The same record for the first expiry at each wait site (0..31), for diagnosis.
+__device__ int g_clear_device_diag_sites[32][8];
+
+// Records an expired wait (first one wins) and raises the CTA's abort flag.
+__device__ __forceinline__ void record_timeout(volatile int* abort_flag, int err_code, int site, int parity, int c0,
+                                               int c1, int c2) {
+  *abort_flag = 1;
+  const int si = site & 31;
+  if (atomicCAS(&g_clear_device_diag_sites[si][0], 0, err_code) == 0) {
+    g_clear_device_diag_sites[si][1] = site;
+    g_clear_device_diag_sites[si][2] = blockIdx.x;
+    g_clear_device_diag_sites[si][3] = threadIdx.x;
+    g_clear_device_diag_sites[si][4] = parity;
+    g_clear_device_diag_sites[si][5] = c0;
+    g_clear_device_diag_sites[si][6] = c1;
+    g_clear_device_diag_sites[si][7] = c2;
+  }
+  if (atomicCAS(&g_clear_device_error, 0, err_code) == 0) {
+    g_clear_device_diag[0] = err_code;
+    g_clear_device_diag[1] = site;
+    g_clear_device_diag[2] = blockIdx.x;
+    g_clear_device_diag[3] = threadIdx.x;
+    g_clear_device_diag[4] = parity;
+    g_clear_device_diag[5] = c0;
+    g_clear_device_diag[6] = c1;
+    g_clear_device_diag[7] = c2;
+    __threadfence();
+  }
+}
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
@@ -85,15 +116,15 @@ struct PollWatchdog {
   uint64_t t0;
   uint32_t idle;
   __device__ __forceinline__ void start() { t0 = globaltimer_ns(); idle = 0; }
-  __device__ __forceinline__ bool tick(bool progressed, volatile int* abort_flag, int err_code) {
+  __device__ __forceinline__ bool tick(bool progressed, volatile int* abort_flag, int err_code, int site = 0,
+                                       int c0 = 0, int c1 = 0, int c2 = 0) {
     if (progressed) { idle = 0; return true; }
     if (++idle == 1) t0 = globaltimer_ns();
     if (idle > 2) __nanosleep(20);  // leave issue slots to the softmax warps of this sub-partition
     if ((idle & 255u) == 0) {
       if (*abort_flag) return false;
       if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        *abort_flag = 1;
-        atomicCAS(&g_clear_device_error, 0, err_code);
+        record_timeout(abort_flag, err_code, site, -1, c0, c1, c2);
         return false;
       }
     }
@@ -104,7 +135,7 @@ struct PollWatchdog {
 // Bounded wait for the phase with the given parity to complete. `abort_flag` (shared memory)
 // lets every role of a CTA give up quickly once one of them has timed out.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int err_code) {
+                                          int err_code, int site = 0, int c0 = 0, int c1 = 0) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -114,8 +145,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if ((++spins & 255u) == 0) {
       if (*abort_flag) return false;
       if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        *abort_flag = 1;
-        atomicCAS(&g_clear_device_error, 0, err_code);
+        record_timeout(abort_flag, err_code, site, (int)parity, c0, c1, (int)(a & 0xffff));
         return false;
       }
     }

@@ -9,7 +9,8 @@ import pytest
 import local_circular_window_b200 as L
 import oracle
 
-KQH, KQW, KKH, KKW, TILE = 8, 16, 8, 16, 128
+KQH, KQW, KKH, KKW, TILE = 8, 16, 4, 16, 128
+KCHUNK = 64  # forward key tiles: 64-token chunks or 4 x 16 rectangles
 
 
 def _keys_of_tile(tile, n_text, H, W, T):
@@ -28,7 +29,7 @@ def _raw_keys_of_tile(tile, n_text, H, W):
     """All 128 slots of a tile, None where the slot is outside the grid / past the valid count."""
     kind, a, b, flags = tile
     if kind == 0:
-        return [a + c if c < b else None for c in range(TILE)]
+        return [a + c if c < b else None for c in range(KCHUNK)]
     out = []
     for y in range(a, a + KKH):
         for x in range(b, b + KKW):
@@ -103,7 +104,7 @@ def test_pair_counts(n_text, H, W, r):
     products = 0
     for i in range(n_txt_items + n_img_items):
         products += sum(((t[3] & 1) != 0) + ((t[3] & 2) != 0) for t in L.item_tiles(p, i)[1])
-    assert executed == products * TILE * TILE
+    assert executed == products * TILE * KCHUNK
 
 
 def test_radius_beyond_diagonal_is_clamped_to_full_attention():
@@ -118,5 +119,5 @@ def test_split_shape_at_8k():
     p = L.make_params(1, 24, 512, 512, 512, 128, 8)
     n_txt_items, n_img_items, S, cps = L.forward_shape(p)
     assert n_img_items == 24 * (512 // 16) * (512 // 16)
-    assert S * cps >= (512 + 512 * 512 + 127) // 128 and S <= 32
+    assert S * cps >= (512 + 512 * 512 + 63) // 64 and S <= 32
     assert n_txt_items == 24 * 2 * S
