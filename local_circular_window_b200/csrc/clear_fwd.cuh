@@ -12,15 +12,20 @@
 // and multiplied by whichever halves reach it.
 //   warps 0-3   softmax / epilogue of half A (thread t owns query row t = TMEM lane t);
 //   warps 4-7   softmax / epilogue of half B;
-//   warp 8      TMA producer: Q of both halves once per pair, K and V tiles into 4-slot rings;
+//   warp 8      TMA producer: Q of both halves once per pair, K and V tiles into 4-slot rings. It
+//               enumerates each union tile once and publishes its descriptor (kind, origin, per-half
+//               need / full bits, last-of-pair bit, head) in a 16-entry shared ring that the V
+//               stream and both MMA issuers read, so nobody else re-runs the enumeration;
 //   warps 9/10  MMA issuers, one per half. Each polls two walks over the pair's union tiles: the
 //               QK walk issues S_j = Q K_j^T into one of two 64-column TMEM buffers (up to one
-//               needed tile ahead of P V); the PV walk issues O += P_j V_j once the softmax has
-//               written P_j over S_j (bf16, in TMEM; A operand from TMEM). Tiles a half does not
-//               need are still observed (their "full" phase) and released by that half, so each
-//               half sees every phase of every ring slot in order, which is what makes the
-//               parity-based barrier waits exact. Polling (instead of blocking) keeps either walk
-//               from holding up the other, so every wait depends only on earlier tiles;
+//               needed tile ahead of P V) and posts the tile to its softmax through a two-slot
+//               mailbox; the PV walk issues O += P_j V_j once the softmax has written P_j over S_j
+//               (bf16, in TMEM; A operand from TMEM). Tiles a half does not need are still
+//               observed (their "full" phase) and released by that half, so each half sees every
+//               phase of every ring slot in order, which keeps the parity-based waits exact.
+//               Polling (instead of blocking) keeps either walk from holding up the other, so
+//               every wait depends only on earlier tiles. The end of a pair is posted to the
+//               softmax as a mailbox message;
 //   warp 11     idle (it completes the third warpgroup, whose registers go to the softmax).
 // TMEM columns of half h: S buffers [256h, 256h+64) and [256h+64, 256h+128), O [256h+128, 256h+256).
 // The running max is rescaled lazily: O and l are only rescaled when a row's max grows by more
@@ -44,7 +49,10 @@ constexpr uint32_t kRegsLow = 72;
 constexpr uint32_t kRegsHigh = 216;
 static_assert(2 * 128 * kRegsHigh + 128 * kRegsLow <= 384 * 168, "register split exceeds the launch allocation");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-constexpr int kLastTile = 16;              // mailbox flag: last needed tile of the half in this pair
+constexpr int kTileRing = 16;              // union tile descriptors in flight (producer -> others)
+// Mailbox message kinds (issuer -> softmax); tiles use their KeyKind (kLinear / kRect).
+constexpr int kMsgEndPair = 2;             // the half's last tile of the current pair was posted
+constexpr int kMsgEndAll = 3;              // no more pairs for this CTA
 
 struct FwdParams {
   Geom g;
@@ -73,12 +81,14 @@ struct FwdLayout {
   static constexpr int bVEmpty = bVFull + kVStages;      // + slot
   static constexpr int bSFull = bVEmpty + kVStages;      // + 2 * half + buffer
   static constexpr int bPFull = bSFull + 4;              // + 2 * half + buffer
-  static constexpr int bInfo = bPFull + 4;               // + 2 * half + buffer
-  static constexpr int bODone = bInfo + 4;               // + half: last P V of the half's pair done
+  static constexpr int bMsgFull = bPFull + 4;            // + 2 * half + slot: mailbox message posted
+  static constexpr int bMsgEmpty = bMsgFull + 4;         // + 2 * half + slot: mailbox slot read
+  static constexpr int bODone = bMsgEmpty + 4;           // + half: last P V of the half's pair done
   static constexpr int bOReady = bODone + 2;             // + half: every P V done (one phase per tile)
   static constexpr int kNumBars = bOReady + 2;
-  static constexpr int kInfo = kBars + kNumBars * 8;     // int4[2][2]: {kind, a, b, flags | kLastTile}
-  static constexpr int kMisc = kInfo + 64;
+  static constexpr int kMsg = kBars + kNumBars * 8;      // int4[2][2] mailbox: {kind, a, b, flags | ordinal << 8}
+  static constexpr int kRing = kMsg + 64;                // int4[kTileRing]: {kind | flags << 4 | last << 12, a, b, bh}
+  static constexpr int kMisc = kRing + kTileRing * 16;
   static constexpr int kWTab = kMisc + 16;               // int[kMaxRTable] (tile enumeration)
   static constexpr int kHwTab = kWTab + kMaxRTable * 4;  // int16[hw_table_size(r, H)] (masks)
   static constexpr int kFixed = kHwTab + 1024;           // + slack for 1024-byte alignment
@@ -117,7 +127,8 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   int* wtab = reinterpret_cast<int*>(smem + L::kWTab);
   int16_t* hwtab = reinterpret_cast<int16_t*>(smem + L::kHwTab);
-  int4* info = reinterpret_cast<int4*>(smem + L::kInfo);
+  int4* msg = reinterpret_cast<int4*>(smem + L::kMsg);
+  int4* ring = reinterpret_cast<int4*>(smem + L::kRing);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -137,7 +148,8 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
     for (int i = 0; i < 4; ++i) {
       mbar_init(&bars[L::bSFull + i], 1);
       mbar_init(&bars[L::bPFull + i], 128);
-      mbar_init(&bars[L::bInfo + i], 1);
+      mbar_init(&bars[L::bMsgFull + i], 1);
+      mbar_init(&bars[L::bMsgEmpty + i], 128);
     }
     for (int h = 0; h < 2; ++h) {
       mbar_init(&bars[L::bODone + h], 1);
@@ -171,16 +183,22 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
       tma_prefetch_desc(&tm_v_lin); tma_prefetch_desc(&tm_v_img);
       long long wq = blockIdx.x;
       uint32_t q_loads = 0;
-      long long wk = blockIdx.x, wv = blockIdx.x;
-      PairItem itk{}, itv{};
-      PairKeyIter kik, kiv;
-      KeyTile tk{}, tv{};
-      bool kval = wk < p.n_work, vval = kval;
-      if (kval) { itk = decode_pair(g, wk); kik.init(g, itk, wtab, wtn); kik.next(&tk); itv = itk; kiv = kik; tv = tk; }
+      // K stream: the current union tile and a one-tile lookahead (for the last-of-pair bit).
+      long long wk = blockIdx.x;
+      PairItem itk{};
+      PairKeyIter kik;
+      KeyTile tcur{}, tnext{};
+      bool kval = wk < p.n_work, next_in_pair = false;
+      if (kval) {
+        itk = decode_pair(g, wk);
+        kik.init(g, itk, wtab, wtn);
+        kik.next(&tcur);
+        next_in_pair = kik.next(&tnext);
+      }
       uint32_t Gk = 0, Gv = 0;
       PollWatchdog wd;
       wd.start();
-      while (wq < p.n_work || kval || vval) {
+      while (wq < p.n_work || kval || Gv < Gk) {
         bool prog = false;
         if (wq < p.n_work && (q_loads == 0 || mbar_test(&bars[L::bQEmpty], (q_loads - 1) & 1))) {
           const PairItem it = decode_pair(g, wq);
@@ -200,33 +218,40 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
           wq += stride;
           prog = true;
         }
-        if (kval) {
+        if (kval && Gk - Gv < (uint32_t)kTileRing) {
           const uint32_t ks = Gk % kKStages;
           if (mbar_test(&bars[L::bKEmpty + ks], ((Gk / kKStages) & 1) ^ 1)) {
+            // Publish the descriptor before the load: the K barrier's completion makes it visible.
+            ring[Gk % kTileRing] = make_int4(tcur.kind | (tcur.flags << 4) | (next_in_pair ? 0 : (1 << 12)), tcur.a,
+                                             tcur.b, itk.bh);
             mbar_arrive_expect_tx(&bars[L::bKFull + ks], L::kKVTileBytes);
-            load_kv64<D>(smem + L::kK + ks * L::kKVTileBytes, &tm_k_lin, &tm_k_img, &bars[L::bKFull + ks], tk.kind,
-                         tk.a, tk.b, itk.bh);
+            load_kv64<D>(smem + L::kK + ks * L::kKVTileBytes, &tm_k_lin, &tm_k_img, &bars[L::bKFull + ks], tcur.kind,
+                         tcur.a, tcur.b, itk.bh);
             ++Gk;
-            if (!kik.next(&tk)) {
+            if (next_in_pair) {
+              tcur = tnext;
+              next_in_pair = kik.next(&tnext);
+            } else {
               wk += stride;
               kval = wk < p.n_work;
-              if (kval) { itk = decode_pair(g, wk); kik.init(g, itk, wtab, wtn); kik.next(&tk); }
+              if (kval) {
+                itk = decode_pair(g, wk);
+                kik.init(g, itk, wtab, wtn);
+                kik.next(&tcur);
+                next_in_pair = kik.next(&tnext);
+              }
             }
             prog = true;
           }
         }
-        if (vval && Gv < Gk) {
+        if (Gv < Gk) {
           const uint32_t vs = Gv % kVStages;
           if (mbar_test(&bars[L::bVEmpty + vs], ((Gv / kVStages) & 1) ^ 1)) {
+            const int4 e = ring[Gv % kTileRing];
             mbar_arrive_expect_tx(&bars[L::bVFull + vs], L::kKVTileBytes);
-            load_kv64<D>(smem + L::kV + vs * L::kKVTileBytes, &tm_v_lin, &tm_v_img, &bars[L::bVFull + vs], tv.kind,
-                         tv.a, tv.b, itv.bh);
+            load_kv64<D>(smem + L::kV + vs * L::kKVTileBytes, &tm_v_lin, &tm_v_img, &bars[L::bVFull + vs], e.x & 15,
+                         e.y, e.z, e.w);
             ++Gv;
-            if (!kiv.next(&tv)) {
-              wv += stride;
-              vval = wv < p.n_work;
-              if (vval) { itv = decode_pair(g, wv); kiv.init(g, itv, wtab, wtn); kiv.next(&tv); }
-            }
             prog = true;
           }
         }
@@ -244,88 +269,98 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
       const int need_bit = h == 0 ? kNeedA : kNeedB;
       const uint32_t q_addr = smem_u32(smem + L::kQ + h * L::kQTileBytes);
       const uint32_t o_tm = tmem + L::o_col(h);
-      // QK walk over the union tiles (union index Gq, needed-tile counter nqk).
-      long long wq = blockIdx.x;
-      uint32_t items = 0, Gq = 0, nqk = 0;
-      PairKeyIter ki;
-      KeyTile t{};
-      bool in_item = false, q_seen = false, have = false, done = false;
-      int jq = 0, nitem = 0;
+      // Shared-memory matrix descriptors, advanced per 16-element K step with plain adds.
+      const uint64_t qdesc = smem_desc_sw128(q_addr, 16, 1024);
+      const uint64_t kdesc0 = smem_desc_sw128(smem_u32(smem + L::kK), 16, 1024);
+      const uint64_t vdesc0 = smem_desc_sw128(smem_u32(smem + L::kV), L::kKVBlock, 1024);
+      const uint32_t n_pairs = (uint32_t)((p.n_work - blockIdx.x + stride - 1) / stride);
+      // QK walk over the union tiles (union index Gq); pairs are observed in order.
+      uint32_t pair = 0, Gq = 0, nqk = 0, nmsg = 0;
+      bool q_seen = false, had = false, end_pending = false, all_posted = false;
       // PV walk: union index Gp; up to two needed tiles whose Q K^T is issued and P V is not.
       uint32_t Gp = 0, npv = 0;
       uint32_t pend_G[2] = {0, 0};
-      int pend_fl[2] = {0, 0};  // bit 0: first of item, bit 1: last of item
+      int pend_fl[2] = {0, 0};  // bit 0: first of the pair (overwrite O), bit 1: commit o_done after it
       int pend = 0;
       PollWatchdog wd;
       wd.start();
-      while (!done || Gp < Gq) {
+      while (!all_posted || Gp < Gq || pend > 0) {
         bool prog = false;
         // ---- QK walk step
-        if (!done && !in_item) {
-          if (wq >= p.n_work) {
-            done = true;
-          } else {
-            const PairItem it = decode_pair(g, wq);
-            int nu, na, nb;
-            count_pair_tiles(g, it, wtab, wtn, &nu, &na, &nb);
-            nitem = h == 0 ? na : nb;
-            jq = 0;
-            ki.init(g, it, wtab, wtn);
-            in_item = true;
-            q_seen = false;
-            have = false;
-          }
-        }
-        if (in_item && !q_seen && mbar_test(&bars[L::bQFull], items & 1)) {
-          q_seen = true;  // every half observes every Q phase; a half without queries here
-          if (nitem == 0) mbar_arrive(&bars[L::bQEmpty]);  // releases Q at once
-          prog = true;
-        }
-        if (in_item && q_seen && !have) {
-          if (ki.next(&t)) {
-            have = true;
-          } else {
-            in_item = false;
-            ++items;
-            wq += stride;
+        if (end_pending || (pair >= n_pairs && !all_posted)) {
+          // Post an end-of-pair (or end-of-work) message once the mailbox slot is free.
+          const uint32_t ms = nmsg & 1;
+          if (mbar_test(&bars[L::bMsgEmpty + 2 * h + ms], ((nmsg >> 1) & 1) ^ 1)) {
+            msg[2 * h + ms] = make_int4(end_pending ? kMsgEndPair : kMsgEndAll, 0, 0, 0);
+            mbar_arrive(&bars[L::bMsgFull + 2 * h + ms]);
+            ++nmsg;
+            if (end_pending) end_pending = false; else all_posted = true;
             prog = true;
           }
-        }
-        if (have) {
-          const uint32_t ks = Gq % kKStages;
-          const bool needed = (t.flags & need_bit) != 0;
-          if ((!needed || pend < 2) && mbar_test(&bars[L::bKFull + ks], (Gq / kKStages) & 1)) {
-            if (!needed) {
-              mbar_arrive(&bars[L::bKEmpty + ks]);  // observed and released
-            } else {
-              const bool last = (jq == nitem - 1);
-              const uint32_t b = nqk & 1;
-              // Hand the tile to this half's softmax. Slot b was last used by needed tile nqk - 2,
-              // whose P has been consumed (its P V is issued before this Q K^T can be).
-              info[2 * h + b] = make_int4(t.kind, t.a, t.b, t.flags | (last ? kLastTile : 0));
-              mbar_arrive(&bars[L::bInfo + 2 * h + b]);
-              tc_fence_after();
-              const uint32_t k_addr = smem_u32(smem + L::kK + ks * L::kKVTileBytes);
-              #pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t qoff = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-                const uint32_t koff = (kk >> 2) * L::kKVBlock + (kk & 3) * 32;
-                umma_ss(tmem + L::s_col(h, b), smem_desc_sw128(q_addr + qoff, 16, 1024),
-                        smem_desc_sw128(k_addr + koff, 16, 1024), idesc_qk, kk > 0);
-              }
-              umma_commit(&bars[L::bSFull + 2 * h + b]);
-              umma_commit(&bars[L::bKEmpty + ks]);
-              if (last) umma_commit(&bars[L::bQEmpty]);
-              const int slot = (npv + pend) & 1;
-              pend_G[slot] = Gq;
-              pend_fl[slot] = (jq == 0 ? 1 : 0) | (last ? 2 : 0);
-              ++pend;
-              ++nqk;
-              ++jq;
+        } else if (pair < n_pairs) {
+          if (!q_seen) {
+            if (mbar_test(&bars[L::bQFull], pair & 1)) {  // every half observes every Q phase
+              q_seen = true;
+              had = false;
+              prog = true;
             }
-            ++Gq;
-            have = false;
-            prog = true;
+          } else {
+            const uint32_t ks = Gq % kKStages;
+            if (mbar_test(&bars[L::bKFull + ks], (Gq / kKStages) & 1)) {
+              const int4 e = ring[Gq % kTileRing];
+              const int flags = (e.x >> 4) & 255;
+              const bool last_of_pair = (e.x >> 12) & 1;
+              const bool needed = (flags & need_bit) != 0;
+              const uint32_t ms = nmsg & 1;
+              bool done_tile = false;
+              if (!needed) {
+                mbar_arrive(&bars[L::bKEmpty + ks]);  // observed and released
+                done_tile = true;
+              } else if (pend < 2 && mbar_test(&bars[L::bMsgEmpty + 2 * h + ms], ((nmsg >> 1) & 1) ^ 1)) {
+                const uint32_t b = nqk & 1;
+                msg[2 * h + ms] = make_int4(e.x & 15, e.y, e.z, flags | (int)(pair << 8));
+                mbar_arrive(&bars[L::bMsgFull + 2 * h + ms]);
+                ++nmsg;
+                tc_fence_after();
+                const uint64_t kd = kdesc0 + (uint64_t)((ks * L::kKVTileBytes) >> 4);
+                #pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                  const uint32_t qoff = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+                  const uint32_t koff = ((kk >> 2) * L::kKVBlock + (kk & 3) * 32) >> 4;
+                  umma_ss(tmem + L::s_col(h, b), qdesc + qoff, kd + koff, idesc_qk, kk > 0);
+                }
+                umma_commit(&bars[L::bSFull + 2 * h + b]);
+                umma_commit(&bars[L::bKEmpty + ks]);
+                const int slot = (npv + pend) & 1;
+                pend_G[slot] = Gq;
+                pend_fl[slot] = had ? 0 : 1;
+                ++pend;
+                ++nqk;
+                had = true;
+                done_tile = true;
+              }
+              if (done_tile) {
+                ++Gq;
+                prog = true;
+                if (last_of_pair) {
+                  // Pair finished for this half: release Q, arrange o_done, tell the softmax.
+                  if (had) {
+                    umma_commit(&bars[L::bQEmpty]);
+                    // o_done follows this half's last P V of the pair: mark it if still pending
+                    // (it is the most recent needed tile), else commit now.
+                    if (pend > 0)
+                      pend_fl[(npv + pend - 1) & 1] |= 2;
+                    else
+                      umma_commit(&bars[L::bODone + h]);
+                    end_pending = true;
+                  } else {
+                    mbar_arrive(&bars[L::bQEmpty]);
+                  }
+                  ++pair;
+                  q_seen = false;
+                }
+              }
+            }
           }
         }
         // ---- PV walk step (tiles the QK walk has passed, in order)
@@ -344,12 +379,12 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
             if (mbar_test(&bars[L::bPFull + 2 * h + b], (npv >> 1) & 1) &&
                 mbar_test(&bars[L::bVFull + vs], (Gp / kVStages) & 1)) {
               tc_fence_after();
-              const uint32_t v_addr = smem_u32(smem + L::kV + vs * L::kKVTileBytes);
+              const uint64_t vd = vdesc0 + (uint64_t)((vs * L::kKVTileBytes) >> 4);
               const uint32_t s_tm = tmem + L::s_col(h, b);
               const bool first = pend_fl[slot] & 1;
               #pragma unroll
               for (int kk = 0; kk < kFChunk / 16; ++kk)
-                umma_ts(o_tm, s_tm + kk * 8, smem_desc_sw128(v_addr + kk * 2048, L::kKVBlock, 1024), idesc_pv,
+                umma_ts(o_tm, s_tm + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv,
                         (!first || kk > 0) ? 1u : 0u);
               umma_commit(&bars[L::bVEmpty + vs]);
               umma_commit(&bars[L::bOReady + h]);
@@ -362,7 +397,7 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
           }
         }
         if (!wd.tick(prog, abort_flag, kDevTimeoutMma, 2 + h, (int)Gq, (int)(Gp | (npv << 16)),
-                     pend | (have ? 4 : 0) | (done ? 8 : 0) | (q_seen ? 16 : 0) | ((int)items << 8))) break;
+                     pend | (end_pending ? 4 : 0) | (all_posted ? 8 : 0) | (q_seen ? 16 : 0) | ((int)pair << 8))) break;
       }
     }
     __syncwarp();
@@ -376,36 +411,97 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t o_tm = tmem + lane_base + L::o_col(half);
     const int full_bit = half == 0 ? kFullA : kFullB;
-    uint32_t nq = 0, n_out = 0;
+    uint32_t nq = 0, n_out = 0, nmsg = 0;
     const float sl2 = p.scale_log2;
-    for (long long w = blockIdx.x; w < p.n_work; w += stride) {
-      const PairItem it = decode_pair(g, w);
-      if (half == 1 && !it.validB) continue;
-      int yq = 0, xq = 0, tq = 0;
-      bool row_valid;
-      if (it.is_text) {
-        tq = it.q0 + half * kTile + row;
-        row_valid = tq < g.n_text;
-      } else {
-        yq = it.q0 + half * kQH + (row >> 4);
-        xq = it.x0 + (row & 15);
-        row_valid = (yq < g.H) && (xq < g.W);
-      }
-      float m_used = -INFINITY;  // running max, scaled log2 units
-      float l = 0.f;
-      int j = 0;
-      bool last = false;
-      while (!last) {
-        const uint32_t b = nq & 1, ph = (nq >> 1) & 1;
-        if (!mbar_wait(&bars[L::bInfo + 2 * half + b], ph, abort_flag, kDevTimeoutSoftmax, 10 + half, (int)nq, j))
+    // Per-pair state, set up at the pair's first tile.
+    PairItem it{};
+    int yq = 0, xq = 0, tq = 0;
+    bool row_valid = false;
+    float m_used = -INFINITY;  // running max, scaled log2 units
+    float l = 0.f;
+    int j = 0;
+    while (true) {
+      const uint32_t ms = nmsg & 1;
+      if (!mbar_wait(&bars[L::bMsgFull + 2 * half + ms], (nmsg >> 1) & 1, abort_flag, kDevTimeoutSoftmax, 10 + half,
+                     (int)nmsg, j))
+        goto softmax_done;
+      const int4 mv = msg[2 * half + ms];
+      mbar_arrive(&bars[L::bMsgEmpty + 2 * half + ms]);
+      ++nmsg;
+      if (mv.x == kMsgEndAll) break;
+      if (mv.x == kMsgEndPair) {
+        // ---- epilogue: wait for this half's last P V, then write O / l (or the split partial)
+        if (!mbar_wait(&bars[L::bODone + half], n_out & 1, abort_flag, kDevTimeoutSoftmax, 16 + half, (int)nq,
+                       (int)n_out))
           goto softmax_done;
-        const int4 ti = info[2 * half + b];
-        KeyTile t;
-        t.kind = ti.x;
-        t.a = ti.y;
-        t.b = ti.z;
-        t.flags = ti.w;
-        last = (ti.w & kLastTile) != 0;
+        ++n_out;
+        tc_fence_after();
+        if (it.is_text) {
+          const size_t prow = ((size_t)it.split * g.BH + it.bh) * g.n_text + (row_valid ? tq : 0);
+          float* dst = p.opart + prow * D;
+          #pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(o_tm + c * 32, ov);
+            tmem_wait_ld();
+            if (row_valid) {
+              float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+              #pragma unroll
+              for (int e = 0; e < 8; ++e)
+                d4[e] = make_float4(__uint_as_float(ov[4 * e]), __uint_as_float(ov[4 * e + 1]),
+                                    __uint_as_float(ov[4 * e + 2]), __uint_as_float(ov[4 * e + 3]));
+            }
+          }
+          if (row_valid) p.ml[prow] = make_float2(m_used, l);
+        } else {
+          const size_t orow = (size_t)it.bh * g.T + g.n_text + (size_t)yq * g.W + xq;
+          const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+          __nv_bfloat16* dst = p.o + orow * D;
+          #pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(o_tm + c * 32, ov);
+            tmem_wait_ld();
+            if (row_valid) {
+              uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+              #pragma unroll
+              for (int e = 0; e < 4; ++e)
+                d4[e] = make_uint4(
+                    pack_bf16x2(__uint_as_float(ov[8 * e + 0]) * inv_l, __uint_as_float(ov[8 * e + 1]) * inv_l),
+                    pack_bf16x2(__uint_as_float(ov[8 * e + 2]) * inv_l, __uint_as_float(ov[8 * e + 3]) * inv_l),
+                    pack_bf16x2(__uint_as_float(ov[8 * e + 4]) * inv_l, __uint_as_float(ov[8 * e + 5]) * inv_l),
+                    pack_bf16x2(__uint_as_float(ov[8 * e + 6]) * inv_l, __uint_as_float(ov[8 * e + 7]) * inv_l));
+            }
+          }
+          if (row_valid) p.lse[orow] = (m_used + __log2f(l)) * 0.69314718055994530942f;
+        }
+        // The next pair's first P V overwrites O; it waits for this half's next P, which is
+        // signalled after these TMEM reads.
+        tc_fence_before();
+        j = 0;
+        continue;
+      }
+      // ---- a tile: {kind, a, b, flags | pair ordinal << 8}
+      KeyTile t;
+      t.kind = mv.x;
+      t.a = mv.y;
+      t.b = mv.z;
+      t.flags = mv.w & 255;
+      if (j == 0) {  // first tile of a pair: its geometry, fresh statistics
+        it = decode_pair(g, blockIdx.x + (long long)(mv.w >> 8) * stride);
+        if (it.is_text) {
+          tq = it.q0 + half * kTile + row;
+          row_valid = tq < g.n_text;
+        } else {
+          yq = it.q0 + half * kQH + (row >> 4);
+          xq = it.x0 + (row & 15);
+          row_valid = (yq < g.H) && (xq < g.W);
+        }
+        m_used = -INFINITY;
+        l = 0.f;
+      }
+      {
+        const uint32_t b = nq & 1, ph = (nq >> 1) & 1;
         if (!mbar_wait(&bars[L::bSFull + 2 * half + b], ph, abort_flag, kDevTimeoutSoftmax, 12 + half, (int)nq, j))
           goto softmax_done;
         tc_fence_after();
@@ -499,53 +595,6 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
         ++nq;
         ++j;
       }
-      // ---- epilogue: wait for this half's last P V, then write O / l (or the split partial)
-      if (!mbar_wait(&bars[L::bODone + half], n_out & 1, abort_flag, kDevTimeoutSoftmax, 16 + half, (int)nq, (int)n_out))
-        goto softmax_done;
-      ++n_out;
-      tc_fence_after();
-      if (it.is_text) {
-        const size_t prow = ((size_t)it.split * g.BH + it.bh) * g.n_text + (row_valid ? tq : 0);
-        float* dst = p.opart + prow * D;
-        #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t ov[32];
-          tmem_ld32(o_tm + c * 32, ov);
-          tmem_wait_ld();
-          if (row_valid) {
-            float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
-            #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              d4[e] = make_float4(__uint_as_float(ov[4 * e]), __uint_as_float(ov[4 * e + 1]),
-                                  __uint_as_float(ov[4 * e + 2]), __uint_as_float(ov[4 * e + 3]));
-          }
-        }
-        if (row_valid) p.ml[prow] = make_float2(m_used, l);
-      } else {
-        const size_t orow = (size_t)it.bh * g.T + g.n_text + (size_t)yq * g.W + xq;
-        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-        __nv_bfloat16* dst = p.o + orow * D;
-        #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t ov[32];
-          tmem_ld32(o_tm + c * 32, ov);
-          tmem_wait_ld();
-          if (row_valid) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
-            #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              d4[e] = make_uint4(
-                  pack_bf16x2(__uint_as_float(ov[8 * e + 0]) * inv_l, __uint_as_float(ov[8 * e + 1]) * inv_l),
-                  pack_bf16x2(__uint_as_float(ov[8 * e + 2]) * inv_l, __uint_as_float(ov[8 * e + 3]) * inv_l),
-                  pack_bf16x2(__uint_as_float(ov[8 * e + 4]) * inv_l, __uint_as_float(ov[8 * e + 5]) * inv_l),
-                  pack_bf16x2(__uint_as_float(ov[8 * e + 6]) * inv_l, __uint_as_float(ov[8 * e + 7]) * inv_l));
-          }
-        }
-        if (row_valid) p.lse[orow] = (m_used + __log2f(l)) * 0.69314718055994530942f;
-      }
-      // The next pair's first P V overwrites O; it waits for this half's next P, which is
-      // signalled after these TMEM reads.
-      tc_fence_before();
     }
   softmax_done:;
   }
