@@ -93,6 +93,27 @@ CLEAR_API clear_status_t clear_attn_fwd(const clear_attn_params_t* params, const
                               size_t workspace_bytes, void* stream);
 
 /*
+ * Forward for callers that cannot allocate device memory: same inputs, outputs and results as
+ * clear_attn_fwd (up to the summation order of the text rows), but no workspace argument. The
+ * paper has no counterpart; this entry point exists for integration. Some callers cannot call
+ * cudaMalloc or hand out scratch buffers: a plugin invoked inside another framework's execution
+ * step, where allocating would break that framework's memory plan, or a serving loop that reserved
+ * all device memory up front. This call uses a scratch array of 32 MiB compiled into the library
+ * instead (a static __device__ array: every GPU that loads the library holds it until exit), and
+ * allocates nothing itself.
+ *   - The text-row split count is lowered until the split partials fit in the 32 MiB; if one split
+ *     of B * heads * n_text rows (4 * d + 8 bytes each) does not fit, the call returns
+ *     CLEAR_ERR_WORKSPACE and launches nothing.
+ *   - The first call on a device looks up the scratch array's device address (with that device
+ *     current); make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents. Nothing in it needs to
+ *     start at zero: every value a call reads there is written earlier in the same call. Calls
+ *     that overlap on the GPU (different streams, or different host threads) race on it.
+ */
+CLEAR_API clear_status_t clear_attn_fwd_noalloc(const clear_attn_params_t* params, const void* q, const void* k,
+                                      const void* v, void* o, float* lse, void* stream);
+
+/*
  * Backward of clear_attn_fwd with respect to q, k and v, given the upstream gradient dO and the
  * forward's o and lse (analytic softmax-attention gradient restricted to the mask):
  *   dV = P^T dO;  dP = dO V^T;  D = rowsum(dO o O);  dS = P o (dP - D);

@@ -52,6 +52,8 @@ _lib.clear_attn_bwd_workspace_size.restype = ctypes.c_size_t
 _lib.clear_attn_bwd_workspace_size.argtypes = [_P, ctypes.POINTER(_i)]
 _lib.clear_attn_fwd.restype = _i
 _lib.clear_attn_fwd.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+_lib.clear_attn_fwd_noalloc.restype = _i
+_lib.clear_attn_fwd_noalloc.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.clear_attn_bwd.restype = _i
 _lib.clear_attn_bwd.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 _lib.clear_attn_check.restype = _i

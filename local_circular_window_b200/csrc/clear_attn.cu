@@ -16,6 +16,11 @@
 
 using namespace clear;
 
+// Scratch of the allocation-free forward (clear_attn_fwd_noalloc): the text-row split partials.
+// Every device that loads this library holds these bytes until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
 namespace {
 
 constexpr int kVersion = 100;  // 0.1.0
@@ -189,6 +194,43 @@ clear_status_t launch_fwd(const Geom& g, const QKVMaps& m, void* o, float* lse, 
   return CLEAR_OK;
 }
 
+// Device address of g_noalloc_scratch on the current device. The symbol's name is only a host-side
+// stand-in; the address is looked up once per device, with that device current.
+struct NoAllocSlot {
+  std::once_flag once;
+  void* ptr = nullptr;
+  cudaError_t err = cudaSuccess;
+};
+constexpr int kMaxDevices = 64;
+NoAllocSlot g_noalloc_slots[kMaxDevices];
+
+clear_status_t noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CLEAR_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return CLEAR_ERR_UNSUPPORTED;
+  NoAllocSlot& slot = g_noalloc_slots[dev];
+  std::call_once(slot.once, [&slot] { slot.err = cudaGetSymbolAddress(&slot.ptr, g_noalloc_scratch); });
+  if (slot.err != cudaSuccess || slot.ptr == nullptr) return CLEAR_ERR_CUDA;
+  *out = slot.ptr;
+  return CLEAR_OK;
+}
+
+// The forward's schedule with its text-row split count lowered until the partials fit in the
+// static scratch; CLEAR_ERR_WORKSPACE when even one split does not fit.
+clear_status_t noalloc_geom(Geom* g) {
+  if (g->n_text == 0) return CLEAR_OK;
+  for (int cap = g->fS; cap >= 1; --cap) {
+    Geom t = *g;
+    choose_splits(t.fnC, 2 * kSplitTargetChunks, cap, &t.fS, &t.fcps);
+    t.n_txt_pairs = (long long)t.BH * t.nTq2 * t.fS;
+    if (fwd_workspace_layout(t).total <= kNoAllocScratchBytes) {
+      *g = t;
+      return CLEAR_OK;
+    }
+  }
+  return CLEAR_ERR_WORKSPACE;
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------------------------------------
@@ -241,6 +283,28 @@ clear_status_t clear_attn_fwd(const clear_attn_params_t* params, const void* q, 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return c.g.d == 128 ? launch_fwd<128>(c.g, maps, o, lse, workspace, num_sms, s)
                       : launch_fwd<64>(c.g, maps, o, lse, workspace, num_sms, s);
+}
+
+clear_status_t clear_attn_fwd_noalloc(const clear_attn_params_t* params, const void* q, const void* k,
+                                      const void* v, void* o, float* lse, void* stream) {
+  const Checked c = check_params(params);
+  if (c.st != CLEAR_OK) return c.st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return CLEAR_ERR_INVALID_ARG;
+  Geom g = c.g;
+  clear_status_t st = noalloc_geom(&g);
+  if (st != CLEAR_OK) return st;
+  int num_sms = 0;
+  st = check_device(&num_sms);
+  if (st != CLEAR_OK) return st;
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != CLEAR_OK) return st;
+  QKVMaps maps;
+  if (!make_fwd_maps(&maps, q, k, v, g)) return CLEAR_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return g.d == 128 ? launch_fwd<128>(g, maps, o, lse, scratch, num_sms, s)
+                    : launch_fwd<64>(g, maps, o, lse, scratch, num_sms, s);
 }
 
 clear_status_t clear_attn_bwd(const clear_attn_params_t* params, const void* q, const void* k,
