@@ -319,6 +319,7 @@ struct PairKeyIter {
   int ky_begin, ky_end;
   int lin_next, lin_end;
   int band_ky, kx, kx_end;
+  int band_step, n_bands;     // bands are visited ends-inward: 0, n-1, 1, n-2, ...
 
   CLEAR_HD void init(const Geom& g, const PairItem& it, const int* table = nullptr, int table_n = 0) {
     wtab = table;
@@ -329,6 +330,7 @@ struct PairKeyIter {
       lin_end = it.c_end;
       band_ky = 1; ky_end = 0; kx = 1; kx_end = 0;
       y0 = x0 = xl = yA0 = yAl = yB0 = yBl = 0; ky_begin = 0;
+      band_step = n_bands = 0;
       return;
     }
     lin_next = 0;
@@ -340,17 +342,24 @@ struct PairKeyIter {
     const int ylast = validB ? yBl : yAl;
     ky_begin = imax(0, y0 - (r - 1));
     ky_end = imin(H - 1, ylast + (r - 1));
-    band_ky = ky_begin - kFKH;
+    n_bands = (ky_end - ky_begin) / kFKH + 1;
+    band_step = 0;
+    band_ky = ky_begin;
     kx = 1; kx_end = 0;
   }
 
   CLEAR_HD int hw(int dy) const { return (dy < wtab_n) ? wtab[dy] : half_width(r, dy); }
 
+  // Next band with kept columns. The first and last bands are reached by one half only (the
+  // top ones by half A, the bottom ones by half B); alternating from both ends keeps both halves
+  // busy instead of leaving one idle at the start of the pair and the other at its end.
   CLEAR_HD bool advance_band() {
     const int ylast = validB ? yBl : yAl;
     while (true) {
-      band_ky += kFKH;
-      if (band_ky > ky_end) return false;
+      if (band_step >= n_bands) return false;
+      const int k = (band_step & 1) ? n_bands - 1 - (band_step >> 1) : (band_step >> 1);
+      ++band_step;
+      band_ky = ky_begin + k * kFKH;
       const int band_last = imin(band_ky + kFKH - 1, H - 1);
       const int dmin = imax(0, imax(y0 - band_last, band_ky - ylast));
       const int w = hw(dmin);
