@@ -15,6 +15,7 @@ full call.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -32,6 +33,29 @@ from clear_inputs import WORKLOADS, Workload, make_inputs  # noqa: E402
 
 METRIC = "CLEAR attn useful TFLOP/s & ms/call (bf16, 512² grid, r=8); % of TC peak"
 FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# DRAM traffic of clear_fwd_kernel<128> from one ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum) on the 8K r=8 shape cut to 2 heads (the full 24-head launch is too large
+# to capture), per head; heads are independent, so a full launch moves heads x this. Valid only
+# for the kernel sources it was taken on (hash below); any change to them reports null.
+FWD_TRAFFIC = {"8k_r8": {"bytes_per_head": (730.410752e6 + 139.224576e6) / 2, "src": "db9b720e774e7819"}}
+FWD_SOURCES = ("clear_fwd.cuh", "clear_sched.cuh", "clear_common.cuh", "sm100_ptx.cuh")
+
+
+def _fwd_src_hash():
+    h = hashlib.sha256()
+    for f in FWD_SOURCES:
+        with open(os.path.join(ROOT, "local_circular_window_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _fwd_traffic(wl):
+    rec = FWD_TRAFFIC.get(wl.name)
+    if rec is None or wl.heads != WORKLOADS[wl.name].heads or _fwd_src_hash() != rec["src"]:
+        return None
+    return rec["bytes_per_head"] * wl.B * wl.heads
 
 
 def _peaks():
@@ -331,7 +355,7 @@ def run_clear(args):
             "padded_tflops": executed / (kernel_ms * 1e-3) / 1e12,
             "useful_gflop_per_call": useful / 1e9, "executed_gflop_per_call": executed / 1e9,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": None,
+                         "frac": achieved / peak, "traffic": _fwd_traffic(wl),
                          "peak_source": f"{peak_kind} bf16 dense (burst; kernel timed alone)",
                          "kernel": "clear_fwd_kernel + clear_fwd_combine_kernel (one call, CUDA events)"},
             "e2e": e2e, "cpu_baseline": cpu, "bwd": bwd, "clocks": clocks,
