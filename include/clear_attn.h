@@ -138,6 +138,19 @@ CLEAR_API clear_status_t clear_attn_check(void* stream);
  * For diagnosis only; the layout may change between versions. */
 CLEAR_API void clear_attn_device_diag(int* out8);
 
+/* Self-test of the failure-detection path (the paper has no counterpart). Launches, on `stream`,
+ * one small kernel whose single waiting thread waits on a shared-memory barrier that nothing ever
+ * arrives on; after `limit_ms` milliseconds (1..5000) the wait gives up, records the expiry in the
+ * same device error word and diagnostic record the attention kernels use (code 5, wait site 31)
+ * and the kernel returns. Nothing faults or hangs, and the CUDA context stays usable. The caller
+ * then sees CLEAR_ERR_DEVICE_TIMEOUT from clear_attn_check(stream), which also clears the word,
+ * and the record from clear_attn_device_diag().
+ * Returns CLEAR_OK once the kernel is launched, CLEAR_ERR_INVALID_ARG for a limit outside 1..5000
+ * (checked before any CUDA call), CLEAR_ERR_UNSUPPORTED on a device other than sm_100,
+ * CLEAR_ERR_CUDA if the launch fails. It shares the device error word with every other call on
+ * the device: do not run it concurrently with attention calls whose status you need. */
+CLEAR_API clear_status_t clear_attn_selftest_expiry(int limit_ms, void* stream);
+
 /* ---------------------------------------------------------------------------------------------
  * Host-only scheduler queries (no GPU needed). They expose the tile enumeration the kernels use,
  * so its coverage can be checked against a brute-force mask on the CPU.

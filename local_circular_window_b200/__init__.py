@@ -10,7 +10,7 @@ import importlib
 _EXPORTS = {
     "CLEAR_OK", "ClearError", "ClearParams", "LIB_PATH", "bwd_workspace_size", "clear_attn_bwd",
     "clear_attn_check", "clear_attn_fwd", "device_diag", "forward_shape", "fwd_workspace_size", "header_functions",
-    "item_tiles", "lib", "make_params", "pair_counts", "status_string", "version",
+    "item_tiles", "lib", "make_params", "pair_counts", "selftest_expiry", "status_string", "version",
 }
 
 

@@ -58,6 +58,8 @@ _lib.clear_attn_bwd.restype = _i
 _lib.clear_attn_bwd.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 _lib.clear_attn_check.restype = _i
 _lib.clear_attn_check.argtypes = [_vp]
+_lib.clear_attn_selftest_expiry.restype = _i
+_lib.clear_attn_selftest_expiry.argtypes = [_i, _vp]
 _lib.clear_attn_device_diag.restype = None
 _lib.clear_attn_device_diag.argtypes = [ctypes.POINTER(_i)]
 _lib.clear_sched_forward_shape.restype = _i
@@ -211,3 +213,9 @@ def device_diag() -> list:
     out = (_i * 8)()
     _lib.clear_attn_device_diag(out)
     return list(out)
+
+
+def selftest_expiry(limit_ms: int, stream=None) -> int:
+    """Launches the failure-detection self-test (a wait that expires after limit_ms); returns the
+    launch status. clear_attn_check() then reports CLEAR_ERR_DEVICE_TIMEOUT."""
+    return _lib.clear_attn_selftest_expiry(int(limit_ms), _stream_ptr(stream))

@@ -231,6 +231,30 @@ clear_status_t noalloc_geom(Geom* g) {
   return CLEAR_ERR_WORKSPACE;
 }
 
+// One thread waits on a barrier that nothing arrives on, gives up after limit_ns and records the
+// expiry exactly as a timed-out wait of the attention kernels does (failure-detection self-test).
+__global__ void clear_selftest_expiry_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t a = smem_u32(&bar);
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(a, 0)) {
+      if (globaltimer_ns() - t0 > limit_ns) {
+        record_timeout(&abort_flag, kDevTimeoutOther, 31, 0, (int)(limit_ns / 1000000ull), 0, 0);
+        break;
+      }
+    }
+  }
+  __syncthreads();
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------------------------------------
@@ -362,6 +386,16 @@ clear_status_t clear_attn_check(void* stream) {
 void clear_attn_device_diag(int* out8) {
   if (!out8) return;
   for (int i = 0; i < 8; ++i) out8[i] = t_last_diag[i];
+}
+
+clear_status_t clear_attn_selftest_expiry(int limit_ms, void* stream) {
+  if (limit_ms < 1 || limit_ms > 5000) return CLEAR_ERR_INVALID_ARG;
+  int num_sms = 0;
+  const clear_status_t st = check_device(&num_sms);
+  if (st != CLEAR_OK) return st;
+  clear_selftest_expiry_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      (unsigned long long)limit_ms * 1000000ull);
+  return cudaGetLastError() == cudaSuccess ? CLEAR_OK : CLEAR_ERR_CUDA;
 }
 
 clear_status_t clear_sched_forward_shape(const clear_attn_params_t* params, long long* n_text_items,

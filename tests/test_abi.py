@@ -80,6 +80,11 @@ def test_backward_argument_errors_launch_nothing():
         assert (a == 0x5A).all()
 
 
+@pytest.mark.parametrize("limit_ms", [0, -5, 5001])
+def test_selftest_rejects_bad_limits_before_any_cuda_call(limit_ms):
+    assert L.status_string(L.lib().clear_attn_selftest_expiry(limit_ms, None)) == "CLEAR_ERR_INVALID_ARG"
+
+
 def test_workspace_sizes():
     # Forward scratch holds the split partials of the text rows: S * BH * n_text rows of d fp32 plus
     # (max, sum) pairs; none without text.
