@@ -202,7 +202,14 @@ __global__ void clear_bwd_reduce_kernel(const float* __restrict__ part, __nv_bfl
 // ------------------------------------------------------------------------------------------------
 // dQ kernel (Q-stationary)
 // ------------------------------------------------------------------------------------------------
-constexpr int kBwdThreads = 192;
+// 3 warpgroups: two softmax warpgroups (each owns 64 of the 128 key or query columns of a tile),
+// then the TMA producer (warp 8), the MMA issuer / TMEM owner (warp 9) and two idle warps.
+constexpr int kBwdThreads = 384;
+// Launched at 168 registers per thread; the producer / MMA warpgroup drops to kBwdRegsLow and the
+// softmax warpgroups grow to kBwdRegsHigh.
+constexpr uint32_t kBwdRegsLow = 104;
+constexpr uint32_t kBwdRegsHigh = 200;
+static_assert(2 * 128 * kBwdRegsHigh + 128 * kBwdRegsLow <= 384 * 168, "register split exceeds the launch allocation");
 
 template <int D, int NST>
 struct DqLayout {
@@ -246,8 +253,8 @@ clear_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_c
     mbar_init(&bars[L::bQFull], 1);
     mbar_init(&bars[L::bQEmpty], 1);
     mbar_init(&bars[L::bSdpFull], 1);
-    mbar_init(&bars[L::bSdpFree], 128);
-    mbar_init(&bars[L::bDsFull], 128);
+    mbar_init(&bars[L::bSdpFree], 256);
+    mbar_init(&bars[L::bDsFull], 256);
     mbar_init(&bars[L::bDsEmpty], 1);
     mbar_init(&bars[L::bAccDone], 1);
     for (int s = 0; s < NST; ++s) {
@@ -259,7 +266,7 @@ clear_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_c
     fence_barrier_init();
   }
   for (int i = threadIdx.x; i < kMaxRTable; i += blockDim.x) wtab[i] = half_width(g.r, i);
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
   }
@@ -268,7 +275,8 @@ clear_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_c
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
+    regs_dec<kBwdRegsLow>();
     if (lane == 0) {
       int stage = 0;
       uint32_t ring_ph = 0, q_empty_ph = 0;
@@ -306,7 +314,8 @@ clear_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_c
     producer_done:;
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
+    regs_dec<kBwdRegsLow>();
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, 0, 1);
@@ -348,9 +357,13 @@ clear_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_c
     mma_done:;
     }
     __syncwarp();
-  } else {
-    const int row = threadIdx.x;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  } else if (warp < 8) {
+    regs_inc<kBwdRegsHigh>();
+    const int wg = warp >> 2;                // key columns [64 wg, 64 wg + 64) of every tile
+    const int row = threadIdx.x & 127;       // query row = TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    constexpr int kC = kTile / 2;
+    constexpr int kHalfD = D / 2;            // output columns of this warpgroup
     const uint32_t ds_addr = smem_u32(smem + L::kDS);
     uint32_t sdp_full_ph = 0, ds_empty_ph = 0, acc_ph = 0;
     const float sl2 = p.scale_log2;
@@ -378,18 +391,25 @@ clear_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_c
         if (!mbar_wait(&bars[L::bSdpFull], sdp_full_ph, abort_flag, kDevTimeoutSoftmax)) goto softmax_done;
         sdp_full_ph ^= 1;
         tc_fence_after();
-        float s[kTile];
-        tmem_ld128(tmem + lane_base + L::kTmemS, s);
-        // P = 2^(s * c - lse2) on kept pairs, 0 elsewhere
+        float s[kC];
+        {
+          uint32_t sr[2][32];
+          tmem_ld32(tmem + lane_base + L::kTmemS + kC * wg, sr[0]);
+          tmem_ld32(tmem + lane_base + L::kTmemS + kC * wg + 32, sr[1]);
+          tmem_wait_ld();
+          #pragma unroll
+          for (int c = 0; c < kC; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
+        }
+        // P = 2^(s * c - lse2) on kept pairs, 0 elsewhere (this warpgroup's four key rows / 64 keys)
         if (t.flags != kFull) {
           if (t.kind == kLinear) {
             #pragma unroll
-            for (int c = 0; c < kTile; ++c)
-              if (c >= t.b) s[c] = -INFINITY;
+            for (int c = 0; c < kC; ++c)
+              if (kC * wg + c >= t.b) s[c] = -INFINITY;
           } else {
             #pragma unroll
-            for (int kr = 0; kr < kKH; ++kr) {
-              const uint32_t bits = rect_row_bits(g, wtab, yq, xq, t.a + kr, t.b);
+            for (int kr = 0; kr < kKH / 2; ++kr) {
+              const uint32_t bits = rect_row_bits(g, wtab, yq, xq, t.a + (kKH / 2) * wg + kr, t.b);
               #pragma unroll
               for (int c = 0; c < kKW; ++c)
                 if (!((bits >> c) & 1u)) s[kr * kKW + c] = -INFINITY;
@@ -397,24 +417,32 @@ clear_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_c
           }
         }
         #pragma unroll
-        for (int c = 0; c < kTile; ++c) s[c] = ex2_approx(fmaf(s[c], sl2, -lse2));
-        float dp[kTile];
-        tmem_ld128(tmem + lane_base + L::kTmemDP, dp);
+        for (int c = 0; c < kC; ++c) s[c] = ex2_approx(fmaf(s[c], sl2, -lse2));
+        float dp[kC];
+        {
+          uint32_t dr[2][32];
+          tmem_ld32(tmem + lane_base + L::kTmemDP + kC * wg, dr[0]);
+          tmem_ld32(tmem + lane_base + L::kTmemDP + kC * wg + 32, dr[1]);
+          tmem_wait_ld();
+          #pragma unroll
+          for (int c = 0; c < kC; ++c) dp[c] = __uint_as_float(dr[c >> 5][c & 31]);
+        }
         tc_fence_before();
         mbar_arrive(&bars[L::bSdpFree]);
         #pragma unroll
-        for (int c = 0; c < kTile; ++c) s[c] = s[c] * (dp[c] - dd);  // dS
+        for (int c = 0; c < kC; ++c) s[c] = s[c] * (dp[c] - dd);  // dS
         if (ds_pending) {
           if (!mbar_wait(&bars[L::bDsEmpty], ds_empty_ph, abort_flag, kDevTimeoutSoftmax)) goto softmax_done;
           ds_empty_ph ^= 1;
         }
-        store_row_sw128(ds_addr, row, s);
+        store_chunk32_sw128(ds_addr, row, 2 * wg, s);
+        store_chunk32_sw128(ds_addr, row, 2 * wg + 1, s + 32);
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&bars[L::bDsFull]);
         ds_pending = true;
       }
-      // epilogue
+      // epilogue: this warpgroup's half of the dQ row
       if (!mbar_wait(&bars[L::bAccDone], acc_ph, abort_flag, kDevTimeoutSoftmax)) goto softmax_done;
       acc_ph ^= 1;
       if (ds_pending) {  // the last dQ MMA has completed too
@@ -424,22 +452,23 @@ clear_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_c
       }
       tc_fence_after();
       {
-        const uint32_t abase = tmem + lane_base + L::kTmemAcc;
+        const uint32_t abase = tmem + lane_base + L::kTmemAcc + wg * kHalfD;
         #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < kHalfD / 32; ++c) {
           uint32_t ov[32];
           tmem_ld32(abase + c * 32, ov);
           tmem_wait_ld();
           if (!row_valid) continue;
+          const int col = wg * kHalfD + c * 32;
           if (it.is_text) {
-            float* dst = p.part_a + (((size_t)it.split * g.BH + it.bh) * g.n_text + it.q0 + row) * D + c * 32;
+            float* dst = p.part_a + (((size_t)it.split * g.BH + it.bh) * g.n_text + it.q0 + row) * D + col;
             float4* d4 = reinterpret_cast<float4*>(dst);
             #pragma unroll
             for (int e = 0; e < 8; ++e)
               d4[e] = make_float4(__uint_as_float(ov[4 * e]), __uint_as_float(ov[4 * e + 1]),
                                   __uint_as_float(ov[4 * e + 2]), __uint_as_float(ov[4 * e + 3]));
           } else {
-            uint4* d4 = reinterpret_cast<uint4*>(p.out_a + grow * D + c * 32);
+            uint4* d4 = reinterpret_cast<uint4*>(p.out_a + grow * D + col);
             const float sc = p.scale;
             #pragma unroll
             for (int e = 0; e < 4; ++e)
@@ -453,10 +482,12 @@ clear_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_c
       tc_fence_before();
     }
   softmax_done:;
+  } else {
+    regs_dec<kBwdRegsLow>();
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
   }
@@ -511,16 +542,16 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
     mbar_init(&bars[L::bQFull], 1);
     mbar_init(&bars[L::bQEmpty], 1);
     mbar_init(&bars[L::bSFull], 1);
-    mbar_init(&bars[L::bSFree], 128);
-    mbar_init(&bars[L::bPFull], 128);
-    mbar_init(&bars[L::bDsFull], 128);
+    mbar_init(&bars[L::bSFree], 256);
+    mbar_init(&bars[L::bPFull], 256);
+    mbar_init(&bars[L::bDsFull], 256);
     mbar_init(&bars[L::bPdsEmpty], 1);
     mbar_init(&bars[L::bAccDone], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   for (int i = threadIdx.x; i < kMaxRTable; i += blockDim.x) wtab[i] = half_width(g.r, i);
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
   }
@@ -529,7 +560,8 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
+    regs_dec<kBwdRegsLow>();
     if (lane == 0) {
       uint32_t kv_empty_ph = 0, q_empty_ph = 0;
       bool first_item = true, first_tile = true;
@@ -563,7 +595,8 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
     producer_done:;
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
+    regs_dec<kBwdRegsLow>();
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, 0, 1);
@@ -605,9 +638,12 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
     mma_done:;
     }
     __syncwarp();
-  } else {
-    const int row = threadIdx.x;  // key row of the stationary tile
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  } else if (warp < 8) {
+    regs_inc<kBwdRegsHigh>();
+    const int wg = warp >> 2;                // partner query columns [64 wg, 64 wg + 64) of every tile
+    const int row = threadIdx.x & 127;       // key row of the stationary tile = TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    constexpr int kHalfD = D / 2;            // output columns of this warpgroup
     const uint32_t pt_addr = smem_u32(smem + L::kPT);
     const uint32_t dst_addr = smem_u32(smem + L::kDST);
     uint32_t s_full_ph = 0, pds_empty_ph = 0, acc_ph = 0;
@@ -632,10 +668,10 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
       ki.init(g, it);
       KeyTile t;
       while (ki.next(&t)) {
-        // Row statistics of the 128 partner queries into smem (column c <- thread c).
+        // Row statistics of the 128 partner queries into smem (column c <- thread c of warpgroup 0).
         float* lse_s = vec + (tile_counter & 1) * 2 * kTile;
         float* dv_s = lse_s + kTile;
-        {
+        if (wg == 0) {
           const int c = row;
           bool ok;
           size_t qrow;
@@ -650,7 +686,7 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
           lse_s[c] = ok ? p.l2vec[qrow] : INFINITY;
           dv_s[c] = ok ? p.dvec[qrow] : 0.f;
         }
-        named_bar_sync(1, 128);
+        named_bar_sync(1, 256);
         ++tile_counter;
         if (!mbar_wait(&bars[L::bSFull], s_full_ph, abort_flag, kDevTimeoutSoftmax)) goto softmax_done;
         s_full_ph ^= 1;
@@ -661,7 +697,7 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
         tc_fence_after();
         // 32 partner columns at a time: P^T = 2^(s c - lse2) on kept pairs, dS^T = P^T (dP^T - D).
         #pragma unroll 1
-        for (int ch = 0; ch < kTile / 32; ++ch) {
+        for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
           uint32_t sr[32], dr[32];
           tmem_ld32(tmem + lane_base + L::kTmemS + ch * 32, sr);
           tmem_ld32(tmem + lane_base + L::kTmemDP + ch * 32, dr);
@@ -703,18 +739,19 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
       }
       tc_fence_after();
       #pragma unroll
-      for (int which = 0; which < 2; ++which) {  // 0: dK, 1: dV
-        const uint32_t abase = tmem + lane_base + (which == 0 ? L::kTmemDK : L::kTmemDV);
+      for (int which = 0; which < 2; ++which) {  // 0: dK, 1: dV; this warpgroup's half of each row
+        const uint32_t abase = tmem + lane_base + (which == 0 ? L::kTmemDK : L::kTmemDV) + wg * kHalfD;
         const float sc = which == 0 ? p.scale : 1.f;
         #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < kHalfD / 32; ++c) {
           uint32_t ov[32];
           tmem_ld32(abase + c * 32, ov);
           tmem_wait_ld();
           if (!row_valid) continue;
+          const int col = wg * kHalfD + c * 32;
           if (it.is_text) {
             float* part = which == 0 ? p.part_a : p.part_b;
-            float* dst = part + (((size_t)it.split * g.BH + it.bh) * g.n_text + it.q0 + row) * D + c * 32;
+            float* dst = part + (((size_t)it.split * g.BH + it.bh) * g.n_text + it.q0 + row) * D + col;
             float4* d4 = reinterpret_cast<float4*>(dst);
             #pragma unroll
             for (int e = 0; e < 8; ++e)
@@ -722,7 +759,7 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
                                   __uint_as_float(ov[4 * e + 2]), __uint_as_float(ov[4 * e + 3]));
           } else {
             __nv_bfloat16* out = which == 0 ? p.out_a : p.out_b;
-            uint4* d4 = reinterpret_cast<uint4*>(out + grow * D + c * 32);
+            uint4* d4 = reinterpret_cast<uint4*>(out + grow * D + col);
             #pragma unroll
             for (int e = 0; e < 4; ++e)
               d4[e] = make_uint4(pack_bf16x2(__uint_as_float(ov[8 * e + 0]) * sc, __uint_as_float(ov[8 * e + 1]) * sc),
@@ -735,10 +772,12 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
       tc_fence_before();
     }
   softmax_done:;
+  } else {
+    regs_dec<kBwdRegsLow>();
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
   }
