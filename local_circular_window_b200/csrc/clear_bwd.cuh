@@ -9,14 +9,17 @@
 //
 // Kernels (all deterministic, no floating-point atomics):
 //   preprocess  D and LSE * log2(e) per row                             (CUDA cores, HBM-bound)
-//   dq kernel   Q-stationary: per query tile, visit the forward's key tiles; S, dP -> TMEM,
-//               dS -> smem (bf16), dQ += dS K in TMEM. Text query tiles are split over key
-//               chunks into fp32 partials.
+//   dq kernel   Q-stationary: per query tile, visit its 128-key tiles; S, dP -> TMEM,
+//               dS -> smem (bf16), dQ += dS K in TMEM; S and dP of the next key tile are issued
+//               before dQ of this one. Text query tiles are split over key chunks into fp32
+//               partials.
 //   dkdv kernel KV-stationary: per key tile, visit the query tiles that keep it. The mask is
-//               symmetric, so the forward's tile enumeration with the roles of query and key
-//               swapped gives exactly those tiles. S^T, dP^T -> TMEM; P^T, dS^T -> smem (bf16);
-//               dV += P^T dO, dK += dS^T Q in TMEM. Text key tiles are split over query chunks
-//               into fp32 partials.
+//               symmetric, so the same tile enumeration with the roles of query and key swapped
+//               gives exactly those tiles. S^T, dP^T -> TMEM; P^T, dS^T written back over them
+//               (bf16); dV += P^T dO, dK += dS^T Q in TMEM with the A operand read from TMEM;
+//               partner Q / dO double-buffered. Text key tiles are split over query chunks into
+//               fp32 partials.
+// Both kernels split each tile's 128 columns over two softmax warpgroups (64 each).
 //   reduce      sums the split partials of the text rows in a fixed order and writes bf16.
 #pragma once
 #include <cuda_bf16.h>
@@ -207,8 +210,8 @@ __global__ void clear_bwd_reduce_kernel(const float* __restrict__ part, __nv_bfl
 constexpr int kBwdThreads = 384;
 // Launched at 168 registers per thread; the producer / MMA warpgroup drops to kBwdRegsLow and the
 // softmax warpgroups grow to kBwdRegsHigh.
-constexpr uint32_t kBwdRegsLow = 104;
-constexpr uint32_t kBwdRegsHigh = 200;
+constexpr uint32_t kBwdRegsLow = 120;
+constexpr uint32_t kBwdRegsHigh = 192;
 static_assert(2 * 128 * kBwdRegsHigh + 128 * kBwdRegsLow <= 384 * 168, "register split exceeds the launch allocation");
 
 template <int D, int NST>
@@ -322,36 +325,44 @@ clear_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_c
       const uint32_t q_addr = smem_u32(smem + L::kQ);
       const uint32_t do_addr = smem_u32(smem + L::kDO);
       const uint32_t ds_addr = smem_u32(smem + L::kDS);
+      static_assert(NST == 2, "S and dP of the next key tile are issued while dQ still reads this one's K");
       int stage = 0;
       uint32_t ring_ph = 0, q_full_ph = 0, ds_full_ph = 0, sdp_free_ph = 0;
+      // S = Q K^T and dP = dO V^T of key tile j into TMEM (K/V ring slot `stage`), once the softmax
+      // has read the previous pair.
+      auto issue_sdp = [&](int j, int n) -> bool {
+        if (!mbar_wait(&bars[L::bSdpFree], sdp_free_ph ^ 1, abort_flag, kDevTimeoutMma)) return false;
+        sdp_free_ph ^= 1;
+        if (!mbar_wait(&bars[L::bKFull + stage], ring_ph, abort_flag, kDevTimeoutMma)) return false;
+        if (!mbar_wait(&bars[L::bVFull + stage], ring_ph, abort_flag, kDevTimeoutMma)) return false;
+        tc_fence_after();
+        mma_kmajor<D>(tmem + L::kTmemS, q_addr, smem_u32(smem + L::kK + stage * L::kTileBytes), idesc_s);
+        mma_kmajor<D>(tmem + L::kTmemDP, do_addr, smem_u32(smem + L::kV + stage * L::kTileBytes), idesc_s);
+        umma_commit(&bars[L::bSdpFull]);
+        if (j == n - 1) umma_commit(&bars[L::bQEmpty]);  // Q and dO: last reads issued
+        return true;
+      };
       for (long long w = blockIdx.x; w < p.n_work; w += gridDim.x) {
         const WorkItem it = decode_work(g, w);
         const int n = count_key_tiles(g, it);
         if (!mbar_wait(&bars[L::bQFull], q_full_ph, abort_flag, kDevTimeoutMma)) goto mma_done;
         q_full_ph ^= 1;
         tc_fence_after();
+        if (!issue_sdp(0, n)) goto mma_done;
         for (int j = 0; j < n; ++j) {
-          // S = Q K^T and dP = dO V^T into TMEM, once the softmax has read the previous pair.
-          if (!mbar_wait(&bars[L::bSdpFree], sdp_free_ph ^ 1, abort_flag, kDevTimeoutMma)) goto mma_done;
-          sdp_free_ph ^= 1;
-          if (!mbar_wait(&bars[L::bKFull + stage], ring_ph, abort_flag, kDevTimeoutMma)) goto mma_done;
-          if (!mbar_wait(&bars[L::bVFull + stage], ring_ph, abort_flag, kDevTimeoutMma)) goto mma_done;
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(smem + L::kK + stage * L::kTileBytes);
-          const uint32_t v_addr = smem_u32(smem + L::kV + stage * L::kTileBytes);
-          mma_kmajor<D>(tmem + L::kTmemS, q_addr, k_addr, idesc_s);
-          mma_kmajor<D>(tmem + L::kTmemDP, do_addr, v_addr, idesc_s);
-          umma_commit(&bars[L::bSdpFull]);
-          if (j == n - 1) umma_commit(&bars[L::bQEmpty]);  // Q and dO: last reads issued
+          const int cur = stage;
+          if (++stage == NST) { stage = 0; ring_ph ^= 1; }
+          // S and dP of tile j + 1 run while the softmax turns tile j into dS.
+          if (j + 1 < n && !issue_sdp(j + 1, n)) goto mma_done;
           // dQ += dS K
           if (!mbar_wait(&bars[L::bDsFull], ds_full_ph, abort_flag, kDevTimeoutMma)) goto mma_done;
           ds_full_ph ^= 1;
           tc_fence_after();
-          mma_a_kmajor_b_mnmajor<D>(tmem + L::kTmemAcc, ds_addr, k_addr, idesc_dq, j > 0);
+          mma_a_kmajor_b_mnmajor<D>(tmem + L::kTmemAcc, ds_addr, smem_u32(smem + L::kK + cur * L::kTileBytes), idesc_dq,
+                                    j > 0);
           umma_commit(&bars[L::bDsEmpty]);
-          umma_commit(&bars[L::bKVEmpty + stage]);
+          umma_commit(&bars[L::bKVEmpty + cur]);
           if (j == n - 1) umma_commit(&bars[L::bAccDone]);
-          if (++stage == NST) { stage = 0; ring_ph ^= 1; }
         }
       }
     mma_done:;
@@ -501,22 +512,29 @@ struct DkvLayout {
   static constexpr int kTileBytes = kTile * D * 2;
   static constexpr int kK = 0;
   static constexpr int kV = kK + kTileBytes;
-  static constexpr int kQ = kV + kTileBytes;
-  static constexpr int kDO = kQ + kTileBytes;
-  static constexpr int kPT = kDO + kTileBytes;
-  static constexpr int kDST = kPT + kTile * kTile * 2;
-  static constexpr int kVec = kDST + kTile * kTile * 2;  // float lse2[2][128], dvec[2][128]
+  // Two buffers of the partner query tile's Q and dO, so the next tile loads during this one.
+  static constexpr int kQ = kV + kTileBytes;             // + buf * kQStride
+  static constexpr int kDO = kQ + kTileBytes;            // + buf * kQStride
+  static constexpr int kQStride = 2 * kTileBytes;
+  static constexpr int kVec = kQ + 2 * kQStride;         // float lse2/dvec [2][2][128]
   static constexpr int kBars = kVec + 4 * kTile * 4;
-  static constexpr int bKVFull = 0, bKVEmpty = 1, bQFull = 2, bQEmpty = 3, bSFull = 4, bSFree = 5, bPFull = 6,
-                       bDsFull = 7, bPdsEmpty = 8, bAccDone = 9;
-  static constexpr int kNumBars = 10;
+  static constexpr int bKVFull = 0, bKVEmpty = 1, bQFull = 2 /* + buf */, bQEmpty = 4 /* + buf */, bSFull = 6,
+                       bPFull = 7, bAccDone = 8;
+  static constexpr int kNumBars = 9;
   static constexpr int kMisc = kBars + kNumBars * 8;
   static constexpr int kWTab = kMisc + 16;
   static constexpr int kTotal = kWTab + kMaxRTable * 4;
   static constexpr int kAlloc = kTotal + 1024;
+  // TMEM: S^T (P^T as bf16 pairs over its first 64 columns once the softmax has read it), dP^T
+  // (dS^T likewise), and the dV, dK accumulators.
   static constexpr uint32_t kTmemS = 0, kTmemDP = 128, kTmemDV = 256, kTmemDK = 256 + D, kTmemCols = 512;
 };
 
+// KV-stationary: one CTA holds a key tile's K and V and visits its partner query tiles (the
+// mask is symmetric, so they are the key tiles KeyIter lists for a query tile at the same place):
+// S^T = K Q^T and dP^T = V dO^T into TMEM, P^T = 2^(S^T c - lse2) and dS^T = P^T (dP^T - D)
+// written back over them as bf16, then dV += P^T dO and dK += dS^T Q with the A operand read from
+// TMEM. Partner Q / dO tiles are double-buffered.
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_constant__ CUtensorMap tm_q_img,
@@ -539,13 +557,12 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
   if (threadIdx.x == 0) {
     mbar_init(&bars[L::bKVFull], 1);
     mbar_init(&bars[L::bKVEmpty], 1);
-    mbar_init(&bars[L::bQFull], 1);
-    mbar_init(&bars[L::bQEmpty], 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars[L::bQFull + b], 1);
+      mbar_init(&bars[L::bQEmpty + b], 1);
+    }
     mbar_init(&bars[L::bSFull], 1);
-    mbar_init(&bars[L::bSFree], 256);
     mbar_init(&bars[L::bPFull], 256);
-    mbar_init(&bars[L::bDsFull], 256);
-    mbar_init(&bars[L::bPdsEmpty], 1);
     mbar_init(&bars[L::bAccDone], 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -563,8 +580,8 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
   if (warp == 8) {
     regs_dec<kBwdRegsLow>();
     if (lane == 0) {
-      uint32_t kv_empty_ph = 0, q_empty_ph = 0;
-      bool first_item = true, first_tile = true;
+      uint32_t kv_empty_ph = 0, c = 0;  // c: partner tiles loaded so far
+      bool first_item = true;
       for (long long w = blockIdx.x; w < p.n_work; w += gridDim.x) {
         const WorkItem it = decode_work(g, w);  // the stationary key tile
         if (!first_item) {
@@ -581,17 +598,17 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
         ki.init(g, it);
         KeyTile t;
         while (ki.next(&t)) {  // partner query tiles
-          if (!first_tile) {
-            if (!mbar_wait(&bars[L::bQEmpty], q_empty_ph, abort_flag, kDevTimeoutTmaEmpty)) goto producer_done;
-            q_empty_ph ^= 1;
-          }
-          first_tile = false;
-          mbar_arrive_expect_tx(&bars[L::bQFull], 2 * L::kTileBytes);
-          load_tile<D>(smem + L::kQ, &tm_q_lin, &tm_q_img, &bars[L::bQFull], t.kind, t.a, t.b, it.bh);
-          load_tile<D>(smem + L::kDO, &tm_do_lin, &tm_do_img, &bars[L::bQFull], t.kind, t.a, t.b, it.bh);
+          const uint32_t qb = c & 1;
+          if (c >= 2 && !mbar_wait(&bars[L::bQEmpty + qb], ((c >> 1) - 1) & 1, abort_flag, kDevTimeoutTmaEmpty))
+            goto producer_done;
+          mbar_arrive_expect_tx(&bars[L::bQFull + qb], 2 * L::kTileBytes);
+          load_tile<D>(smem + L::kQ + qb * L::kQStride, &tm_q_lin, &tm_q_img, &bars[L::bQFull + qb], t.kind, t.a,
+                       t.b, it.bh);
+          load_tile<D>(smem + L::kDO + qb * L::kQStride, &tm_do_lin, &tm_do_img, &bars[L::bQFull + qb], t.kind,
+                       t.a, t.b, it.bh);
+          ++c;
         }
       }
-      if (!first_tile) mbar_wait(&bars[L::bQEmpty], q_empty_ph, abort_flag, kDevTimeoutTmaEmpty);
     producer_done:;
     }
     __syncwarp();
@@ -602,35 +619,37 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
       constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t k_addr = smem_u32(smem + L::kK);
       const uint32_t v_addr = smem_u32(smem + L::kV);
-      const uint32_t q_addr = smem_u32(smem + L::kQ);
-      const uint32_t do_addr = smem_u32(smem + L::kDO);
-      const uint32_t pt_addr = smem_u32(smem + L::kPT);
-      const uint32_t dst_addr = smem_u32(smem + L::kDST);
-      uint32_t kv_full_ph = 0, q_full_ph = 0, s_free_ph = 0, p_full_ph = 0, ds_full_ph = 0;
+      uint32_t kv_full_ph = 0, p_full_ph = 0, c = 0;
       for (long long w = blockIdx.x; w < p.n_work; w += gridDim.x) {
         const WorkItem it = decode_work(g, w);
         const int n = count_key_tiles(g, it);
         if (!mbar_wait(&bars[L::bKVFull], kv_full_ph, abort_flag, kDevTimeoutMma)) goto mma_done;
         kv_full_ph ^= 1;
-        for (int i = 0; i < n; ++i) {
-          if (!mbar_wait(&bars[L::bSFree], s_free_ph ^ 1, abort_flag, kDevTimeoutMma)) goto mma_done;
-          s_free_ph ^= 1;
-          if (!mbar_wait(&bars[L::bQFull], q_full_ph, abort_flag, kDevTimeoutMma)) goto mma_done;
-          q_full_ph ^= 1;
+        for (int i = 0; i < n; ++i, ++c) {
+          const uint32_t qb = c & 1;
+          const uint32_t q_addr = smem_u32(smem + L::kQ + qb * L::kQStride);
+          const uint32_t do_addr = smem_u32(smem + L::kDO + qb * L::kQStride);
+          if (!mbar_wait(&bars[L::bQFull + qb], (c >> 1) & 1, abort_flag, kDevTimeoutMma)) goto mma_done;
           tc_fence_after();
+          // S^T and dP^T overwrite the previous tile's P^T and dS^T: the products reading those
+          // were issued before, by this thread, and run first.
           mma_kmajor<D>(tmem + L::kTmemS, k_addr, q_addr, idesc_s);    // S^T = K Q^T
           mma_kmajor<D>(tmem + L::kTmemDP, v_addr, do_addr, idesc_s);  // dP^T = V dO^T
           umma_commit(&bars[L::bSFull]);
           if (!mbar_wait(&bars[L::bPFull], p_full_ph, abort_flag, kDevTimeoutMma)) goto mma_done;
           p_full_ph ^= 1;
           tc_fence_after();
-          mma_a_kmajor_b_mnmajor<D>(tmem + L::kTmemDV, pt_addr, do_addr, idesc_acc, i > 0);   // dV += P^T dO
-          if (!mbar_wait(&bars[L::bDsFull], ds_full_ph, abort_flag, kDevTimeoutMma)) goto mma_done;
-          ds_full_ph ^= 1;
-          tc_fence_after();
-          mma_a_kmajor_b_mnmajor<D>(tmem + L::kTmemDK, dst_addr, q_addr, idesc_acc, i > 0);  // dK += dS^T Q
-          umma_commit(&bars[L::bQEmpty]);
-          umma_commit(&bars[L::bPdsEmpty]);
+          const uint64_t do_desc = smem_desc_sw128(do_addr, kHalfBytes, 1024);
+          const uint64_t q_desc = smem_desc_sw128(q_addr, kHalfBytes, 1024);
+          #pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)  // dV += P^T dO
+            umma_ts(tmem + L::kTmemDV, tmem + L::kTmemS + kk * 8, do_desc + (uint64_t)((kk * 2048) >> 4), idesc_acc,
+                    (i > 0 || kk > 0) ? 1u : 0u);
+          #pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)  // dK += dS^T Q
+            umma_ts(tmem + L::kTmemDK, tmem + L::kTmemDP + kk * 8, q_desc + (uint64_t)((kk * 2048) >> 4), idesc_acc,
+                    (i > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&bars[L::bQEmpty + qb]);
         }
         umma_commit(&bars[L::bAccDone]);
         umma_commit(&bars[L::bKVEmpty]);
@@ -644,11 +663,8 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
     const int row = threadIdx.x & 127;       // key row of the stationary tile = TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     constexpr int kHalfD = D / 2;            // output columns of this warpgroup
-    const uint32_t pt_addr = smem_u32(smem + L::kPT);
-    const uint32_t dst_addr = smem_u32(smem + L::kDST);
-    uint32_t s_full_ph = 0, pds_empty_ph = 0, acc_ph = 0;
+    uint32_t s_full_ph = 0, acc_ph = 0;
     const float sl2 = p.scale_log2;
-    bool pds_pending = false;
     uint32_t tile_counter = 0;
     for (long long w = blockIdx.x; w < p.n_work; w += gridDim.x) {
       const WorkItem it = decode_work(g, w);
@@ -671,6 +687,7 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
         // Row statistics of the 128 partner queries into smem (column c <- thread c of warpgroup 0).
         float* lse_s = vec + (tile_counter & 1) * 2 * kTile;
         float* dv_s = lse_s + kTile;
+        ++tile_counter;
         if (wg == 0) {
           const int c = row;
           bool ok;
@@ -686,57 +703,56 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
           lse_s[c] = ok ? p.l2vec[qrow] : INFINITY;
           dv_s[c] = ok ? p.dvec[qrow] : 0.f;
         }
-        named_bar_sync(1, 256);
-        ++tile_counter;
         if (!mbar_wait(&bars[L::bSFull], s_full_ph, abort_flag, kDevTimeoutSoftmax)) goto softmax_done;
         s_full_ph ^= 1;
-        if (pds_pending) {  // the previous tile's dV/dK MMAs have finished reading P^T and dS^T
-          if (!mbar_wait(&bars[L::bPdsEmpty], pds_empty_ph, abort_flag, kDevTimeoutSoftmax)) goto softmax_done;
-          pds_empty_ph ^= 1;
-        }
         tc_fence_after();
-        // 32 partner columns at a time: P^T = 2^(s c - lse2) on kept pairs, dS^T = P^T (dP^T - D).
-        #pragma unroll 1
-        for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
-          uint32_t sr[32], dr[32];
-          tmem_ld32(tmem + lane_base + L::kTmemS + ch * 32, sr);
-          tmem_ld32(tmem + lane_base + L::kTmemDP + ch * 32, dr);
-          tmem_wait_ld();
+        uint32_t sr[2][32], dr[2][32];
+        tmem_ld32(tmem + lane_base + L::kTmemS + 64 * wg, sr[0]);
+        tmem_ld32(tmem + lane_base + L::kTmemS + 64 * wg + 32, sr[1]);
+        tmem_ld32(tmem + lane_base + L::kTmemDP + 64 * wg, dr[0]);
+        tmem_ld32(tmem + lane_base + L::kTmemDP + 64 * wg + 32, dr[1]);
+        tmem_wait_ld();
+        // Every thread has read its S^T / dP^T columns (P^T / dS^T overwrite columns of the other
+        // warpgroup's half) and warpgroup 0 has stored the partner statistics.
+        tc_fence_before();
+        named_bar_sync(1, 256);
+        tc_fence_after();
+        // P^T = 2^(s c - lse2) on kept pairs, dS^T = P^T (dP^T - D), as bf16 pairs.
+        uint32_t pw[32], dw[32];
+        #pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          const int gch = 2 * wg + ch;  // 32-column chunk of the tile
           uint32_t keep = 0xffffffffu;
           if (t.flags != kFull) {
             if (t.kind == kLinear) {
-              const int lim = t.b - ch * 32;
+              const int lim = t.b - gch * 32;
               keep = lim >= 32 ? 0xffffffffu : (lim <= 0 ? 0u : ((1u << lim) - 1u));
             } else {
-              keep = rect_row_bits(g, wtab, yk, xk, t.a + 2 * ch, t.b) |
-                     (rect_row_bits(g, wtab, yk, xk, t.a + 2 * ch + 1, t.b) << 16);
+              keep = rect_row_bits(g, wtab, yk, xk, t.a + 2 * gch, t.b) |
+                     (rect_row_bits(g, wtab, yk, xk, t.a + 2 * gch + 1, t.b) << 16);
             }
           }
-          float pv[32], dsv[32];
           #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int c = ch * 32 + e;
-            const float x = ((keep >> e) & 1u) ? __uint_as_float(sr[e]) : -INFINITY;
-            pv[e] = ex2_approx(fmaf(x, sl2, -lse_s[c]));
-            dsv[e] = pv[e] * (__uint_as_float(dr[e]) - dv_s[c]);
+          for (int e = 0; e < 32; e += 2) {
+            const int c = gch * 32 + e;
+            const float x0 = ((keep >> e) & 1u) ? __uint_as_float(sr[ch][e]) : -INFINITY;
+            const float x1 = ((keep >> (e + 1)) & 1u) ? __uint_as_float(sr[ch][e + 1]) : -INFINITY;
+            const float p0 = ex2_approx(fmaf(x0, sl2, -lse_s[c]));
+            const float p1 = ex2_approx(fmaf(x1, sl2, -lse_s[c + 1]));
+            const float d0 = p0 * (__uint_as_float(dr[ch][e]) - dv_s[c]);
+            const float d1 = p1 * (__uint_as_float(dr[ch][e + 1]) - dv_s[c + 1]);
+            pw[ch * 16 + e / 2] = pack_bf16x2(p0, p1);
+            dw[ch * 16 + e / 2] = pack_bf16x2(d0, d1);
           }
-          store_chunk32_sw128(pt_addr, row, ch, pv);
-          store_chunk32_sw128(dst_addr, row, ch, dsv);
         }
+        tmem_st32(tmem + lane_base + L::kTmemS + 32 * wg, pw);
+        tmem_st32(tmem + lane_base + L::kTmemDP + 32 * wg, dw);
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars[L::bSFree]);
-        fence_proxy_async_smem();
         mbar_arrive(&bars[L::bPFull]);
-        mbar_arrive(&bars[L::bDsFull]);
-        pds_pending = true;
       }
       if (!mbar_wait(&bars[L::bAccDone], acc_ph, abort_flag, kDevTimeoutSoftmax)) goto softmax_done;
       acc_ph ^= 1;
-      if (pds_pending) {
-        if (!mbar_wait(&bars[L::bPdsEmpty], pds_empty_ph, abort_flag, kDevTimeoutSoftmax)) goto softmax_done;
-        pds_empty_ph ^= 1;
-        pds_pending = false;
-      }
       tc_fence_after();
       #pragma unroll
       for (int which = 0; which < 2; ++which) {  // 0: dK, 1: dV; this warpgroup's half of each row
