@@ -132,13 +132,21 @@ def _dist():
     return world, rank, local
 
 
-def _max_over_ranks(x: float, world: int) -> float:
+def _max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job(total_ms_local: float, steps: int, useful_flops_per_call: float, world: int, device: str = "cuda"):
+    """Per-step time as the slowest rank's, and whole-job throughput: every rank runs its own
+    independent call per step, so the job does world x useful FLOPs per step."""
+    total_ms = _max_over_ranks(total_ms_local, world, device)
+    ms = total_ms / steps
+    return ms, useful_flops_per_call * world / (ms * 1e-3) / 1e12
 
 
 def _barrier(world):
@@ -265,9 +273,7 @@ def run_clear(args):
         _barrier(world)
     if L.clear_attn_check() != 0:
         raise RuntimeError("device error during timing")
-    total_ms = _max_over_ranks(total_ms, world)
-    ms = total_ms / args.steps
-    value = useful * world / (ms * 1e-3) / 1e12
+    ms, value = whole_job(total_ms, args.steps, useful, world)
     kernel_ms = statistics.mean(per)
     achieved = useful / (kernel_ms * 1e-3) / 1e12
 
