@@ -45,8 +45,8 @@ constexpr int kFwdThreads = 384;           // 3 warpgroups: softmax A, softmax B
 // Launched at 168 registers per thread (65536 / 384, rounded to 8). The producer / MMA warpgroup
 // drops to kRegsLow and the two softmax warpgroups grow to kRegsHigh:
 // 2 * 128 * kRegsHigh + 128 * kRegsLow <= 384 * 168.
-constexpr uint32_t kRegsLow = 72;
-constexpr uint32_t kRegsHigh = 216;
+constexpr uint32_t kRegsLow = 88;
+constexpr uint32_t kRegsHigh = 208;
 static_assert(2 * 128 * kRegsHigh + 128 * kRegsLow <= 384 * 168, "register split exceeds the launch allocation");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kTileRing = 16;              // union tile descriptors in flight (producer -> others)
@@ -286,6 +286,40 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
       wd.start();
       while (!all_posted || Gp < Gq || pend > 0) {
         bool prog = false;
+        // ---- PV walk step (tiles the QK walk has passed, in order). It goes first: a ready P V
+        // frees the S buffer the next Q K^T needs.
+        if (Gp < Gq) {
+          const uint32_t vs = Gp % kVStages;
+          const int slot = npv & 1;
+          const bool needed = pend > 0 && pend_G[slot] == Gp;
+          if (!needed) {
+            if (mbar_test(&bars[L::bVFull + vs], (Gp / kVStages) & 1)) {
+              mbar_arrive(&bars[L::bVEmpty + vs]);  // observed and released
+              ++Gp;
+              prog = true;
+            }
+          } else {
+            const uint32_t b = npv & 1;
+            if (mbar_test(&bars[L::bPFull + 2 * h + b], (npv >> 1) & 1) &&
+                mbar_test(&bars[L::bVFull + vs], (Gp / kVStages) & 1)) {
+              tc_fence_after();
+              const uint64_t vd = vdesc0 + (uint64_t)((vs * L::kKVTileBytes) >> 4);
+              const uint32_t s_tm = tmem + L::s_col(h, b);
+              const bool first = pend_fl[slot] & 1;
+              #pragma unroll
+              for (int kk = 0; kk < kFChunk / 16; ++kk)
+                umma_ts(o_tm, s_tm + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv,
+                        (!first || kk > 0) ? 1u : 0u);
+              umma_commit(&bars[L::bVEmpty + vs]);
+              umma_commit(&bars[L::bOReady + h]);
+              if (pend_fl[slot] & 2) umma_commit(&bars[L::bODone + h]);
+              ++npv;
+              --pend;
+              ++Gp;
+              prog = true;
+            }
+          }
+        }
         // ---- QK walk step
         if (end_pending || (pair >= n_pairs && !all_posted)) {
           // Post an end-of-pair (or end-of-work) message once the mailbox slot is free.
@@ -360,39 +394,6 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
                   q_seen = false;
                 }
               }
-            }
-          }
-        }
-        // ---- PV walk step (tiles the QK walk has passed, in order)
-        if (Gp < Gq) {
-          const uint32_t vs = Gp % kVStages;
-          const int slot = npv & 1;
-          const bool needed = pend > 0 && pend_G[slot] == Gp;
-          if (!needed) {
-            if (mbar_test(&bars[L::bVFull + vs], (Gp / kVStages) & 1)) {
-              mbar_arrive(&bars[L::bVEmpty + vs]);  // observed and released
-              ++Gp;
-              prog = true;
-            }
-          } else {
-            const uint32_t b = npv & 1;
-            if (mbar_test(&bars[L::bPFull + 2 * h + b], (npv >> 1) & 1) &&
-                mbar_test(&bars[L::bVFull + vs], (Gp / kVStages) & 1)) {
-              tc_fence_after();
-              const uint64_t vd = vdesc0 + (uint64_t)((vs * L::kKVTileBytes) >> 4);
-              const uint32_t s_tm = tmem + L::s_col(h, b);
-              const bool first = pend_fl[slot] & 1;
-              #pragma unroll
-              for (int kk = 0; kk < kFChunk / 16; ++kk)
-                umma_ts(o_tm, s_tm + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv,
-                        (!first || kk > 0) ? 1u : 0u);
-              umma_commit(&bars[L::bVEmpty + vs]);
-              umma_commit(&bars[L::bOReady + h]);
-              if (pend_fl[slot] & 2) umma_commit(&bars[L::bODone + h]);
-              ++npv;
-              --pend;
-              ++Gp;
-              prog = true;
             }
           }
         }
