@@ -1,7 +1,9 @@
 """CPU float64 oracle for CLEAR attention. Test infrastructure only: imported by tests/,
 __graft_entry__.smoke() and bench.py's CPU-baseline / reference legs, never by the product path."""
 from .clear_attention import (  # noqa: F401
+    WINDOWS,
     token_coords,
+    window_half_width,
     clear_mask,
     clear_attention_forward,
     clear_attention_rows,

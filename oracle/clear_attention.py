@@ -22,6 +22,13 @@ Revs Pre-Trained Diffusion Transformers Up"):
    by gradient descent [pith review, "The reading"], so the gradient is the analytic gradient of
    the forward above (standard softmax-attention calculus, written out in `clear_attention_backward`).
 
+5. Square-window variant (a comparison mask, not CLEAR's): the pages contrast the circular window
+   with "the traditional square sliding window" [nav.superapi.store page, "Technical Principles of
+   CLEAR"] and give the circle's cost as about pi/4 of a square window's [pith review, "What
+   carries the argument"]. Read as the same rule with the Chebyshev distance: image tokens i and j
+   are kept iff |dx| < r and |dy| < r (the square circumscribing the disc, same strictness).
+   Every function below takes window="circle" (CLEAR, the default) or window="square".
+
 Readings where the pages leave a step open (each listed with its reason in the design notes):
 strict "<" in the radius test; image tokens in row-major order t = n_text + y*W + x; windows are
 clipped at the grid border (border queries see fewer keys); text queries attend to every token
@@ -57,18 +64,26 @@ def token_coords(n_text: int, H: int, W: int):
     return y, x, is_text
 
 
-def clear_mask(n_text: int, H: int, W: int, r: int, rows=None) -> np.ndarray:
+WINDOWS = ("circle", "square")
+
+
+def clear_mask(n_text: int, H: int, W: int, r: int, rows=None, window: str = "circle") -> np.ndarray:
     """Boolean CLEAR mask M [len(rows), T] (all T rows if rows is None).
 
     [pith review, "Core claim"]: M_ij = 1 if i <= n_text or j <= n_text or
-    (d^x_ij)^2 + (d^y_ij)^2 < r^2 (1-based there; 0-based "< n_text" here).
+    (d^x_ij)^2 + (d^y_ij)^2 < r^2 (1-based there; 0-based "< n_text" here). With window="square"
+    the last test is |dx| < r and |dy| < r.
     """
+    assert window in WINDOWS
     y, x, is_text = token_coords(n_text, H, W)
     T = y.shape[0]
     rows = np.arange(T) if rows is None else np.asarray(rows, dtype=np.int64)
     dy = y[rows][:, None] - y[None, :]
     dx = x[rows][:, None] - x[None, :]
-    near = dx * dx + dy * dy < r * r
+    if window == "circle":
+        near = dx * dx + dy * dy < r * r
+    else:
+        near = (np.abs(dx) < r) & (np.abs(dy) < r)
     return is_text[rows][:, None] | is_text[None, :] | near
 
 
@@ -93,7 +108,7 @@ def _masked_softmax_rows(S: np.ndarray, M: np.ndarray):
     return P, lse
 
 
-def clear_attention_forward(q, k, v, n_text: int, H: int, W: int, r: int, scale=None):
+def clear_attention_forward(q, k, v, n_text: int, H: int, W: int, r: int, scale=None, window: str = "circle"):
     """O = softmax_M(Q K^T * scale) V and LSE for every (batch, head).
 
     q, k, v: [B, heads, T, d] (numpy or torch; upcast exactly to float64).
@@ -104,7 +119,7 @@ def clear_attention_forward(q, k, v, n_text: int, H: int, W: int, r: int, scale=
     B, Hh, T, d = q.shape
     assert T == n_text + H * W, "T must equal n_text + H*W"
     scale = 1.0 / math.sqrt(d) if scale is None else scale
-    M = clear_mask(n_text, H, W, r)
+    M = clear_mask(n_text, H, W, r, window=window)
     O = np.empty_like(q)
     LSE = np.empty((B, Hh, T))
     for b in range(B):
@@ -117,7 +132,7 @@ def clear_attention_forward(q, k, v, n_text: int, H: int, W: int, r: int, scale=
 
 
 def clear_attention_rows(q, k, v, n_text: int, H: int, W: int, r: int, b: int, h: int, rows,
-                         scale=None):
+                         scale=None, window: str = "circle"):
     """Forward outputs for selected query rows of one (b, h) only; mask rows built explicitly.
 
     Used where the full T x T mask does not fit (e.g. a 512 x 512 grid, T = 262,656).
@@ -127,13 +142,14 @@ def clear_attention_rows(q, k, v, n_text: int, H: int, W: int, r: int, b: int, h
     kb, vb = _as_f64(k[b, h]), _as_f64(v[b, h])
     d = qb.shape[-1]
     scale = 1.0 / math.sqrt(d) if scale is None else scale
-    M = clear_mask(n_text, H, W, r, rows=rows)
+    M = clear_mask(n_text, H, W, r, rows=rows, window=window)
     S = (qb @ kb.T) * scale
     P, lse = _masked_softmax_rows(S, M)
     return P @ vb, lse
 
 
-def clear_attention_backward(q, k, v, dO, n_text: int, H: int, W: int, r: int, scale=None):
+def clear_attention_backward(q, k, v, dO, n_text: int, H: int, W: int, r: int, scale=None,
+                             window: str = "circle"):
     """Analytic gradient of the forward above with respect to q, k and v, given dO.
 
     With S = scale * Q K^T, P = softmax_M(S) row-wise and O = P V:
@@ -148,7 +164,7 @@ def clear_attention_backward(q, k, v, dO, n_text: int, H: int, W: int, r: int, s
     q, k, v, dO = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(dO)
     B, Hh, T, d = q.shape
     scale = 1.0 / math.sqrt(d) if scale is None else scale
-    M = clear_mask(n_text, H, W, r)
+    M = clear_mask(n_text, H, W, r, window=window)
     dq = np.empty_like(q)
     dk = np.empty_like(k)
     dv = np.empty_like(v)
@@ -170,12 +186,22 @@ def clear_attention_backward(q, k, v, dO, n_text: int, H: int, W: int, r: int, s
 # Counting: window size, kept pairs, useful FLOPs
 # ----------------------------------------------------------------------------------------------
 
-def window_lattice_count(r: int) -> int:
+def window_half_width(r: int, ady: int, window: str = "circle") -> int:
+    """Largest dx >= 0 kept at vertical distance ady >= 0, or -1 if none."""
+    if window == "square":
+        return r - 1 if ady < r else -1
+    rem = r * r - ady * ady
+    return math.isqrt(rem - 1) if rem > 0 else -1  # largest dx with dx^2 < rem
+
+
+def window_lattice_count(r: int, window: str = "circle") -> int:
     """Keys in an interior query's window: #{(dx, dy) in Z^2 : dx^2 + dy^2 < r^2}.
 
     [pith review, "What carries the argument"]: the window's key count is constant in the
-    resolution and is about pi/4 of the square window's.
+    resolution and is about pi/4 of the square window's. window="square" counts |dx|, |dy| < r.
     """
+    if window == "square":
+        return (2 * r - 1) ** 2
     n = 0
     for dy in range(-r, r + 1):
         rem = r * r - dy * dy
@@ -186,24 +212,24 @@ def window_lattice_count(r: int) -> int:
     return n
 
 
-def window_pairs(H: int, W: int, r: int) -> int:
+def window_pairs(H: int, W: int, r: int, window: str = "circle") -> int:
     """Kept image-image pairs P(r) with border clipping: sum over offsets of the overlap area."""
     total = 0
     for dy in range(-(r - 1), r):
-        rem = r * r - dy * dy
-        w = math.isqrt(rem - 1)
+        w = window_half_width(r, abs(dy), window)
         for dx in range(-w, w + 1):
             total += max(0, H - abs(dy)) * max(0, W - abs(dx))
     return total
 
 
-def kept_pairs(n_text: int, H: int, W: int, r: int) -> int:
+def kept_pairs(n_text: int, H: int, W: int, r: int, window: str = "circle") -> int:
     """Number of ones in M: text rows (all T keys) + image rows x text keys + window pairs."""
     N = H * W
     T = n_text + N
-    return n_text * T + N * n_text + window_pairs(H, W, r)
+    return n_text * T + N * n_text + window_pairs(H, W, r, window)
 
 
-def useful_flops_fwd(B: int, heads: int, n_text: int, H: int, W: int, r: int, d: int) -> int:
+def useful_flops_fwd(B: int, heads: int, n_text: int, H: int, W: int, r: int, d: int,
+                     window: str = "circle") -> int:
     """Forward FLOPs on kept pairs only: 2*d for q.k plus 2*d for p*v, per kept (q, k) pair."""
-    return 4 * d * B * heads * kept_pairs(n_text, H, W, r)
+    return 4 * d * B * heads * kept_pairs(n_text, H, W, r, window)

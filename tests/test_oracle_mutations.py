@@ -8,9 +8,10 @@ import pytest
 import oracle
 import oracle.clear_attention as oc
 import test_oracle as pins
+import test_oracle_square as sq_pins
 
 
-def _mask_le(n_text, H, W, r, rows=None):          # "<=" instead of the printed strict "<"
+def _mask_le(n_text, H, W, r, rows=None, window="circle"):  # "<=" instead of the printed strict "<"
     y, x, is_text = oc.token_coords(n_text, H, W)
     rows = np.arange(y.shape[0]) if rows is None else np.asarray(rows)
     dy = y[rows][:, None] - y[None, :]
@@ -18,7 +19,7 @@ def _mask_le(n_text, H, W, r, rows=None):          # "<=" instead of the printed
     return is_text[rows][:, None] | is_text[None, :] | (dx * dx + dy * dy <= r * r)
 
 
-def _mask_no_global_text_rows(n_text, H, W, r, rows=None):   # text queries only see text keys
+def _mask_no_global_text_rows(n_text, H, W, r, rows=None, window="circle"):  # text rows: text keys only
     y, x, is_text = oc.token_coords(n_text, H, W)
     rows = np.arange(y.shape[0]) if rows is None else np.asarray(rows)
     dy = y[rows][:, None] - y[None, :]
@@ -34,7 +35,7 @@ def _softmax_no_max(S, M):                         # forgets the max shift: LSE 
     return E / l, np.log(l)[:, 0] + 1e-3
 
 
-def _kept_pairs_square(n_text, H, W, r):           # counts the square window, not the disc
+def _kept_pairs_square(n_text, H, W, r, window="circle"):  # counts the square window, not the disc
     N = H * W
     T = n_text + N
     tot = 0
@@ -44,11 +45,11 @@ def _kept_pairs_square(n_text, H, W, r):           # counts the square window, n
     return n_text * T + N * n_text + tot
 
 
-def _backward_no_D(q, k, v, dO, n_text, H, W, r, scale=None):   # drops the D = rowsum(dO o O) term
+def _backward_no_D(q, k, v, dO, n_text, H, W, r, scale=None, window="circle"):  # drops D = rowsum(dO o O)
     q, k, v, dO = (oc._as_f64(a) for a in (q, k, v, dO))
     B, Hh, T, d = q.shape
     scale = 1.0 / math.sqrt(d) if scale is None else scale
-    M = oc.clear_mask(n_text, H, W, r)
+    M = oc.clear_mask(n_text, H, W, r, window=window)
     dq, dk, dv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
     for b in range(B):
         for h in range(Hh):
@@ -60,12 +61,45 @@ def _backward_no_D(q, k, v, dO, n_text, H, W, r, scale=None):   # drops the D = 
     return dq, dk, dv
 
 
-def _backward_transposed_dk(q, k, v, dO, n_text, H, W, r, scale=None):   # dK from dS, not dS^T
-    dq, dk, dv = _orig_backward(q, k, v, dO, n_text, H, W, r, scale)
+def _backward_transposed_dk(q, k, v, dO, n_text, H, W, r, scale=None, window="circle"):  # dK from dS
+    dq, dk, dv = _orig_backward(q, k, v, dO, n_text, H, W, r, scale, window)
     return dq, dk[:, :, ::-1].copy(), dv
 
 
 _orig_backward = oc.clear_attention_backward
+_orig_mask = oc.clear_mask
+
+
+def _square_le(n_text, H, W, r, rows=None, window="circle"):  # square window with "<=" at its edge
+    if window != "square":
+        return _orig_mask(n_text, H, W, r, rows, window)
+    y, x, is_text = oc.token_coords(n_text, H, W)
+    rows = np.arange(y.shape[0]) if rows is None else np.asarray(rows)
+    dy = y[rows][:, None] - y[None, :]
+    dx = x[rows][:, None] - x[None, :]
+    return is_text[rows][:, None] | is_text[None, :] | ((np.abs(dx) <= r) & (np.abs(dy) <= r))
+
+
+def _square_is_circle(n_text, H, W, r, rows=None, window="circle"):  # ignores the window argument
+    return _orig_mask(n_text, H, W, r, rows, "circle")
+
+
+def _all_square_pins():
+    """Run every square-window pin; return the number that failed."""
+    failures = 0
+    calls = [
+        lambda: sq_pins.test_square_matches_brute_force(3, 5, 7),
+        lambda: [sq_pins.test_square_interior_row_count(r) for r in (2, 4)],
+        lambda: sq_pins.test_square_kept_pairs_equals_mask_sum(3, 10, 5, 6),
+        lambda: sq_pins.test_circle_is_inside_square(1, 9, 9, 4),
+        lambda: sq_pins.test_square_full_radius_is_full_attention(4, 6, 9),
+    ]
+    for c in calls:
+        try:
+            c()
+        except AssertionError:
+            failures += 1
+    return failures
 
 
 def _all_pins():
@@ -101,6 +135,13 @@ def _patch_mask(monkeypatch, fn):
 
 def test_unmutated_oracle_passes_all_pins():
     assert _all_pins() == 0
+    assert _all_square_pins() == 0
+
+
+@pytest.mark.parametrize("mutant", [_square_le, _square_is_circle])
+def test_square_mutant_is_caught(monkeypatch, mutant):
+    _patch_mask(monkeypatch, mutant)
+    assert _all_square_pins() >= 1, f"mutant {mutant.__name__} survived every square pin"
 
 
 @pytest.mark.parametrize("mutant", ["mask_le", "coords_swapped", "no_global_text_rows",
