@@ -64,7 +64,12 @@ typedef struct {
   int H, W;     /* image token grid, >= 1 each */
   int d;        /* head dim: 64 or 128 */
   int r;        /* window radius in grid units (strict: dx^2 + dy^2 < r^2), >= 1 */
+  int window;   /* CLEAR_WINDOW_CIRCLE (0, CLEAR's mask) or CLEAR_WINDOW_SQUARE (1): keep image pairs
+                   with |dx| < r and |dy| < r instead, the square sliding window the pages compare
+                   the circle with. Any other value is CLEAR_ERR_INVALID_ARG. */
 } clear_attn_params_t;
+
+enum { CLEAR_WINDOW_CIRCLE = 0, CLEAR_WINDOW_SQUARE = 1 };
 
 /* Library version (major * 10000 + minor * 100 + patch). */
 CLEAR_API int clear_attn_version(void);

@@ -29,7 +29,14 @@ STATUS_NAMES = {0: "CLEAR_OK", 1: "CLEAR_ERR_INVALID_ARG", 2: "CLEAR_ERR_UNSUPPO
 class ClearParams(ctypes.Structure):
     """Mirror of clear_attn_params_t."""
     _fields_ = [("B", ctypes.c_int), ("heads", ctypes.c_int), ("n_text", ctypes.c_int), ("H", ctypes.c_int),
-                ("W", ctypes.c_int), ("d", ctypes.c_int), ("r", ctypes.c_int)]
+                ("W", ctypes.c_int), ("d", ctypes.c_int), ("r", ctypes.c_int), ("window", ctypes.c_int)]
+
+
+WINDOWS = {"circle": 0, "square": 1}  # CLEAR_WINDOW_CIRCLE, CLEAR_WINDOW_SQUARE
+
+
+def _window_code(window) -> int:
+    return WINDOWS[window] if isinstance(window, str) else int(window)
 
 
 class ClearError(RuntimeError):
@@ -82,8 +89,8 @@ def header_functions() -> list[str]:
     return sorted(set(re.findall(r"\b(clear_[a-z_]+)\s*\(", text)))
 
 
-def make_params(B: int, heads: int, n_text: int, H: int, W: int, d: int, r: int) -> ClearParams:
-    return ClearParams(B, heads, n_text, H, W, d, r)
+def make_params(B: int, heads: int, n_text: int, H: int, W: int, d: int, r: int, window="circle") -> ClearParams:
+    return ClearParams(B, heads, n_text, H, W, d, r, _window_code(window))
 
 
 def version() -> int:
@@ -157,14 +164,16 @@ def _check_qkv(name, t, shape):
         raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {tuple(shape)}")
 
 
-def clear_attn_fwd(q, k, v, n_text: int, H: int, W: int, r: int, o=None, lse=None, workspace=None, stream=None):
-    """CLEAR attention forward through the C ABI. Returns (o, lse); raises ClearError on failure."""
+def clear_attn_fwd(q, k, v, n_text: int, H: int, W: int, r: int, o=None, lse=None, workspace=None, stream=None,
+                   window="circle"):
+    """CLEAR attention forward through the C ABI. Returns (o, lse); raises ClearError on failure.
+    window: "circle" (CLEAR's mask) or "square" (|dx| < r and |dy| < r)."""
     B, heads, T, d = q.shape
     if T != n_text + H * W:
         raise ValueError("T must equal n_text + H * W")
     for name, t in (("q", q), ("k", k), ("v", v)):
         _check_qkv(name, t, q.shape)
-    p = make_params(B, heads, n_text, H, W, d, r)
+    p = make_params(B, heads, n_text, H, W, d, r, window)
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
@@ -181,14 +190,14 @@ def clear_attn_fwd(q, k, v, n_text: int, H: int, W: int, r: int, o=None, lse=Non
 
 
 def clear_attn_bwd(q, k, v, o, lse, dO, n_text: int, H: int, W: int, r: int, dq=None, dk=None, dv=None,
-                   workspace=None, stream=None):
-    """CLEAR attention backward through the C ABI. Returns (dq, dk, dv)."""
+                   workspace=None, stream=None, window="circle"):
+    """CLEAR attention backward through the C ABI. Returns (dq, dk, dv). window as for the forward."""
     B, heads, T, d = q.shape
     if T != n_text + H * W:
         raise ValueError("T must equal n_text + H * W")
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dO", dO)):
         _check_qkv(name, t, q.shape)
-    p = make_params(B, heads, n_text, H, W, d, r)
+    p = make_params(B, heads, n_text, H, W, d, r, window)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv

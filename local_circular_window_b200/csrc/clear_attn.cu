@@ -23,7 +23,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 namespace {
 
-constexpr int kVersion = 100;  // 0.1.0
+constexpr int kVersion = 110;  // 0.1.1: window shape in the params
 
 // ------------------------------------------------------------------------------------------------
 // Validation
@@ -33,8 +33,10 @@ struct Checked {
   Geom g;
 };
 
-// Radius beyond which every pair of the grid is kept; larger radii are clamped to it.
-int full_radius(int H, int W) {
+// Radius beyond which every pair of the grid is kept; larger radii are clamped to it. Circle: the
+// smallest r with r^2 above the squared diagonal; square: max(H, W).
+int full_radius(int H, int W, int window) {
+  if (window == kSquare) return H > W ? H : W;
   long long d2 = (long long)(H - 1) * (H - 1) + (long long)(W - 1) * (W - 1);
   long long r = (long long)std::sqrt((double)d2);
   while (r * r > d2) --r;
@@ -47,6 +49,7 @@ Checked check_params(const clear_attn_params_t* p) {
   c.st = CLEAR_ERR_INVALID_ARG;
   if (!p) return c;
   if (p->B < 1 || p->heads < 1 || p->n_text < 0 || p->H < 1 || p->W < 1 || p->r < 1) return c;
+  if (p->window != kCircle && p->window != kSquare) return c;
   if (p->d != 64 && p->d != 128) {
     c.st = CLEAR_ERR_UNSUPPORTED;
     return c;
@@ -56,12 +59,13 @@ Checked check_params(const clear_attn_params_t* p) {
   const long long BH = (long long)p->B * p->heads;
   if (N > (1ll << 28) || p->n_text > (1 << 24) || T > (1ll << 30) || BH > (1ll << 20)) return c;
   if (BH * T * p->d >= (1ll << 40)) return c;
-  const int r = p->r < full_radius(p->H, p->W) ? p->r : full_radius(p->H, p->W);
+  const int rfull = full_radius(p->H, p->W, p->window);
+  const int r = p->r < rfull ? p->r : rfull;
   if (hw_table_size(r, p->H) > kMaxHwTable) {  // half-width table must fit in shared memory
     c.st = CLEAR_ERR_UNSUPPORTED;
     return c;
   }
-  c.g = make_geom(p->B, p->heads, p->n_text, p->H, p->W, p->d, r);
+  c.g = make_geom(p->B, p->heads, p->n_text, p->H, p->W, p->d, r, p->window);
   c.st = CLEAR_OK;
   return c;
 }
@@ -445,10 +449,10 @@ clear_status_t clear_sched_pair_counts(const clear_attn_params_t* params, long l
   const Checked c = check_params(params);
   if (c.st != CLEAR_OK) return c.st;
   const Geom& g = c.g;
-  // Kept pairs: text rows see all T keys, image rows see all text keys plus their clipped disc.
+  // Kept pairs: text rows see all T keys, image rows see all text keys plus their clipped window.
   long long win = 0;
   for (int dy = -(g.r - 1); dy <= g.r - 1; ++dy) {
-    const int w = half_width(g.r, dy < 0 ? -dy : dy);
+    const int w = half_width(g.r, dy < 0 ? -dy : dy, g.window);
     if (w < 0) continue;
     const long long rows = g.H - (dy < 0 ? -dy : dy);
     if (rows <= 0) continue;

@@ -80,7 +80,7 @@ __device__ __forceinline__ uint32_t rect_row_bits(const Geom& g, const int* wtab
   const int dy = ky - yp;
   const int ady = dy < 0 ? -dy : dy;
   if (ady >= g.r) return 0u;
-  const int wdt = (ady < kMaxRTable) ? wtab[ady] : half_width(g.r, ady);
+  const int wdt = (ady < kMaxRTable) ? wtab[ady] : half_width(g.r, ady, g.window);
   if (wdt < 0) return 0u;
   int lo = imax(xp - wdt, 0) - kx;
   int hi = imin(xp + wdt, g.W - 1) - kx;
@@ -268,7 +268,7 @@ clear_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_c
     *abort_flag = 0;
     fence_barrier_init();
   }
-  for (int i = threadIdx.x; i < kMaxRTable; i += blockDim.x) wtab[i] = half_width(g.r, i);
+  for (int i = threadIdx.x; i < kMaxRTable; i += blockDim.x) wtab[i] = half_width(g.r, i, g.window);
   if (warp == 9) {
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
@@ -567,7 +567,7 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
     *abort_flag = 0;
     fence_barrier_init();
   }
-  for (int i = threadIdx.x; i < kMaxRTable; i += blockDim.x) wtab[i] = half_width(g.r, i);
+  for (int i = threadIdx.x; i < kMaxRTable; i += blockDim.x) wtab[i] = half_width(g.r, i, g.window);
   if (warp == 9) {
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();

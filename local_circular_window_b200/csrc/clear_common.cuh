@@ -32,7 +32,7 @@ __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* lin, 
 }
 
 // Half-width for |dy| beyond the shared-memory table (only for radii above kMaxRTable).
-__device__ __noinline__ int half_width_slow(int r, int dy) { return half_width(r, dy); }
+__device__ __noinline__ int half_width_slow(int r, int dy, int window) { return half_width(r, dy, window); }
 
 // Kept column range [lo, hi] (tile-local, 0..15) of key row ky of a rectangle tile starting at
 // column kx, seen from grid point (yq, xq): keys inside the grid with dx^2 + dy^2 < r^2. An empty
@@ -42,7 +42,7 @@ __device__ __forceinline__ void rect_row_range(const Geom& g, const int* wtab, i
                                                int* lo_out, int* hi_out) {
   const int dy = ky - yq;
   const int ady = dy < 0 ? -dy : dy;
-  int w = (ady < kMaxRTable) ? wtab[ady] : half_width_slow(g.r, ady);
+  int w = (ady < kMaxRTable) ? wtab[ady] : half_width_slow(g.r, ady, g.window);
   if ((unsigned)ky >= (unsigned)g.H) w = -1;
   int lo = imax(imax(xq - w, 0) - kx, 0);
   int hi = imin(imin(xq + w, g.W - 1) - kx, kKW - 1);

@@ -160,9 +160,9 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
   }
   // Half-width tables: wtab[dy] (tile enumeration, first kMaxRTable rows) and the int16 table
   // hwtab[dy] for every |dy| < min(r, H) (masks).
-  for (int i = threadIdx.x; i < kMaxRTable; i += blockDim.x) wtab[i] = half_width(g.r, i);
+  for (int i = threadIdx.x; i < kMaxRTable; i += blockDim.x) wtab[i] = half_width(g.r, i, g.window);
   const int hwn = hw_table_size(g.r, g.H);
-  for (int i = threadIdx.x; i < hwn; i += blockDim.x) hwtab[i] = (int16_t)half_width(g.r, i);
+  for (int i = threadIdx.x; i < hwn; i += blockDim.x) hwtab[i] = (int16_t)half_width(g.r, i, g.window);
   if (warp == 9) {
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();

@@ -57,8 +57,13 @@ struct KeyTile {
   int flags;  // kFull or kNeedsMask
 };
 
+// Window shapes: the circle (CLEAR's mask, dx^2 + dy^2 < r^2) and the square of the same radius
+// (|dx| < r and |dy| < r). Everything downstream sees a window only through half_width and within.
+enum WindowShape : int { kCircle = 0, kSquare = 1 };
+
 struct Geom {
   int B, heads, n_text, H, W, d, r;
+  int window;        // WindowShape
   int T, BH;
   int nqy, nqx, nQ;  // image query tiles per (b, h): ceil(H/8) x ceil(W/16)
   int nTq;           // text query tiles: ceil(n_text / 128)
@@ -89,11 +94,18 @@ CLEAR_HD int isqrt_below(int rem) {
   return w;
 }
 
-// Horizontal half-width of the window at vertical distance dy: largest dx with dx^2 + dy^2 < r^2,
-// or -1 when no key at that vertical distance is within radius.
-CLEAR_HD int half_width(int r, int dy) {
+// Horizontal half-width of the window at vertical distance dy >= 0: the largest kept dx, or -1
+// when no key at that vertical distance is kept. Circle: largest dx with dx^2 + dy^2 < r^2;
+// square: r - 1 for dy < r.
+CLEAR_HD int half_width(int r, int dy, int window = kCircle) {
+  if (window == kSquare) return dy < r ? r - 1 : -1;
   int rem = r * r - dy * dy;
   return rem <= 0 ? -1 : isqrt_below(rem);
+}
+
+// Whether the offset (dx, dy), both >= 0, is inside the window.
+CLEAR_HD bool within(int r, int window, int dx, int dy) {
+  return window == kSquare ? (dx < r && dy < r) : (dx * dx + dy * dy < r * r);
 }
 
 // Text split count: enough splits that each covers about `target` chunks, capped so the fp32
@@ -111,9 +123,10 @@ CLEAR_HD void choose_splits(int nC, int target, int max_splits, int* S, int* cps
 constexpr int kSplitTargetChunks = 64;
 constexpr int kMaxSplits = 32;
 
-CLEAR_HD Geom make_geom(int B, int heads, int n_text, int H, int W, int d, int r) {
+CLEAR_HD Geom make_geom(int B, int heads, int n_text, int H, int W, int d, int r, int window = kCircle) {
   Geom g;
   g.B = B; g.heads = heads; g.n_text = n_text; g.H = H; g.W = W; g.d = d; g.r = r;
+  g.window = window;
   g.T = n_text + H * W;
   g.BH = B * heads;
   g.nqy = cdiv(H, kQH);
@@ -179,7 +192,7 @@ struct KeyIter {
   // fixed per item
   const int* wtab;        // optional half-width table (device shared memory), entries [0, wtab_n)
   int wtab_n;
-  int is_text, r, H, W, n_text, T;
+  int is_text, r, window, H, W, n_text, T;
   int y0, yl, x0, xl;     // image query tile, clipped to the grid (rows y0..yl, cols x0..xl)
   int ky_begin, ky_end;   // key rows that any query of the tile can reach
   // state
@@ -190,7 +203,7 @@ struct KeyIter {
   CLEAR_HD void init(const Geom& g, const WorkItem& it, const int* table = nullptr, int table_n = 0) {
     wtab = table;
     wtab_n = table_n;
-    is_text = it.is_text; r = g.r; H = g.H; W = g.W; n_text = g.n_text; T = g.T;
+    is_text = it.is_text; r = g.r; window = g.window; H = g.H; W = g.W; n_text = g.n_text; T = g.T;
     if (is_text) {
       lin_next = it.c_begin;
       lin_end = it.c_end;
@@ -217,7 +230,7 @@ struct KeyIter {
       if (band_ky > ky_end) return false;
       int band_last = imin(band_ky + kKH - 1, H - 1);
       int dmin = imax(0, imax(y0 - band_last, band_ky - yl));
-      int w = (dmin < wtab_n) ? wtab[dmin] : half_width(r, dmin);
+      int w = (dmin < wtab_n) ? wtab[dmin] : half_width(r, dmin, window);
       if (w < 0) continue;
       kx = imax(0, x0 - w);
       kx_end = imin(W - 1, xl + w);
@@ -247,7 +260,7 @@ struct KeyIter {
     bool inside = (band_ky + kKH - 1 <= H - 1) && (kx + kKW - 1 <= W - 1);
     int mdy = imax(band_ky + kKH - 1 - y0, yl - band_ky);
     int mdx = imax(kx + kKW - 1 - x0, xl - kx);
-    t->flags = (inside && mdy * mdy + mdx * mdx < r * r) ? kFull : kNeedsMask;
+    t->flags = (inside && within(r, window, mdx, mdy)) ? kFull : kNeedsMask;
     kx += kKW;
     return true;
   }
@@ -313,7 +326,7 @@ CLEAR_HD PairItem decode_pair(const Geom& g, long long w) {
 struct PairKeyIter {
   const int* wtab;
   int wtab_n;
-  int is_text, r, H, W, n_text, T, validB;
+  int is_text, r, window, H, W, n_text, T, validB;
   int y0, x0, xl;             // block origin, last column
   int yA0, yAl, yB0, yBl;     // half rows (clipped); B rows only if validB
   int ky_begin, ky_end;
@@ -324,7 +337,8 @@ struct PairKeyIter {
   CLEAR_HD void init(const Geom& g, const PairItem& it, const int* table = nullptr, int table_n = 0) {
     wtab = table;
     wtab_n = table_n;
-    is_text = it.is_text; r = g.r; H = g.H; W = g.W; n_text = g.n_text; T = g.T; validB = it.validB;
+    is_text = it.is_text; r = g.r; window = g.window; H = g.H; W = g.W; n_text = g.n_text; T = g.T;
+    validB = it.validB;
     if (is_text) {
       lin_next = it.c_begin;
       lin_end = it.c_end;
@@ -348,7 +362,7 @@ struct PairKeyIter {
     kx = 1; kx_end = 0;
   }
 
-  CLEAR_HD int hw(int dy) const { return (dy < wtab_n) ? wtab[dy] : half_width(r, dy); }
+  CLEAR_HD int hw(int dy) const { return (dy < wtab_n) ? wtab[dy] : half_width(r, dy, window); }
 
   // Next band with kept columns. The first and last bands are reached by one half only (the
   // top ones by half A, the bottom ones by half B); alternating from both ends keeps both halves
@@ -376,11 +390,11 @@ struct PairKeyIter {
     const int kxl = imin(kxx + kKW - 1, W - 1);
     const int dy = imax(0, imax(qa - kyl, ky - qb));
     const int dx = imax(0, imax(x0 - kxl, kxx - xl));
-    if (dy * dy + dx * dx >= r * r) return 0;
+    if (!within(r, window, dx, dy)) return 0;
     const bool inside = (ky + kFKH - 1 <= H - 1) && (kxx + kKW - 1 <= W - 1);
     const int mdy = imax(ky + kFKH - 1 - qa, qb - ky);
     const int mdx = imax(kxx + kKW - 1 - x0, xl - kxx);
-    return need_bit | ((inside && mdy * mdy + mdx * mdx < r * r) ? full_bit : 0);
+    return need_bit | ((inside && within(r, window, mdx, mdy)) ? full_bit : 0);
   }
 
   CLEAR_HD bool next(KeyTile* t) {

@@ -26,7 +26,7 @@ def test_version_and_status_strings():
 
 @pytest.mark.parametrize("fields,expected", [
     (dict(r=0), 1), (dict(B=0), 1), (dict(heads=0), 1), (dict(H=0), 1), (dict(W=-3), 1), (dict(n_text=-1), 1),
-    (dict(d=96), 2), (dict(d=256), 2), (dict(H=1 << 15, W=1 << 15), 1), (dict(n_text=1 << 25), 1),
+    (dict(d=96), 2), (dict(d=256), 2), (dict(window=2), 1), (dict(window=-1), 1), (dict(H=1 << 15, W=1 << 15), 1), (dict(n_text=1 << 25), 1),
 ])
 def test_invalid_params_statuses(fields, expected):
     base = dict(B=1, heads=2, n_text=16, H=16, W=16, d=64, r=4)

@@ -54,12 +54,13 @@ NEED = (1, 2)
 FULL = (4, 8)
 
 
+@pytest.mark.parametrize("window", ["circle", "square"])
 @pytest.mark.parametrize("n_text,H,W,r", CASES)
-def test_tiles_cover_mask_exactly(n_text, H, W, r):
-    p = L.make_params(1, 1, n_text, H, W, 64, r)
+def test_tiles_cover_mask_exactly(n_text, H, W, r, window):
+    p = L.make_params(1, 1, n_text, H, W, 64, r, window)
     T = n_text + H * W
     n_txt_items, n_img_items, S, cps = L.forward_shape(p)
-    M = oracle.clear_mask(n_text, H, W, r) if T <= 4000 else None
+    M = oracle.clear_mask(n_text, H, W, r, window=window) if T <= 4000 else None
     text_cover = {}
     for item in range(n_txt_items + n_img_items):
         q_info, tiles = L.item_tiles(p, item)
@@ -76,7 +77,7 @@ def test_tiles_cover_mask_exactly(n_text, H, W, r):
             if not queries:
                 assert not any(t[3] & NEED[half] for t in tiles)
                 continue
-            rows = M[queries] if M is not None else oracle.clear_mask(n_text, H, W, r, rows=queries)
+            rows = M[queries] if M is not None else oracle.clear_mask(n_text, H, W, r, rows=queries, window=window)
             need = set(np.nonzero(rows.any(axis=0))[0].tolist())
             covered = set(k for t in tiles if t[3] & NEED[half] for k in _keys_of_tile(t, n_text, H, W, T))
             if not q_info[0]:  # a text split covers its own key range only (checked across splits below)
@@ -94,11 +95,12 @@ def test_tiles_cover_mask_exactly(n_text, H, W, r):
         assert sorted(keys) == list(range(T))
 
 
+@pytest.mark.parametrize("window", ["circle", "square"])
 @pytest.mark.parametrize("n_text,H,W,r", CASES[:6])
-def test_pair_counts(n_text, H, W, r):
-    p = L.make_params(2, 3, n_text, H, W, 64, r)
+def test_pair_counts(n_text, H, W, r, window):
+    p = L.make_params(2, 3, n_text, H, W, 64, r, window)
     useful, executed = L.pair_counts(p)
-    assert useful == 6 * oracle.kept_pairs(n_text, H, W, r)
+    assert useful == 6 * oracle.kept_pairs(n_text, H, W, r, window)
     assert executed >= useful
     n_txt_items, n_img_items, S, cps = L.forward_shape(p)
     products = 0
@@ -113,6 +115,16 @@ def test_radius_beyond_diagonal_is_clamped_to_full_attention():
     useful, executed = L.pair_counts(p)
     T = 16 + 256
     assert useful == T * T
+
+
+@pytest.mark.parametrize("r,full", [(1000, True), (16, True), (15, False)])
+def test_square_radius_clamp(r, full):
+    # The square keeps every pair once r >= max(H, W) (here 16 x 12); r = 15 drops the far corners.
+    p = L.make_params(1, 1, 8, 16, 12, 64, r, "square")
+    useful, _ = L.pair_counts(p)
+    T = 8 + 16 * 12
+    assert (useful == T * T) == full
+    assert useful == oracle.kept_pairs(8, 16, 12, min(r, 16), "square")
 
 
 def test_split_shape_at_8k():
