@@ -28,6 +28,13 @@ Revs Pre-Trained Diffusion Transformers Up"):
    carries the argument"]. Read as the same rule with the Chebyshev distance: image tokens i and j
    are kept iff |dx| < r and |dy| < r (the square circumscribing the disc, same strictness).
    Every function below takes window="circle" (CLEAR, the default) or window="square".
+6. Border-shifted square window (the other comparison mask): the pages name Neighborhood
+   Attention as the prior art CLEAR builds on [codewithpapers page, "Builds on"; pith review,
+   desk verdict: "neighborhood attention with a circular window"]. Neighborhood attention keeps
+   a fixed square of (2r-1) x (2r-1) keys per query and, at the grid border, shifts the window
+   inward instead of clipping it, so every query sees the same number of keys. Read here as:
+   image pair (i, j) kept iff |y_j - cy(y_i)| < r and |x_j - cx(x_i)| < r with the centre clamped,
+   cy(y) = min(max(y, r-1), H-r) (likewise cx); it needs H, W >= 2r-1. window="shifted".
 
 Readings where the pages leave a step open (each listed with its reason in the design notes):
 strict "<" in the radius test; image tokens in row-major order t = n_text + y*W + x; windows are
@@ -64,7 +71,7 @@ def token_coords(n_text: int, H: int, W: int):
     return y, x, is_text
 
 
-WINDOWS = ("circle", "square")
+WINDOWS = ("circle", "square", "shifted")
 
 
 def clear_mask(n_text: int, H: int, W: int, r: int, rows=None, window: str = "circle") -> np.ndarray:
@@ -82,8 +89,13 @@ def clear_mask(n_text: int, H: int, W: int, r: int, rows=None, window: str = "ci
     dx = x[rows][:, None] - x[None, :]
     if window == "circle":
         near = dx * dx + dy * dy < r * r
-    else:
+    elif window == "square":
         near = (np.abs(dx) < r) & (np.abs(dy) < r)
+    else:  # border-shifted square: distances from the clamped window centre of the query
+        assert H >= 2 * r - 1 and W >= 2 * r - 1, "the shifted window needs H, W >= 2r - 1"
+        cy = np.clip(y[rows], r - 1, H - r)[:, None]
+        cx = np.clip(x[rows], r - 1, W - r)[:, None]
+        near = (np.abs(y[None, :] - cy) < r) & (np.abs(x[None, :] - cx) < r)
     return is_text[rows][:, None] | is_text[None, :] | near
 
 
@@ -187,20 +199,20 @@ def clear_attention_backward(q, k, v, dO, n_text: int, H: int, W: int, r: int, s
 # ----------------------------------------------------------------------------------------------
 
 def window_half_width(r: int, ady: int, window: str = "circle") -> int:
-    """Largest dx >= 0 kept at vertical distance ady >= 0, or -1 if none."""
-    if window == "square":
+    """Largest dx >= 0 kept at vertical distance ady >= 0 (from the window centre), or -1 if none."""
+    if window in ("square", "shifted"):
         return r - 1 if ady < r else -1
     rem = r * r - ady * ady
     return math.isqrt(rem - 1) if rem > 0 else -1  # largest dx with dx^2 < rem
 
 
-def window_lattice_count(r: int, window: str = "circle") -> int:
+def window_lattice_count(r: int, window: str = "circle") -> int:  # noqa: C901
     """Keys in an interior query's window: #{(dx, dy) in Z^2 : dx^2 + dy^2 < r^2}.
 
     [pith review, "What carries the argument"]: the window's key count is constant in the
     resolution and is about pi/4 of the square window's. window="square" counts |dx|, |dy| < r.
     """
-    if window == "square":
+    if window in ("square", "shifted"):
         return (2 * r - 1) ** 2
     n = 0
     for dy in range(-r, r + 1):
@@ -213,7 +225,10 @@ def window_lattice_count(r: int, window: str = "circle") -> int:
 
 
 def window_pairs(H: int, W: int, r: int, window: str = "circle") -> int:
-    """Kept image-image pairs P(r) with border clipping: sum over offsets of the overlap area."""
+    """Kept image-image pairs P(r) with border clipping: sum over offsets of the overlap area.
+    The shifted window keeps exactly (2r-1)^2 image keys for every image query."""
+    if window == "shifted":
+        return H * W * (2 * r - 1) ** 2
     total = 0
     for dy in range(-(r - 1), r):
         w = window_half_width(r, abs(dy), window)

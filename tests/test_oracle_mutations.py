@@ -84,6 +84,17 @@ def _square_is_circle(n_text, H, W, r, rows=None, window="circle"):  # ignores t
     return _orig_mask(n_text, H, W, r, rows, "circle")
 
 
+def _shifted_off_by_one(n_text, H, W, r, rows=None, window="circle"):  # centre clamped one row short
+    if window != "shifted":
+        return _orig_mask(n_text, H, W, r, rows, window)
+    y, x, is_text = oc.token_coords(n_text, H, W)
+    rows = np.arange(y.shape[0]) if rows is None else np.asarray(rows)
+    cy = np.clip(y[rows], r, H - r)[:, None]
+    cx = np.clip(x[rows], r - 1, W - r)[:, None]
+    near = (np.abs(y[None, :] - cy) < r) & (np.abs(x[None, :] - cx) < r)
+    return is_text[rows][:, None] | is_text[None, :] | near
+
+
 def _all_square_pins():
     """Run every square-window pin; return the number that failed."""
     failures = 0
@@ -93,6 +104,9 @@ def _all_square_pins():
         lambda: sq_pins.test_square_kept_pairs_equals_mask_sum(3, 10, 5, 6),
         lambda: sq_pins.test_circle_is_inside_square(1, 9, 9, 4),
         lambda: sq_pins.test_square_full_radius_is_full_attention(4, 6, 9),
+        lambda: sq_pins.test_shifted_mask_matches_window_start_formulation(1, 9, 13, 4),
+        lambda: sq_pins.test_shifted_equals_square_away_from_the_border(),
+        lambda: sq_pins.test_shifted_forward_matches_brute_force(),
     ]
     for c in calls:
         try:
@@ -138,7 +152,7 @@ def test_unmutated_oracle_passes_all_pins():
     assert _all_square_pins() == 0
 
 
-@pytest.mark.parametrize("mutant", [_square_le, _square_is_circle])
+@pytest.mark.parametrize("mutant", [_square_le, _square_is_circle, _shifted_off_by_one])
 def test_square_mutant_is_caught(monkeypatch, mutant):
     _patch_mask(monkeypatch, mutant)
     assert _all_square_pins() >= 1, f"mutant {mutant.__name__} survived every square pin"

@@ -113,3 +113,73 @@ def test_square_backward_finite_differences():
             args_m = [xm if n == name else a for n, a in (("q", q), ("k", k), ("v", v))]
             fd = (loss(*args_p) - loss(*args_m)) / (2 * h)
             assert abs(fd - g[idx]) < 1e-6 * max(1.0, abs(fd)), (name, idx, fd, g[idx])
+
+
+# ------------------------------------------------------------------------------------------------
+# Border-shifted square window (neighborhood-attention style): constant key count per query.
+# ------------------------------------------------------------------------------------------------
+
+def _shifted_keys_by_window_start(yi, xi, H, W, r):
+    """Independent formulation: the window's first row / column is the query's minus (r-1),
+    pushed back inside the grid; the window is 2r-1 wide."""
+    k = 2 * r - 1
+    y0 = min(max(yi - (r - 1), 0), H - k)
+    x0 = min(max(xi - (r - 1), 0), W - k)
+    return [(yj, xj) for yj in range(y0, y0 + k) for xj in range(x0, x0 + k)]
+
+
+@pytest.mark.parametrize("n_text,H,W,r", [(0, 7, 9, 3), (3, 5, 5, 3), (2, 11, 8, 2), (1, 9, 13, 4)])
+def test_shifted_mask_matches_window_start_formulation(n_text, H, W, r):
+    M = oracle.clear_mask(n_text, H, W, r, window="shifted")
+    for i in range(n_text, n_text + H * W):
+        yi, xi = divmod(i - n_text, W)
+        ref = np.zeros(n_text + H * W, dtype=bool)
+        ref[:n_text] = True
+        for yj, xj in _shifted_keys_by_window_start(yi, xi, H, W, r):
+            ref[n_text + yj * W + xj] = True
+        assert (M[i] == ref).all(), (yi, xi)
+        assert M[i, n_text:].sum() == (2 * r - 1) ** 2  # constant count, corners included
+    assert M.sum() == oracle.kept_pairs(n_text, H, W, r, "shifted")
+
+
+def test_shifted_equals_square_away_from_the_border():
+    n_text, H, W, r = 2, 13, 14, 3
+    sh = oracle.clear_mask(n_text, H, W, r, window="shifted")
+    sq = oracle.clear_mask(n_text, H, W, r, window="square")
+    differs = 0
+    for y in range(H):
+        for x in range(W):
+            i = n_text + y * W + x
+            if r - 1 <= y <= H - r and r - 1 <= x <= W - r:
+                assert (sh[i] == sq[i]).all(), (y, x)  # interior: the window is not shifted
+            else:
+                differs += int(not (sh[i] == sq[i]).all())
+    assert differs == H * W - (H - 2 * (r - 1)) * (W - 2 * (r - 1))  # every border query is shifted
+    assert not (sh == sh.T).all()  # border queries see farther keys than those keys see them back
+
+
+def test_shifted_window_as_large_as_the_grid_is_full_attention():
+    n_text, H, W, r = 3, 5, 5, 3  # 2r - 1 = 5: every window is the whole grid
+    T = n_text + H * W
+    q, k, v = (_rand((1, 1, T, 8), s) for s in (70, 71, 72))
+    O, LSE = oracle.clear_attention_forward(q, k, v, n_text, H, W, r, window="shifted")
+    s = q[0, 0] @ k[0, 0].T / math.sqrt(8)
+    lse = logsumexp(s, axis=1)
+    np.testing.assert_allclose(O[0, 0], np.exp(s - lse[:, None]) @ v[0, 0], rtol=0, atol=1e-12)
+
+
+def test_shifted_forward_matches_brute_force():
+    n_text, H, W, r = 2, 6, 7, 2
+    T = n_text + H * W
+    q, k, v = (_rand((1, 1, T, 8), s) for s in (80, 81, 82))
+    O, LSE = oracle.clear_attention_forward(q, k, v, n_text, H, W, r, window="shifted")
+    for i in range(T):
+        if i < n_text:
+            keys = list(range(T))
+        else:
+            yi, xi = divmod(i - n_text, W)
+            keys = list(range(n_text)) + [n_text + yj * W + xj for yj, xj in _shifted_keys_by_window_start(yi, xi, H, W, r)]
+        s = q[0, 0, i] @ k[0, 0, keys].T / math.sqrt(8)
+        lse = logsumexp(s)
+        np.testing.assert_allclose(O[0, 0, i], np.exp(s - lse) @ v[0, 0, keys], rtol=0, atol=1e-12)
+        assert abs(LSE[0, 0, i] - lse) < 1e-12
