@@ -64,12 +64,17 @@ typedef struct {
   int H, W;     /* image token grid, >= 1 each */
   int d;        /* head dim: 64 or 128 */
   int r;        /* window radius in grid units (strict: dx^2 + dy^2 < r^2), >= 1 */
-  int window;   /* CLEAR_WINDOW_CIRCLE (0, CLEAR's mask) or CLEAR_WINDOW_SQUARE (1): keep image pairs
+  int window;   /* CLEAR_WINDOW_CIRCLE (0, CLEAR's mask); CLEAR_WINDOW_SQUARE (1): keep image pairs
                    with |dx| < r and |dy| < r instead, the square sliding window the pages compare
-                   the circle with. Any other value is CLEAR_ERR_INVALID_ARG. */
+                   the circle with; CLEAR_WINDOW_SHIFTED (2): the same square around a centre
+                   clamped to [r-1, H-r] x [r-1, W-r] (neighborhood-attention style: every image
+                   query keeps (2r-1)^2 image keys), which needs H, W >= 2r-1 (else
+                   CLEAR_ERR_INVALID_ARG) and has no backward (CLEAR_ERR_UNSUPPORTED from
+                   clear_attn_bwd and its workspace query). Any other value is
+                   CLEAR_ERR_INVALID_ARG. */
 } clear_attn_params_t;
 
-enum { CLEAR_WINDOW_CIRCLE = 0, CLEAR_WINDOW_SQUARE = 1 };
+enum { CLEAR_WINDOW_CIRCLE = 0, CLEAR_WINDOW_SQUARE = 1, CLEAR_WINDOW_SHIFTED = 2 };
 
 /* Library version (major * 10000 + minor * 100 + patch). */
 CLEAR_API int clear_attn_version(void);

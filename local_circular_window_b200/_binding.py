@@ -32,7 +32,7 @@ class ClearParams(ctypes.Structure):
                 ("W", ctypes.c_int), ("d", ctypes.c_int), ("r", ctypes.c_int), ("window", ctypes.c_int)]
 
 
-WINDOWS = {"circle": 0, "square": 1}  # CLEAR_WINDOW_CIRCLE, CLEAR_WINDOW_SQUARE
+WINDOWS = {"circle": 0, "square": 1, "shifted": 2}  # CLEAR_WINDOW_CIRCLE, _SQUARE, _SHIFTED
 
 
 def _window_code(window) -> int:
@@ -167,7 +167,8 @@ def _check_qkv(name, t, shape):
 def clear_attn_fwd(q, k, v, n_text: int, H: int, W: int, r: int, o=None, lse=None, workspace=None, stream=None,
                    window="circle"):
     """CLEAR attention forward through the C ABI. Returns (o, lse); raises ClearError on failure.
-    window: "circle" (CLEAR's mask) or "square" (|dx| < r and |dy| < r)."""
+    window: "circle" (CLEAR's mask), "square" (|dx| < r and |dy| < r) or "shifted" (that square with
+    its centre clamped inside the grid; forward only)."""
     B, heads, T, d = q.shape
     if T != n_text + H * W:
         raise ValueError("T must equal n_text + H * W")

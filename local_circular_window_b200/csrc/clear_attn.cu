@@ -49,7 +49,9 @@ Checked check_params(const clear_attn_params_t* p) {
   c.st = CLEAR_ERR_INVALID_ARG;
   if (!p) return c;
   if (p->B < 1 || p->heads < 1 || p->n_text < 0 || p->H < 1 || p->W < 1 || p->r < 1) return c;
-  if (p->window != kCircle && p->window != kSquare) return c;
+  if (p->window != kCircle && p->window != kSquare && p->window != kShifted) return c;
+  // The shifted window must fit in the grid: it is never clamped to a smaller radius.
+  if (p->window == kShifted && (2 * (long long)p->r - 1 > p->H || 2 * (long long)p->r - 1 > p->W)) return c;
   if (p->d != 64 && p->d != 128) {
     c.st = CLEAR_ERR_UNSUPPORTED;
     return c;
@@ -59,7 +61,7 @@ Checked check_params(const clear_attn_params_t* p) {
   const long long BH = (long long)p->B * p->heads;
   if (N > (1ll << 28) || p->n_text > (1 << 24) || T > (1ll << 30) || BH > (1ll << 20)) return c;
   if (BH * T * p->d >= (1ll << 40)) return c;
-  const int rfull = full_radius(p->H, p->W, p->window);
+  const int rfull = p->window == kShifted ? p->r : full_radius(p->H, p->W, p->window);
   const int r = p->r < rfull ? p->r : rfull;
   if (hw_table_size(r, p->H) > kMaxHwTable) {  // half-width table must fit in shared memory
     c.st = CLEAR_ERR_UNSUPPORTED;
@@ -289,8 +291,9 @@ size_t clear_attn_fwd_workspace_size(const clear_attn_params_t* params, clear_st
 
 size_t clear_attn_bwd_workspace_size(const clear_attn_params_t* params, clear_status_t* status) {
   const Checked c = check_params(params);
-  if (status) *status = c.st;
-  if (c.st != CLEAR_OK) return 0;
+  const clear_status_t st = (c.st == CLEAR_OK && c.g.window == kShifted) ? CLEAR_ERR_UNSUPPORTED : c.st;
+  if (status) *status = st;
+  if (st != CLEAR_OK) return 0;
   return bwd_workspace_layout(c.g).total;
 }
 
@@ -341,6 +344,8 @@ clear_status_t clear_attn_bwd(const clear_attn_params_t* params, const void* q, 
                               void* stream) {
   const Checked c = check_params(params);
   if (c.st != CLEAR_OK) return c.st;
+  // The shifted window's mask is not symmetric, which the KV-stationary dK/dV kernel relies on.
+  if (c.g.window == kShifted) return CLEAR_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
       !aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return CLEAR_ERR_INVALID_ARG;
@@ -449,9 +454,11 @@ clear_status_t clear_sched_pair_counts(const clear_attn_params_t* params, long l
   const Checked c = check_params(params);
   if (c.st != CLEAR_OK) return c.st;
   const Geom& g = c.g;
-  // Kept pairs: text rows see all T keys, image rows see all text keys plus their clipped window.
+  // Kept pairs: text rows see all T keys, image rows see all text keys plus their window (clipped,
+  // or for the shifted window exactly (2r-1)^2 keys).
   long long win = 0;
-  for (int dy = -(g.r - 1); dy <= g.r - 1; ++dy) {
+  if (g.window == kShifted) win = (long long)g.H * g.W * (2 * g.r - 1) * (2 * g.r - 1);
+  for (int dy = -(g.r - 1); dy <= g.r - 1 && g.window != kShifted; ++dy) {
     const int w = half_width(g.r, dy < 0 ? -dy : dy, g.window);
     if (w < 0) continue;
     const long long rows = g.H - (dy < 0 ? -dy : dy);

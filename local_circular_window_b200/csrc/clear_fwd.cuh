@@ -417,6 +417,7 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
     // Per-pair state, set up at the pair's first tile.
     PairItem it{};
     int yq = 0, xq = 0, tq = 0;
+    int yc = 0, xc = 0;  // the window's centre: (yq, xq), clamped inside the grid for shifted windows
     bool row_valid = false;
     float m_used = -INFINITY;  // running max, scaled log2 units
     float l = 0.f;
@@ -497,6 +498,8 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
           yq = it.q0 + half * kQH + (row >> 4);
           xq = it.x0 + (row & 15);
           row_valid = (yq < g.H) && (xq < g.W);
+          yc = window_center(yq, g.r, g.H, g.window);
+          xc = window_center(xq, g.r, g.W, g.window);
         }
         m_used = -INFINITY;
         l = 0.f;
@@ -528,8 +531,8 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
             #pragma unroll
             for (int q = 0; q < kFKH / 2; ++q) {
               int lo0, hi0, lo1, hi1;
-              row_range_tab(g, hwtab, hwn, yq, xq, t.a + 2 * q, t.b, &lo0, &hi0);
-              row_range_tab(g, hwtab, hwn, yq, xq, t.a + 2 * q + 1, t.b, &lo1, &hi1);
+              row_range_tab(g, hwtab, hwn, yc, xc, t.a + 2 * q, t.b, &lo0, &hi0);
+              row_range_tab(g, hwtab, hwn, yc, xc, t.a + 2 * q + 1, t.b, &lo1, &hi1);
               const int n0 = imax(hi0 - lo0 + 1, 0), n1 = imax(hi1 - lo1 + 1, 0);
               keep[q] = (((1u << n0) - 1u) << (lo0 & 15)) | ((((1u << n1) - 1u) << (lo1 & 15)) << 16);
             }

@@ -57,9 +57,11 @@ struct KeyTile {
   int flags;  // kFull or kNeedsMask
 };
 
-// Window shapes: the circle (CLEAR's mask, dx^2 + dy^2 < r^2) and the square of the same radius
-// (|dx| < r and |dy| < r). Everything downstream sees a window only through half_width and within.
-enum WindowShape : int { kCircle = 0, kSquare = 1 };
+// Window shapes: the circle (CLEAR's mask, dx^2 + dy^2 < r^2), the square of the same radius
+// (|dx| < r and |dy| < r), and the border-shifted square (the same square around a centre clamped
+// to [r-1, n-r] per axis, so every query keeps (2r-1)^2 image keys; forward only). Everything
+// downstream sees a window only through half_width / within, applied to window_center coordinates.
+enum WindowShape : int { kCircle = 0, kSquare = 1, kShifted = 2 };
 
 struct Geom {
   int B, heads, n_text, H, W, d, r;
@@ -98,14 +100,22 @@ CLEAR_HD int isqrt_below(int rem) {
 // when no key at that vertical distance is kept. Circle: largest dx with dx^2 + dy^2 < r^2;
 // square: r - 1 for dy < r.
 CLEAR_HD int half_width(int r, int dy, int window = kCircle) {
-  if (window == kSquare) return dy < r ? r - 1 : -1;
+  if (window != kCircle) return dy < r ? r - 1 : -1;
   int rem = r * r - dy * dy;
   return rem <= 0 ? -1 : isqrt_below(rem);
 }
 
 // Whether the offset (dx, dy), both >= 0, is inside the window.
 CLEAR_HD bool within(int r, int window, int dx, int dy) {
-  return window == kSquare ? (dx < r && dy < r) : (dx * dx + dy * dy < r * r);
+  return window != kCircle ? (dx < r && dy < r) : (dx * dx + dy * dy < r * r);
+}
+
+// The grid coordinate (row or column, axis length n) the window is measured from: the query's own
+// coordinate, or for the shifted window the centre clamped so the window stays inside the grid.
+CLEAR_HD int window_center(int v, int r, int n, int window) {
+  if (window != kShifted) return v;
+  const int lo = r - 1, hi = n - r;
+  return v < lo ? lo : (v > hi ? hi : v);
 }
 
 // Text split count: enough splits that each covers about `target` chunks, capped so the fp32
@@ -353,6 +363,12 @@ struct PairKeyIter {
     xl = imin(x0 + kQW - 1, W - 1);
     yA0 = y0; yAl = imin(y0 + kQH - 1, H - 1);
     yB0 = y0 + kQH; yBl = imin(y0 + 2 * kQH - 1, H - 1);
+    if (window == kShifted) {  // clamping is monotone: a query rectangle maps to a centre rectangle
+      x0 = window_center(x0, r, W, window); xl = window_center(xl, r, W, window);
+      yA0 = window_center(yA0, r, H, window); yAl = window_center(yAl, r, H, window);
+      yB0 = window_center(yB0, r, H, window); yBl = window_center(yBl, r, H, window);
+      y0 = yA0;
+    }
     const int ylast = validB ? yBl : yAl;
     ky_begin = imax(0, y0 - (r - 1));
     ky_end = imin(H - 1, ylast + (r - 1));

@@ -26,7 +26,7 @@ def test_version_and_status_strings():
 
 @pytest.mark.parametrize("fields,expected", [
     (dict(r=0), 1), (dict(B=0), 1), (dict(heads=0), 1), (dict(H=0), 1), (dict(W=-3), 1), (dict(n_text=-1), 1),
-    (dict(d=96), 2), (dict(d=256), 2), (dict(window=2), 1), (dict(window=-1), 1), (dict(H=1 << 15, W=1 << 15), 1), (dict(n_text=1 << 25), 1),
+    (dict(d=96), 2), (dict(d=256), 2), (dict(window=3), 1), (dict(window=-1), 1), (dict(H=1 << 15, W=1 << 15), 1), (dict(n_text=1 << 25), 1),
 ])
 def test_invalid_params_statuses(fields, expected):
     base = dict(B=1, heads=2, n_text=16, H=16, W=16, d=64, r=4)
@@ -83,6 +83,23 @@ def test_backward_argument_errors_launch_nothing():
 @pytest.mark.parametrize("limit_ms", [0, -5, 5001])
 def test_selftest_rejects_bad_limits_before_any_cuda_call(limit_ms):
     assert L.status_string(L.lib().clear_attn_selftest_expiry(limit_ms, None)) == "CLEAR_ERR_INVALID_ARG"
+
+
+def test_shifted_window_limits():
+    # Needs H, W >= 2r - 1 (never clamped) and has no backward.
+    st = ctypes.c_int(0)
+    bad = L.make_params(1, 2, 16, 16, 9, 64, 6, "shifted")   # 2r - 1 = 11 > W = 9
+    assert L.lib().clear_attn_fwd_workspace_size(ctypes.byref(bad), ctypes.byref(st)) == 0
+    assert L.status_string(st.value) == "CLEAR_ERR_INVALID_ARG"
+    ok = L.make_params(1, 2, 16, 16, 11, 64, 6, "shifted")
+    L.lib().clear_attn_fwd_workspace_size(ctypes.byref(ok), ctypes.byref(st))
+    assert st.value == 0
+    assert L.lib().clear_attn_bwd_workspace_size(ctypes.byref(ok), ctypes.byref(st)) == 0
+    assert L.status_string(st.value) == "CLEAR_ERR_UNSUPPORTED"
+    bufs = [_canary() for _ in range(10)]
+    assert L.status_string(L.lib().clear_attn_bwd(ctypes.byref(ok), *(p_ for _, p_ in bufs), ctypes.c_size_t(1 << 20),
+                                                  None)) == "CLEAR_ERR_UNSUPPORTED"
+    assert all((a == 0x5A).all() for a, _ in bufs)
 
 
 def test_workspace_sizes():

@@ -54,9 +54,15 @@ NEED = (1, 2)
 FULL = (4, 8)
 
 
-@pytest.mark.parametrize("window", ["circle", "square"])
+def _skip_unfit(window, H, W, r):
+    if window == "shifted" and (2 * r - 1 > H or 2 * r - 1 > W):
+        pytest.skip("the shifted window needs H, W >= 2r - 1")
+
+
+@pytest.mark.parametrize("window", ["circle", "square", "shifted"])
 @pytest.mark.parametrize("n_text,H,W,r", CASES)
 def test_tiles_cover_mask_exactly(n_text, H, W, r, window):
+    _skip_unfit(window, H, W, r)
     p = L.make_params(1, 1, n_text, H, W, 64, r, window)
     T = n_text + H * W
     n_txt_items, n_img_items, S, cps = L.forward_shape(p)
@@ -95,9 +101,10 @@ def test_tiles_cover_mask_exactly(n_text, H, W, r, window):
         assert sorted(keys) == list(range(T))
 
 
-@pytest.mark.parametrize("window", ["circle", "square"])
+@pytest.mark.parametrize("window", ["circle", "square", "shifted"])
 @pytest.mark.parametrize("n_text,H,W,r", CASES[:6])
 def test_pair_counts(n_text, H, W, r, window):
+    _skip_unfit(window, H, W, r)
     p = L.make_params(2, 3, n_text, H, W, 64, r, window)
     useful, executed = L.pair_counts(p)
     assert useful == 6 * oracle.kept_pairs(n_text, H, W, r, window)

@@ -80,3 +80,53 @@ def test_square_backward_full_oracle(wl):
     assert_close(dq.float().cpu().numpy(), rq, f"square {wl.name} dQ")
     assert_close(dk.float().cpu().numpy(), rk, f"square {wl.name} dK")
     assert_close(dv.float().cpu().numpy(), rv, f"square {wl.name} dV")
+
+
+# ------------------------------------------------------------------------------------------------
+# Border-shifted square window (window="shifted"): forward only.
+# ------------------------------------------------------------------------------------------------
+
+SHIFTED = [
+    Workload("sh_ragged_d128", 2, 3, 77, 24, 40, 128, 5),
+    Workload("sh_no_text", 1, 2, 0, 19, 21, 128, 3),
+    Workload("sh_wide_text_d64", 1, 2, 200, 13, 50, 64, 7),
+    Workload("sh_window_is_grid", 1, 2, 16, 15, 15, 64, 8),  # 2r - 1 = 15: every window is the grid
+    Workload("sh_text300_r16", 1, 2, 300, 32, 32, 128, 16),
+]
+
+
+@pytest.mark.parametrize("wl", SHIFTED, ids=lambda w: w.name)
+def test_shifted_forward_small_full_oracle(wl):
+    q, k, v = gpu_inputs(wl, seed=0)
+    o, lse = L.clear_attn_fwd(q, k, v, wl.n_text, wl.H, wl.W, wl.r, window="shifted")
+    assert L.clear_attn_check() == 0
+    O, LSE = oracle.clear_attention_forward(q.cpu(), k.cpu(), v.cpu(), wl.n_text, wl.H, wl.W, wl.r,
+                                            window="shifted")
+    assert_close(o.float().cpu().numpy(), O, f"shifted {wl.name} O")
+    assert_close(lse.cpu().numpy(), LSE, f"shifted {wl.name} LSE", max_abs=LSE_ABS, mean_abs=LSE_ABS / 10)
+
+
+def test_shifted_flux1024_and_8k_sampled():
+    for name in ("flux1024_r8", "8k_r8"):
+        wl = WORKLOADS[name]
+        q, k, v = make_inputs(wl, seed=0, device="cuda")
+        o, lse = L.clear_attn_fwd(q, k, v, wl.n_text, wl.H, wl.W, wl.r, window="shifted")
+        assert L.clear_attn_check() == 0
+        rows = sample_rows(wl, np.random.default_rng(2), n_interior=64, n_border=48, n_text=16)
+        for h in (0, 23):
+            Or, Lr = oracle.clear_attention_rows(q, k, v, wl.n_text, wl.H, wl.W, wl.r, 0, h, rows, window="shifted")
+            assert_close(o[0, h, rows].float().cpu().numpy(), Or, f"shifted {name} h{h} O")
+            assert_close(lse[0, h, rows].cpu().numpy(), Lr, f"shifted {name} h{h} LSE", max_abs=LSE_ABS,
+                         mean_abs=LSE_ABS)
+        del q, k, v, o, lse
+        torch.cuda.empty_cache()
+
+
+def test_shifted_backward_is_unsupported():
+    wl = SHIFTED[1]
+    q, k, v, dO = gpu_inputs(wl, seed=0, grad=True)
+    o, lse = L.clear_attn_fwd(q, k, v, wl.n_text, wl.H, wl.W, wl.r, window="shifted")
+    with pytest.raises(L.ClearError) as e:
+        L.clear_attn_bwd(q, k, v, o, lse, dO, wl.n_text, wl.H, wl.W, wl.r, window="shifted")
+    assert "CLEAR_ERR_UNSUPPORTED" in str(e.value)
+    assert L.clear_attn_check() == 0
