@@ -47,6 +47,25 @@ def test_noalloc_matches_fwd_on_consecutive_calls(wl):
     torch.cuda.empty_cache()
 
 
+@pytest.mark.gpu
+@pytest.mark.parametrize("window", ["square", "shifted"])
+def test_noalloc_window_variants_match_fwd(window):
+    wl = Workload("ragged", 1, 3, 77, 24, 40, 128, 5)
+    q, k, v = make_inputs(wl, seed=8, device="cuda")
+    ref_o, ref_lse = L.clear_attn_fwd(q, k, v, wl.n_text, wl.H, wl.W, wl.r, window=window)
+    p = L.make_params(wl.B, wl.heads, wl.n_text, wl.H, wl.W, wl.d, wl.r, window)
+    o = torch.full_like(q, float("nan"))
+    lse = torch.full((wl.B, wl.heads, wl.T), float("nan"), dtype=torch.float32, device=q.device)
+    st = L.lib().clear_attn_fwd_noalloc(ctypes.byref(p), ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                                        ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(o.data_ptr()),
+                                        ctypes.c_void_p(lse.data_ptr()),
+                                        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0, L.status_string(st)
+    assert L.clear_attn_check() == 0
+    assert_close(o.float().cpu().numpy(), ref_o.float().cpu().numpy(), f"noalloc {window} O")
+    assert_close(lse.cpu().numpy(), ref_lse.cpu().numpy(), f"noalloc {window} LSE", max_abs=LSE_ABS, mean_abs=LSE_ABS)
+
+
 def test_noalloc_rejects_problems_beyond_its_scratch():
     # One split of 1024 heads x 4096 text rows needs 1024 * 4096 * (4 * 128 + 8) bytes > 32 MiB:
     # rejected on the host before anything is launched (host canaries stay untouched).
