@@ -279,8 +279,10 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
       bool q_seen = false, had = false, end_pending = false, all_posted = false;
       // PV walk: union index Gp; up to two needed tiles whose Q K^T is issued and P V is not.
       uint32_t Gp = 0, npv = 0;
-      uint32_t pend_G[2] = {0, 0};
-      int pend_fl[2] = {0, 0};  // bit 0: first of the pair (overwrite O), bit 1: commit o_done after it
+      // The pending tiles form a two-entry FIFO kept in registers (head h*, tail t*): union index,
+      // and flags (bit 0: first of the pair, overwrite O; bit 1: commit o_done after its P V).
+      uint32_t hG = 0, tG = 0;
+      int hF = 0, tF = 0;
       int pend = 0;
       PollWatchdog wd;
       wd.start();
@@ -290,8 +292,7 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
         // frees the S buffer the next Q K^T needs.
         if (Gp < Gq) {
           const uint32_t vs = Gp % kVStages;
-          const int slot = npv & 1;
-          const bool needed = pend > 0 && pend_G[slot] == Gp;
+          const bool needed = pend > 0 && hG == Gp;
           if (!needed) {
             if (mbar_test(&bars[L::bVFull + vs], (Gp / kVStages) & 1)) {
               mbar_arrive(&bars[L::bVEmpty + vs]);  // observed and released
@@ -300,21 +301,24 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
             }
           } else {
             const uint32_t b = npv & 1;
-            if (mbar_test(&bars[L::bPFull + 2 * h + b], (npv >> 1) & 1) &&
-                mbar_test(&bars[L::bVFull + vs], (Gp / kVStages) & 1)) {
+            const bool pr = mbar_test(&bars[L::bPFull + 2 * h + b], (npv >> 1) & 1);
+            const bool vr = mbar_test(&bars[L::bVFull + vs], (Gp / kVStages) & 1);
+            if (pr && vr) {
               tc_fence_after();
               const uint64_t vd = vdesc0 + (uint64_t)((vs * L::kKVTileBytes) >> 4);
               const uint32_t s_tm = tmem + L::s_col(h, b);
-              const bool first = pend_fl[slot] & 1;
+              const bool first = hF & 1;
               #pragma unroll
               for (int kk = 0; kk < kFChunk / 16; ++kk)
                 umma_ts(o_tm, s_tm + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv,
                         (!first || kk > 0) ? 1u : 0u);
               umma_commit(&bars[L::bVEmpty + vs]);
               umma_commit(&bars[L::bOReady + h]);
-              if (pend_fl[slot] & 2) umma_commit(&bars[L::bODone + h]);
+              if (hF & 2) umma_commit(&bars[L::bODone + h]);
               ++npv;
               --pend;
+              hG = tG;
+              hF = tF;
               ++Gp;
               prog = true;
             }
@@ -340,17 +344,22 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
             }
           } else {
             const uint32_t ks = Gq % kKStages;
-            if (mbar_test(&bars[L::bKFull + ks], (Gq / kKStages) & 1)) {
-              const int4 e = ring[Gq % kTileRing];
+            const uint32_t ms = nmsg & 1;
+            // The K barrier, the ring entry and the mailbox are read back to back so their
+            // latencies overlap; the test's acquire orders the ring read, and the entry is used
+            // only once the test has passed.
+            const bool kr = mbar_test(&bars[L::bKFull + ks], (Gq / kKStages) & 1);
+            const int4 e = ring[Gq % kTileRing];
+            const bool mr = mbar_test(&bars[L::bMsgEmpty + 2 * h + ms], ((nmsg >> 1) & 1) ^ 1);
+            if (kr) {
               const int flags = (e.x >> 4) & 255;
               const bool last_of_pair = (e.x >> 12) & 1;
               const bool needed = (flags & need_bit) != 0;
-              const uint32_t ms = nmsg & 1;
               bool done_tile = false;
               if (!needed) {
                 mbar_arrive(&bars[L::bKEmpty + ks]);  // observed and released
                 done_tile = true;
-              } else if (pend < 2 && mbar_test(&bars[L::bMsgEmpty + 2 * h + ms], ((nmsg >> 1) & 1) ^ 1)) {
+              } else if (pend < 2 && mr) {
                 const uint32_t b = nqk & 1;
                 msg[2 * h + ms] = make_int4(e.x & 15, e.y, e.z, flags | (int)(pair << 8));
                 mbar_arrive(&bars[L::bMsgFull + 2 * h + ms]);
@@ -365,9 +374,13 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
                 }
                 umma_commit(&bars[L::bSFull + 2 * h + b]);
                 umma_commit(&bars[L::bKEmpty + ks]);
-                const int slot = (npv + pend) & 1;
-                pend_G[slot] = Gq;
-                pend_fl[slot] = had ? 0 : 1;
+                if (pend == 0) {
+                  hG = Gq;
+                  hF = had ? 0 : 1;
+                } else {
+                  tG = Gq;
+                  tF = had ? 0 : 1;
+                }
                 ++pend;
                 ++nqk;
                 had = true;
@@ -382,8 +395,10 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
                     umma_commit(&bars[L::bQEmpty]);
                     // o_done follows this half's last P V of the pair: mark it if still pending
                     // (it is the most recent needed tile), else commit now.
-                    if (pend > 0)
-                      pend_fl[(npv + pend - 1) & 1] |= 2;
+                    if (pend == 2)
+                      tF |= 2;
+                    else if (pend == 1)
+                      hF |= 2;
                     else
                       umma_commit(&bars[L::bODone + h]);
                     end_pending = true;
