@@ -22,17 +22,18 @@ Revs Pre-Trained Diffusion Transformers Up"):
    by gradient descent [pith review, "The reading"], so the gradient is the analytic gradient of
    the forward above (standard softmax-attention calculus, written out in `clear_attention_backward`).
 
-5. Square-window variant (a comparison mask, not CLEAR's): the pages contrast the circular window
-   with "the traditional square sliding window" [nav.superapi.store page, "Technical Principles of
+5. Square-window variant (a comparison mask, not CLEAR's): the pages set the circular window
+   against the usual square local window [nav.superapi.store page, "Technical Principles of
    CLEAR"] and give the circle's cost as about pi/4 of a square window's [pith review, "What
    carries the argument"]. Read as the same rule with the Chebyshev distance: image tokens i and j
    are kept iff |dx| < r and |dy| < r (the square circumscribing the disc, same strictness).
    Every function below takes window="circle" (CLEAR, the default) or window="square".
 6. Border-shifted square window (the other comparison mask): the pages name Neighborhood
    Attention as the prior art CLEAR builds on [codewithpapers page, "Builds on"; pith review,
-   desk verdict: "neighborhood attention with a circular window"]. Neighborhood attention keeps
-   a fixed square of (2r-1) x (2r-1) keys per query and, at the grid border, shifts the window
-   inward instead of clipping it, so every query sees the same number of keys. Read here as:
+   desk verdict, which reads CLEAR as neighborhood attention with a disc-shaped window].
+   Neighborhood attention keeps a fixed square of (2r-1) x (2r-1) keys per query and, at the
+   grid border, shifts the window inward instead of clipping it, so every query sees the same
+   number of keys. Read here as:
    image pair (i, j) kept iff |y_j - cy(y_i)| < r and |x_j - cx(x_i)| < r with the centre clamped,
    cy(y) = min(max(y, r-1), H-r) (likewise cx); it needs H, W >= 2r-1. window="shifted".
 
