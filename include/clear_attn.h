@@ -123,6 +123,39 @@ CLEAR_API clear_status_t clear_attn_fwd(const clear_attn_params_t* params, const
 CLEAR_API clear_status_t clear_attn_fwd_noalloc(const clear_attn_params_t* params, const void* q, const void* k,
                                       const void* v, void* o, float* lse, void* stream);
 
+/* Bytes of caller-provided device workspace clear_attn_fwd_host needs: device copies of q, k, v,
+ * o and lse, plus clear_attn_fwd's workspace for one slice group. Returns 0 and sets *status (if
+ * non-NULL) on invalid params. */
+CLEAR_API size_t clear_attn_fwd_host_workspace_size(const clear_attn_params_t* params, clear_status_t* status);
+
+/*
+ * Forward from and to HOST memory, for callers whose tensors live on the host (the paper has no
+ * counterpart; this is the transfer-overlapped form of clear_attn_fwd). The B * heads slices are
+ * split into up to 24 groups of consecutive slices; each group's q, k, v are copied to the
+ * device, its forward runs (one clear_attn_fwd call with B = 1, heads = group size), and its o
+ * and lse are copied back. Copies run on two library-owned non-blocking streams per device
+ * (created on first use, kept until exit), so the input copy of one group, the forward of the
+ * previous one and the return copy of the one before overlap.
+ *   q_host, k_host, v_host in : bf16 [B, heads, T, d] in page-locked host memory
+ *   o_host                 out: bf16 [B, heads, T, d] in page-locked host memory
+ *   lse_host               out: fp32 [B, heads, T] in page-locked host memory
+ *   workspace              device scratch of at least clear_attn_fwd_host_workspace_size() bytes;
+ *                          it receives the device copies, so its contents are undefined on return.
+ *   stream                 the copies start after the work already queued on `stream`, and work
+ *                          queued on `stream` after this call runs after o_host and lse_host are
+ *                          written: synchronise `stream` before reading them on the host.
+ * Results: those of clear_attn_fwd on the same inputs, up to the summation order of the text
+ * rows (their split count follows the group size, not B * heads).
+ * Errors (nothing is launched): CLEAR_ERR_INVALID_ARG for a host pointer that is NULL, not 16-byte
+ * aligned or not page-locked (pageable memory cannot overlap; cudaHostAlloc or cudaHostRegister
+ * it), CLEAR_ERR_WORKSPACE for a missing or short workspace, and the argument errors of
+ * clear_attn_fwd. CLEAR_ERR_CUDA if a copy, event or stream call fails.
+ */
+CLEAR_API clear_status_t clear_attn_fwd_host(const clear_attn_params_t* params, const void* q_host,
+                                             const void* k_host, const void* v_host, void* o_host,
+                                             float* lse_host, void* workspace, size_t workspace_bytes,
+                                             void* stream);
+
 /*
  * Backward of clear_attn_fwd with respect to q, k and v, given the upstream gradient dO and the
  * forward's o and lse (analytic softmax-attention gradient restricted to the mask):

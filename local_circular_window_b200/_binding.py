@@ -61,6 +61,10 @@ _lib.clear_attn_fwd.restype = _i
 _lib.clear_attn_fwd.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 _lib.clear_attn_fwd_noalloc.restype = _i
 _lib.clear_attn_fwd_noalloc.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp]
+_lib.clear_attn_fwd_host_workspace_size.restype = ctypes.c_size_t
+_lib.clear_attn_fwd_host_workspace_size.argtypes = [_P, ctypes.POINTER(_i)]
+_lib.clear_attn_fwd_host.restype = _i
+_lib.clear_attn_fwd_host.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 _lib.clear_attn_bwd.restype = _i
 _lib.clear_attn_bwd.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 _lib.clear_attn_check.restype = _i
@@ -106,6 +110,14 @@ def fwd_workspace_size(p: ClearParams) -> int:
     n = _lib.clear_attn_fwd_workspace_size(ctypes.byref(p), ctypes.byref(st))
     if st.value != CLEAR_OK:
         raise ClearError(st.value, "clear_attn_fwd_workspace_size")
+    return n
+
+
+def fwd_host_workspace_size(p: ClearParams) -> int:
+    st = _i(0)
+    n = _lib.clear_attn_fwd_host_workspace_size(ctypes.byref(p), ctypes.byref(st))
+    if st.value != CLEAR_OK:
+        raise ClearError(st.value, "clear_attn_fwd_host_workspace_size")
     return n
 
 
@@ -190,6 +202,36 @@ def clear_attn_fwd(q, k, v, n_text: int, H: int, W: int, r: int, o=None, lse=Non
     return o, lse
 
 
+def clear_attn_fwd_host(q, k, v, n_text: int, H: int, W: int, r: int, o=None, lse=None, workspace=None,
+                        stream=None, window="circle"):
+    """CLEAR attention forward from pinned host tensors to pinned host tensors through the C ABI
+    (clear_attn_fwd_host: the library copies slice groups in and out on its own streams, overlapped
+    with the forward). q, k, v: contiguous bf16 CPU tensors in pinned memory; o, lse: pinned CPU
+    outputs (allocated pinned if None); workspace: a CUDA uint8 tensor on the current device
+    (allocated if None). The call is asynchronous: synchronise `stream` before reading o and lse.
+    Returns (o, lse); raises ClearError on failure."""
+    B, heads, T, d = q.shape
+    if T != n_text + H * W:
+        raise ValueError("T must equal n_text + H * W")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_host(name, t, q.shape, torch.bfloat16)
+    p = make_params(B, heads, n_text, H, W, d, r, window)
+    if o is None:
+        o = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=True)
+    if lse is None:
+        lse = torch.empty((B, heads, T), dtype=torch.float32, pin_memory=True)
+    _check_host("o", o, q.shape, torch.bfloat16)
+    _check_host("lse", lse, (B, heads, T), torch.float32)
+    ws_bytes = fwd_host_workspace_size(p)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    st = _lib.clear_attn_fwd_host(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    if st != CLEAR_OK:
+        raise ClearError(st, "clear_attn_fwd_host")
+    return o, lse
+
+
 def clear_attn_bwd(q, k, v, o, lse, dO, n_text: int, H: int, W: int, r: int, dq=None, dk=None, dv=None,
                    workspace=None, stream=None, window="circle"):
     """CLEAR attention backward through the C ABI. Returns (dq, dk, dv). window as for the forward."""
@@ -229,3 +271,9 @@ def selftest_expiry(limit_ms: int, stream=None) -> int:
     """Launches the failure-detection self-test (a wait that expires after limit_ms); returns the
     launch status. clear_attn_check() then reports CLEAR_ERR_DEVICE_TIMEOUT."""
     return _lib.clear_attn_selftest_expiry(int(limit_ms), _stream_ptr(stream))
+
+
+def _check_host(name, t, shape, dtype):
+    # Page-locking is checked by the library (CLEAR_ERR_INVALID_ARG if missing).
+    if not (t.device.type == "cpu" and t.dtype == dtype and t.is_contiguous() and tuple(t.shape) == tuple(shape)):
+        raise ValueError(f"{name} must be a contiguous CPU {dtype} tensor of shape {tuple(shape)}")

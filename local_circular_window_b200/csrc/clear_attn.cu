@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <new>
 
 #include "clear_attn.h"
 #include "clear_bwd.cuh"
@@ -23,7 +24,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 namespace {
 
-constexpr int kVersion = 110;  // 0.1.1: window shape in the params
+constexpr int kVersion = 112;  // 0.1.2: forward from host buffers
 
 // ------------------------------------------------------------------------------------------------
 // Validation
@@ -261,6 +262,84 @@ __global__ void clear_selftest_expiry_kernel(unsigned long long limit_ns) {
   __syncthreads();
 }
 
+// ------------------------------------------------------------------------------------------------
+// Forward from host buffers: (batch, head) slices are split into groups; the host-to-device copy of
+// group i+1, the forward of group i and the device-to-host copy of group i-1 run concurrently on
+// two library-owned copy streams and the caller's stream.
+// ------------------------------------------------------------------------------------------------
+constexpr long long kHostMaxGroups = 24;
+
+struct HostPlan {
+  long long slices = 0, group = 0, n_groups = 0;
+  size_t slice_bytes = 0, slice_lse_bytes = 0;  // one slice of q (k, v, o) and of lse
+  size_t lse_group_bytes = 0;                   // one group's lse block on the device (256-aligned)
+  size_t q_off = 0, k_off = 0, v_off = 0, o_off = 0, lse_off = 0, fws_off = 0, fws_bytes = 0, total = 0;
+};
+
+// Params of one group: `n` consecutive slices of the flat [B * heads] axis, as B = 1, heads = n.
+clear_attn_params_t group_params(const clear_attn_params_t* p, long long n) {
+  clear_attn_params_t gp = *p;
+  gp.B = 1;
+  gp.heads = (int)n;
+  return gp;
+}
+
+bool host_plan(const clear_attn_params_t* p, const Geom& g, HostPlan* hp) {
+  hp->slices = g.BH;
+  hp->group = (g.BH + kHostMaxGroups - 1) / kHostMaxGroups;
+  hp->n_groups = (g.BH + hp->group - 1) / hp->group;
+  hp->slice_bytes = (size_t)g.T * g.d * 2;
+  hp->slice_lse_bytes = (size_t)g.T * sizeof(float);
+  const size_t tens = align256(hp->slice_bytes * g.BH);
+  hp->q_off = 0;
+  hp->k_off = tens;
+  hp->v_off = 2 * tens;
+  hp->o_off = 3 * tens;
+  hp->lse_off = 4 * tens;
+  // Each group's lse gets its own aligned block: a slice of lse (T floats) is not a multiple of
+  // 16 bytes in general, and the forward wants an aligned lse pointer.
+  hp->lse_group_bytes = align256(hp->slice_lse_bytes * hp->group);
+  hp->fws_off = hp->lse_off + hp->lse_group_bytes * hp->n_groups;
+  const clear_attn_params_t gp = group_params(p, hp->group);
+  const Checked c = check_params(&gp);
+  if (c.st != CLEAR_OK) return false;
+  hp->fws_bytes = fwd_workspace_layout(c.g).total;  // the largest group's; reused group after group
+  hp->total = hp->fws_off + align256(hp->fws_bytes);
+  return true;
+}
+
+// True iff both ends of [ptr, ptr + bytes) lie in page-locked host memory (cudaHostAlloc'd or
+// cudaHostRegister'ed), which asynchronous copies need to overlap anything.
+bool page_locked(const void* ptr, size_t bytes) {
+  const char* ends[2] = {static_cast<const char*>(ptr), static_cast<const char*>(ptr) + bytes - 1};
+  for (const char* a : ends) {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, a) != cudaSuccess) {
+      cudaGetLastError();  // clear the error state the failed query leaves behind
+      return false;
+    }
+    if (at.type != cudaMemoryTypeHost) return false;
+  }
+  return true;
+}
+
+// Two non-blocking copy streams per device, created on first use and kept for the process.
+clear_status_t copy_streams(cudaStream_t* h2d, cudaStream_t* d2h) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static cudaStream_t streams[kMaxDevices][2] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CLEAR_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return CLEAR_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < 2; ++i)
+    if (!streams[dev][i] && cudaStreamCreateWithFlags(&streams[dev][i], cudaStreamNonBlocking) != cudaSuccess)
+      return CLEAR_ERR_CUDA;
+  *h2d = streams[dev][0];
+  *d2h = streams[dev][1];
+  return CLEAR_OK;
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------------------------------------
@@ -336,6 +415,88 @@ clear_status_t clear_attn_fwd_noalloc(const clear_attn_params_t* params, const v
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return g.d == 128 ? launch_fwd<128>(g, maps, o, lse, scratch, num_sms, s)
                     : launch_fwd<64>(g, maps, o, lse, scratch, num_sms, s);
+}
+
+size_t clear_attn_fwd_host_workspace_size(const clear_attn_params_t* params, clear_status_t* status) {
+  const Checked c = check_params(params);
+  HostPlan hp;
+  clear_status_t st = c.st;
+  if (st == CLEAR_OK && !host_plan(params, c.g, &hp)) st = CLEAR_ERR_INVALID_ARG;
+  if (status) *status = st;
+  return st == CLEAR_OK ? hp.total : 0;
+}
+
+clear_status_t clear_attn_fwd_host(const clear_attn_params_t* params, const void* q_host, const void* k_host,
+                                   const void* v_host, void* o_host, float* lse_host, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  const Checked c = check_params(params);
+  if (c.st != CLEAR_OK) return c.st;
+  if (!aligned16(q_host) || !aligned16(k_host) || !aligned16(v_host) || !aligned16(o_host) ||
+      !aligned16(lse_host))
+    return CLEAR_ERR_INVALID_ARG;
+  HostPlan hp;
+  if (!host_plan(params, c.g, &hp)) return CLEAR_ERR_INVALID_ARG;
+  if (workspace_bytes < hp.total || !aligned16(workspace)) return CLEAR_ERR_WORKSPACE;
+  int num_sms = 0;
+  clear_status_t st = check_device(&num_sms);
+  if (st != CLEAR_OK) return st;
+  const size_t tens = hp.slice_bytes * hp.slices, lse_bytes = hp.slice_lse_bytes * hp.slices;
+  if (!page_locked(q_host, tens) || !page_locked(k_host, tens) || !page_locked(v_host, tens) ||
+      !page_locked(o_host, tens) || !page_locked(lse_host, lse_bytes))
+    return CLEAR_ERR_INVALID_ARG;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  st = copy_streams(&h2d, &d2h);
+  if (st != CLEAR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+
+  // Events: [0] entry on the caller's stream, [1] all returns copied, then per group "inputs in"
+  // and "outputs ready".
+  const long long n_ev = 2 + 2 * hp.n_groups;
+  cudaEvent_t* ev = new (std::nothrow) cudaEvent_t[n_ev];
+  if (!ev) return CLEAR_ERR_CUDA;
+  long long made = 0;
+  for (; made < n_ev; ++made)
+    if (cudaEventCreateWithFlags(&ev[made], cudaEventDisableTiming) != cudaSuccess) break;
+  bool ok = made == n_ev;
+  auto cu = [&ok](cudaError_t e) { if (e != cudaSuccess) ok = false; return ok; };
+  // Copies start after the work already queued on the caller's stream (an earlier call may still
+  // read the device buffers this one overwrites).
+  if (ok && cu(cudaEventRecord(ev[0], s)) && cu(cudaStreamWaitEvent(h2d, ev[0], 0)))
+    cu(cudaStreamWaitEvent(d2h, ev[0], 0));
+  for (long long gi = 0; ok && gi < hp.n_groups; ++gi) {
+    const long long s0 = gi * hp.group;
+    const long long n = (hp.slices - s0 < hp.group) ? hp.slices - s0 : hp.group;
+    const size_t off = hp.slice_bytes * s0, bytes = hp.slice_bytes * n;
+    const size_t loff = hp.slice_lse_bytes * s0, lbytes = hp.slice_lse_bytes * n;
+    cudaEvent_t in = ev[2 + 2 * gi], out = ev[3 + 2 * gi];
+    char *dq = ws + hp.q_off + off, *dk = ws + hp.k_off + off, *dv = ws + hp.v_off + off;
+    char *dout = ws + hp.o_off + off, *dlse = ws + hp.lse_off + hp.lse_group_bytes * gi;
+    const cudaMemcpyKind up = cudaMemcpyHostToDevice, down = cudaMemcpyDeviceToHost;
+    if (!(cu(cudaMemcpyAsync(dq, static_cast<const char*>(q_host) + off, bytes, up, h2d)) &&
+          cu(cudaMemcpyAsync(dk, static_cast<const char*>(k_host) + off, bytes, up, h2d)) &&
+          cu(cudaMemcpyAsync(dv, static_cast<const char*>(v_host) + off, bytes, up, h2d)) &&
+          cu(cudaEventRecord(in, h2d)) && cu(cudaStreamWaitEvent(s, in, 0))))
+      break;
+    const clear_attn_params_t gp = group_params(params, n);
+    st = clear_attn_fwd(&gp, dq, dk, dv, dout, reinterpret_cast<float*>(dlse), ws + hp.fws_off, hp.fws_bytes, stream);
+    if (st != CLEAR_OK) {
+      ok = false;
+      break;
+    }
+    if (!(cu(cudaEventRecord(out, s)) && cu(cudaStreamWaitEvent(d2h, out, 0)) &&
+          cu(cudaMemcpyAsync(static_cast<char*>(o_host) + off, dout, bytes, down, d2h)) &&
+          cu(cudaMemcpyAsync(reinterpret_cast<char*>(lse_host) + loff, dlse, lbytes, down, d2h))))
+      break;
+  }
+  // Work queued on the caller's stream from here on runs after every return copy.
+  if (made == n_ev) {
+    if (cudaEventRecord(ev[1], d2h) != cudaSuccess || cudaStreamWaitEvent(s, ev[1], 0) != cudaSuccess) ok = false;
+  }
+  for (long long i = 0; i < made; ++i) cudaEventDestroy(ev[i]);  // released once their work completes
+  delete[] ev;
+  if (st != CLEAR_OK) return st;
+  return ok ? CLEAR_OK : CLEAR_ERR_CUDA;
 }
 
 clear_status_t clear_attn_bwd(const clear_attn_params_t* params, const void* q, const void* k,

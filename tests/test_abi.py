@@ -80,6 +80,44 @@ def test_backward_argument_errors_launch_nothing():
         assert (a == 0x5A).all()
 
 
+def test_host_forward_argument_errors_launch_nothing():
+    # Every argument error is caught before any CUDA call (this runs without a GPU).
+    p = L.make_params(2, 3, 16, 16, 16, 64, 4)
+    bufs = [_canary() for _ in range(6)]
+    q, k, v, o, lse, ws = (b[1] for b in bufs)
+    wsz = L.fwd_host_workspace_size(p)
+    f = L.lib().clear_attn_fwd_host
+    assert f(ctypes.byref(p), None, k, v, o, lse, ws, wsz, None) == 1
+    assert f(ctypes.byref(p), q, k, v, o, None, ws, wsz, None) == 1
+    assert f(ctypes.byref(p), q, ctypes.c_void_p(k.value + 4), v, o, lse, ws, wsz, None) == 1
+    assert f(ctypes.byref(p), q, k, v, o, lse, ws, wsz - 1, None) == 3
+    assert f(ctypes.byref(p), q, k, v, o, lse, None, wsz, None) == 3
+    bad = L.make_params(2, 3, 16, 16, 16, 96, 4)
+    assert f(ctypes.byref(bad), q, k, v, o, lse, ws, wsz, None) == 2
+    for a, _ in bufs:
+        assert (a == 0x5A).all()
+
+
+def _a256(n):
+    return (n + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("B,heads,group", [(1, 24, 1), (2, 24, 2), (1, 5, 1), (3, 17, 3)])
+def test_host_workspace_size(B, heads, group):
+    # Device copies of q, k, v, o (bf16), one aligned lse block (fp32) per group, then the forward
+    # workspace of one group of `group` slices (at most 24 groups of consecutive slices).
+    T, d = 512 + 64 * 64, 128
+    p = L.make_params(B, heads, 512, 64, 64, d, 8)
+    tens = _a256(B * heads * T * d * 2)
+    n_groups = -(-B * heads // group)
+    fws = L.fwd_workspace_size(L.make_params(1, group, 512, 64, 64, d, 8))
+    assert L.fwd_host_workspace_size(p) == 4 * tens + n_groups * _a256(group * T * 4) + fws
+    st = ctypes.c_int(0)
+    assert L.lib().clear_attn_fwd_host_workspace_size(ctypes.byref(L.make_params(1, 2, 16, 16, 16, 64, 0)),
+                                                      ctypes.byref(st)) == 0
+    assert L.status_string(st.value) == "CLEAR_ERR_INVALID_ARG"
+
+
 @pytest.mark.parametrize("limit_ms", [0, -5, 5001])
 def test_selftest_rejects_bad_limits_before_any_cuda_call(limit_ms):
     assert L.status_string(L.lib().clear_attn_selftest_expiry(limit_ms, None)) == "CLEAR_ERR_INVALID_ARG"
