@@ -183,6 +183,8 @@ clear_status_t launch_fwd(const Geom& g, const QKVMaps& m, void* o, float* lse, 
   p.lse = lse;
   const FwdWorkspace wl = fwd_workspace_layout(g);
   p.opart = g.n_text ? reinterpret_cast<float*>(static_cast<char*>(ws) + wl.opart_off) : nullptr;
+  p.wide_o = (reinterpret_cast<uintptr_t>(o) & 31u) == 0;
+  p.wide_part = (reinterpret_cast<uintptr_t>(p.opart) & 31u) == 0;
   p.ml = g.n_text ? reinterpret_cast<float2*>(static_cast<char*>(ws) + wl.ml_off) : nullptr;
   p.n_work = g.n_txt_pairs + g.n_img_pairs;
   if (cudaFuncSetAttribute(clear_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,

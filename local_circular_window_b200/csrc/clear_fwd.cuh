@@ -62,7 +62,44 @@ struct FwdParams {
   float* opart;               // [fS, BH, n_text, d] unnormalised partial O of text rows
   float2* ml;                 // [fS, BH, n_text] (running max in scaled log2 units, sum)
   long long n_work;           // pair items
+  int wide_o, wide_part;      // o / opart are 32-byte aligned: the epilogue may store 32 bytes at once
 };
+
+// Packed fp32 pairs (one 64-bit register, low word first): fma.rn.f32x2 / add.rn.f32x2 do two
+// correctly rounded fp32 operations per instruction, with the same results as two fmaf / fadd.
+__device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float f32x2_lo(uint64_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return lo;
+}
+__device__ __forceinline__ float f32x2_hi(uint64_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return hi;
+}
+__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// One 32-byte global store (the address must be 32-byte aligned).
+__device__ __forceinline__ void st_global_v8(void* ptr, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t a4, uint32_t a5, uint32_t a6, uint32_t a7) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(ptr), "r"(a0), "r"(a1), "r"(a2),
+               "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7)
+               : "memory");
+}
 
 template <int D>
 struct FwdLayout {
@@ -456,17 +493,30 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
         if (it.is_text) {
           const size_t prow = ((size_t)it.split * g.BH + it.bh) * g.n_text + (row_valid ? tq : 0);
           float* dst = p.opart + prow * D;
+          // Two TMEM loads per wait; each row's 512-byte run is written 32 (or 16) bytes at a time.
           #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t ov[32];
-            tmem_ld32(o_tm + c * 32, ov);
+          for (int c = 0; c < D / 32; c += 2) {
+            uint32_t ov[2][32];
+            tmem_ld32(o_tm + c * 32, ov[0]);
+            tmem_ld32(o_tm + c * 32 + 32, ov[1]);
             tmem_wait_ld();
             if (row_valid) {
-              float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
               #pragma unroll
-              for (int e = 0; e < 8; ++e)
-                d4[e] = make_float4(__uint_as_float(ov[4 * e]), __uint_as_float(ov[4 * e + 1]),
-                                    __uint_as_float(ov[4 * e + 2]), __uint_as_float(ov[4 * e + 3]));
+              for (int u = 0; u < 2; ++u) {
+                float* d = dst + (c + u) * 32;
+                if (p.wide_part) {
+                  #pragma unroll
+                  for (int e = 0; e < 4; ++e)
+                    st_global_v8(d + e * 8, ov[u][8 * e], ov[u][8 * e + 1], ov[u][8 * e + 2], ov[u][8 * e + 3],
+                                 ov[u][8 * e + 4], ov[u][8 * e + 5], ov[u][8 * e + 6], ov[u][8 * e + 7]);
+                } else {
+                  float4* d4 = reinterpret_cast<float4*>(d);
+                  #pragma unroll
+                  for (int e = 0; e < 8; ++e)
+                    d4[e] = make_float4(__uint_as_float(ov[u][4 * e]), __uint_as_float(ov[u][4 * e + 1]),
+                                        __uint_as_float(ov[u][4 * e + 2]), __uint_as_float(ov[u][4 * e + 3]));
+                }
+              }
             }
           }
           if (row_valid) p.ml[prow] = make_float2(m_used, l);
@@ -475,19 +525,28 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
           const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
           __nv_bfloat16* dst = p.o + orow * D;
           #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t ov[32];
-            tmem_ld32(o_tm + c * 32, ov);
+          for (int c = 0; c < D / 32; c += 2) {
+            uint32_t ov[2][32];
+            tmem_ld32(o_tm + c * 32, ov[0]);
+            tmem_ld32(o_tm + c * 32 + 32, ov[1]);
             tmem_wait_ld();
             if (row_valid) {
-              uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
               #pragma unroll
-              for (int e = 0; e < 4; ++e)
-                d4[e] = make_uint4(
-                    pack_bf16x2(__uint_as_float(ov[8 * e + 0]) * inv_l, __uint_as_float(ov[8 * e + 1]) * inv_l),
-                    pack_bf16x2(__uint_as_float(ov[8 * e + 2]) * inv_l, __uint_as_float(ov[8 * e + 3]) * inv_l),
-                    pack_bf16x2(__uint_as_float(ov[8 * e + 4]) * inv_l, __uint_as_float(ov[8 * e + 5]) * inv_l),
-                    pack_bf16x2(__uint_as_float(ov[8 * e + 6]) * inv_l, __uint_as_float(ov[8 * e + 7]) * inv_l));
+              for (int u = 0; u < 2; ++u) {
+                uint32_t w[16];
+                #pragma unroll
+                for (int i = 0; i < 16; ++i)
+                  w[i] = pack_bf16x2(__uint_as_float(ov[u][2 * i]) * inv_l, __uint_as_float(ov[u][2 * i + 1]) * inv_l);
+                __nv_bfloat16* d = dst + (c + u) * 32;
+                if (p.wide_o) {
+                  st_global_v8(d, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+                  st_global_v8(d + 16, w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]);
+                } else {
+                  uint4* d4 = reinterpret_cast<uint4*>(d);
+                  #pragma unroll
+                  for (int e = 0; e < 4; ++e) d4[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+                }
+              }
             }
           }
           if (row_valid) p.lse[orow] = (m_used + __log2f(l)) * 0.69314718055994530942f;
@@ -596,18 +655,20 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
         }
         // ---- P = 2^(s * scale_log2 - m), row sum, bf16 pairs written over S in TMEM
         const float base = (m_used == -INFINITY) ? 0.f : m_used;
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const uint64_t sl2x2 = f32x2_pack(sl2, sl2), nbase2 = f32x2_pack(-base, -base);
+        uint64_t acc2[4] = {0, 0, 0, 0};
         uint32_t pw[32];
         #pragma unroll
         for (int q = 0; q < 32; ++q) {
-          const float e0 = ex2_approx(fmaf(s[2 * q], sl2, -base));
-          const float e1 = ex2_approx(fmaf(s[2 * q + 1], sl2, -base));
-          acc[(2 * q) & 7] += e0;
-          acc[(2 * q + 1) & 7] += e1;
+          const uint64_t x = f32x2_fma(f32x2_pack(s[2 * q], s[2 * q + 1]), sl2x2, nbase2);
+          const float e0 = ex2_approx(f32x2_lo(x));
+          const float e1 = ex2_approx(f32x2_hi(x));
+          acc2[q & 3] = f32x2_add(acc2[q & 3], f32x2_pack(e0, e1));
           pw[q] = pack_bf16x2(e0, e1);
         }
         tmem_st32(s_tm, pw);
-        l += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+        l += ((f32x2_lo(acc2[0]) + f32x2_hi(acc2[0])) + (f32x2_lo(acc2[1]) + f32x2_hi(acc2[1]))) +
+             ((f32x2_lo(acc2[2]) + f32x2_hi(acc2[2])) + (f32x2_lo(acc2[3]) + f32x2_hi(acc2[3])));
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars[L::bPFull + 2 * half + b]);

@@ -116,3 +116,22 @@ def test_nonzero_stream_and_outputs_in_place():
     assert L.clear_attn_check(s) == 0
     O, _ = oracle.clear_attention_forward(q.cpu(), k.cpu(), v.cpu(), wl.n_text, wl.H, wl.W, wl.r)
     assert_close(o.float().cpu().numpy(), O, "stream O")
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_outputs_only_16_byte_aligned(d):
+    # The ABI promises 16-byte alignment only; the epilogue's 32-byte stores are used only when o
+    # (and the workspace holding the text partials) are 32-byte aligned. Offsetting both by 16 bytes
+    # takes the narrow-store path, which must give the same bits.
+    wl = Workload("ragged_d", 1, 3, 77, 24, 40, d, 5)
+    q, k, v = gpu_inputs(wl, seed=9)
+    p = L.make_params(wl.B, wl.heads, wl.n_text, wl.H, wl.W, wl.d, wl.r)
+    wsz = L.fwd_workspace_size(p)
+    ref_o, ref_lse = L.clear_attn_fwd(q, k, v, wl.n_text, wl.H, wl.W, wl.r)
+    o_buf = torch.full((q.numel() + 8,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    o = o_buf[8:].view(q.shape)
+    ws = torch.empty(wsz + 16, dtype=torch.uint8, device="cuda")[16:]
+    assert o.data_ptr() % 32 == 16 and ws.data_ptr() % 32 == 16
+    o2, lse2 = L.clear_attn_fwd(q, k, v, wl.n_text, wl.H, wl.W, wl.r, o=o, workspace=ws)
+    assert L.clear_attn_check() == 0
+    assert torch.equal(o2, ref_o) and torch.equal(lse2, ref_lse)
