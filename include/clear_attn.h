@@ -29,7 +29,9 @@
  * the host before anything is launched: the call returns the error status and leaves every output
  * untouched. A kernel whose internal bounded wait expired records a device error word instead of
  * hanging; clear_attn_check() synchronises the stream and reports it as CLEAR_ERR_DEVICE_TIMEOUT.
- * Calls are thread-safe (no mutable global state besides the device error word).
+ * Calls are thread-safe: the only mutable global state is the device error word, the
+ * allocation-free forward's scratch array and the host-buffer forward's per-device copy streams
+ * (created once, under a lock).
  */
 #ifndef CLEAR_ATTN_H_
 #define CLEAR_ATTN_H_
