@@ -146,8 +146,8 @@ CLEAR_API size_t clear_attn_fwd_host_workspace_size(const clear_attn_params_t* p
  *   stream                 the copies start after the work already queued on `stream`, and work
  *                          queued on `stream` after this call runs after o_host and lse_host are
  *                          written: synchronise `stream` before reading them on the host.
- * Results: those of clear_attn_fwd on the same inputs, up to the summation order of the text
- * rows (their split count follows the group size, not B * heads).
+ * Results: those of clear_attn_fwd on the same inputs. Slices are independent and each group runs
+ * the same kernels with the same text split count (it depends only on T).
  * Errors (nothing is launched): CLEAR_ERR_INVALID_ARG for a host pointer that is NULL, not 16-byte
  * aligned or not page-locked (pageable memory cannot overlap; cudaHostAlloc or cudaHostRegister
  * it), CLEAR_ERR_WORKSPACE for a missing or short workspace, and the argument errors of

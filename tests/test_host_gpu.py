@@ -2,10 +2,9 @@
 
 The library copies groups of (batch, head) slices from page-locked host memory to the device, runs
 the forward on each group and copies o and lse back, on its own copy streams. Each group is an
-ordinary forward call, so the image rows must come out bit-identical to one clear_attn_fwd call
-over all slices; the text rows may differ in the last bits (their split count, hence summation
-order, follows the group size) and are held to the usual bf16 tolerance. The oracle checks the
-small case directly.
+ordinary forward call over independent slices, so the image rows must come out bit-identical to
+one clear_attn_fwd call over all slices; the text rows (split partials merged by a second kernel)
+are held to the usual bf16 tolerance. The oracle checks the small case directly.
 """
 import pytest
 import torch
