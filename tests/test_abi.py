@@ -5,6 +5,7 @@ import ctypes
 
 import numpy as np
 import pytest
+import torch
 
 import local_circular_window_b200 as L
 from local_circular_window_b200 import _binding as Bd
@@ -167,3 +168,19 @@ def test_no_fallback_without_library(monkeypatch, tmp_path):
     spec = importlib.util.spec_from_file_location("binding_copy", mod_path)
     with pytest.raises(ImportError):
         spec.loader.exec_module(importlib.util.module_from_spec(spec))
+
+
+def test_host_forward_binding_checks_tensors():
+    # The binding checks device, dtype, layout and shape before calling the library.
+    B, heads, n_text, H, W, d = 1, 2, 16, 8, 8, 64
+    T = n_text + H * W
+    ok = torch.zeros((B, heads, T, d), dtype=torch.bfloat16)
+    lse = torch.zeros((B, heads, T))
+    bad_inputs = (torch.zeros((B, heads, T, d), dtype=torch.float32),                # dtype
+                  torch.zeros((B, heads, d, T), dtype=torch.bfloat16).transpose(2, 3),  # layout
+                  torch.zeros((B, heads, T + 1, d), dtype=torch.bfloat16))             # shape
+    for bad in bad_inputs:
+        with pytest.raises(ValueError):
+            L.clear_attn_fwd_host(ok, bad, ok, n_text, H, W, 2, o=ok.clone(), lse=lse)
+    with pytest.raises(ValueError):  # lse of the wrong dtype
+        L.clear_attn_fwd_host(ok, ok, ok, n_text, H, W, 2, o=ok.clone(), lse=lse.double())
