@@ -240,6 +240,51 @@ def _time_calls(fn, steps, stream):
     return per, evs[0].elapsed_time(evs[-1])
 
 
+# Forward configurations reported beside the headline one (FLUX-shaped calls at 1024^2, 2048^2 and
+# 8192^2 pixels, every radius the workload list names).
+FORWARD_CONFIGS = ("flux1024_r8", "flux1024_r16", "flux1024_r32", "flux2048_r16", "8k_r8", "8k_r32")
+L2_BYTES = 126 << 20
+
+
+def time_forward_config(L, wl: Workload, peak: float, stream, seed: int, calls: int = 0):
+    """Median CUDA-event time of clear_attn_fwd on one configuration, with useful and padded
+    (tile-executed) TFLOP/s and the fraction of the bf16 peak."""
+    useful, executed = _flops(L, wl)
+    q, k, v = make_inputs(wl, seed=seed, device="cuda")
+    o = torch.empty_like(q)
+    lse = torch.empty((wl.B, wl.heads, wl.T), dtype=torch.float32, device="cuda")
+    p = L.make_params(wl.B, wl.heads, wl.n_text, wl.H, wl.W, wl.d, wl.r)
+    ws = torch.empty(max(16, L.fwd_workspace_size(p)), dtype=torch.uint8, device="cuda")
+    small = 3 * q_bytes(wl) < 2 * L2_BYTES
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if small else None
+    calls = calls or (10 if wl.H >= 512 else 20)
+
+    def call():
+        L.clear_attn_fwd(q, k, v, wl.n_text, wl.H, wl.W, wl.r, o=o, lse=lse, workspace=ws, stream=stream)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    per = []
+    for _ in range(calls):
+        if flush is not None:
+            flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        call()
+        b.record(stream)
+        torch.cuda.synchronize()
+        per.append(a.elapsed_time(b))
+    if L.clear_attn_check() != 0:
+        raise RuntimeError(f"device error timing {wl.name}")
+    ms = statistics.median(per)
+    del q, k, v, o, lse, ws, flush
+    return {"ms_per_call": ms, "useful_tflops": useful / (ms * 1e-3) / 1e12,
+            "padded_tflops": executed / (ms * 1e-3) / 1e12, "frac_of_peak": useful / (ms * 1e-3) / 1e12 / peak,
+            "useful_gflop_per_call": useful / 1e9, "executed_gflop_per_call": executed / 1e9, "calls": calls,
+            "l2": "flushed between calls" if small else "inputs larger than L2"}
+
+
 def run_clear(args):
     world, rank, local = _dist()
     torch.cuda.set_device(local)
@@ -341,6 +386,17 @@ def run_clear(args):
                "l2": "flushed between calls (256 MiB write, its time subtracted)"}
         del bq, bk, bv, bdo, bo, blse, bws, gq, gk, gv, flush
 
+    # Every other forward configuration of the workload list, timed the same way (CUDA events on the
+    # launching stream; L2 flushed between calls when the inputs fit in L2).
+    configs = None
+    if not args.no_configs:
+        configs = {}
+        for name in FORWARD_CONFIGS:
+            if name == wl.name:
+                continue
+            configs[name] = time_forward_config(L, WORKLOADS[name], peak, stream, seed=3000 + rank)
+        torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         sec, cores, sample = oracle_call_seconds(wl, args.cpu_budget)
@@ -364,7 +420,7 @@ def run_clear(args):
                          "frac": achieved / peak, "traffic": _fwd_traffic(wl),
                          "peak_source": f"{peak_kind} bf16 dense (burst; kernel timed alone)",
                          "kernel": "clear_fwd_kernel + clear_fwd_combine_kernel (one call, CUDA events)"},
-            "e2e": e2e, "cpu_baseline": cpu, "bwd": bwd, "clocks": clocks,
+            "e2e": e2e, "cpu_baseline": cpu, "bwd": bwd, "configs": configs, "clocks": clocks,
             "gpu_launches": 2 * args.steps,
         }
         print(json.dumps(line), flush=True)
@@ -389,6 +445,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other forward configurations")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU work for cpu_baseline")
     args = ap.parse_args()
     if args.warmup < 3:

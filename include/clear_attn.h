@@ -117,7 +117,10 @@ CLEAR_API clear_status_t clear_attn_fwd(const clear_attn_params_t* params, const
  *     of B * heads * n_text rows (4 * d + 8 bytes each) does not fit, the call returns
  *     CLEAR_ERR_WORKSPACE and launches nothing.
  *   - The first call on a device looks up the scratch array's device address (with that device
- *     current); make that first call before any stream capture.
+ *     current); make that first call before any stream capture, and before reserving the rest
+ *     of device memory: the lookup can load the library's device code, which holds the array.
+ *     A failed lookup returns CLEAR_ERR_CUDA, is not remembered (the next call tries again) and
+ *     leaves no pending CUDA error behind.
  *   - All calls share the one array and it keeps the last call's contents. Nothing in it needs to
  *     start at zero: every value a call reads there is written earlier in the same call. Calls
  *     that overlap on the GPU (different streams, or different host threads) race on it.

@@ -204,23 +204,28 @@ clear_status_t launch_fwd(const Geom& g, const QKVMaps& m, void* o, float* lse, 
 }
 
 // Device address of g_noalloc_scratch on the current device. The symbol's name is only a host-side
-// stand-in; the address is looked up once per device, with that device current.
-struct NoAllocSlot {
-  std::once_flag once;
-  void* ptr = nullptr;
-  cudaError_t err = cudaSuccess;
-};
+// stand-in; the address is looked up with that device current and kept once the lookup succeeded.
+// A failed lookup (e.g. the module could not be loaded because device memory was exhausted, or a
+// capture was in progress) is not cached: the next call tries again. The error the failed call
+// left behind is cleared so that it is not reported by an unrelated later call.
 constexpr int kMaxDevices = 64;
-NoAllocSlot g_noalloc_slots[kMaxDevices];
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
 
 clear_status_t noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return CLEAR_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return CLEAR_ERR_UNSUPPORTED;
-  NoAllocSlot& slot = g_noalloc_slots[dev];
-  std::call_once(slot.once, [&slot] { slot.err = cudaGetSymbolAddress(&slot.ptr, g_noalloc_scratch); });
-  if (slot.err != cudaSuccess || slot.ptr == nullptr) return CLEAR_ERR_CUDA;
-  *out = slot.ptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
+      cudaGetLastError();
+      return CLEAR_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
   return CLEAR_OK;
 }
 
@@ -230,7 +235,7 @@ clear_status_t noalloc_geom(Geom* g) {
   if (g->n_text == 0) return CLEAR_OK;
   for (int cap = g->fS; cap >= 1; --cap) {
     Geom t = *g;
-    choose_splits(t.fnC, 2 * kSplitTargetChunks, cap, &t.fS, &t.fcps);
+    choose_splits(t.fnC, kFSplitTargetChunks, cap, &t.fS, &t.fcps);
     t.n_txt_pairs = (long long)t.BH * t.nTq2 * t.fS;
     if (fwd_workspace_layout(t).total <= kNoAllocScratchBytes) {
       *g = t;

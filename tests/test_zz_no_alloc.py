@@ -15,8 +15,9 @@ import pytest
 import torch
 
 import local_circular_window_b200 as L
+import oracle
 from clear_inputs import WORKLOADS, Workload, make_inputs
-from gpu_util import LSE_ABS, assert_close
+from gpu_util import LSE_ABS, assert_close, gpu_inputs
 
 
 def _noalloc(wl, q, k, v):
@@ -45,6 +46,25 @@ def test_noalloc_matches_fwd_on_consecutive_calls(wl):
         assert_close(lse.cpu().numpy(), ref_lse.cpu().numpy(), f"{wl.name} LSE", max_abs=LSE_ABS, mean_abs=LSE_ABS)
     del q, k, v
     torch.cuda.empty_cache()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("wl", [Workload("no_text", 1, 2, 0, 16, 24, 128, 4), Workload("d64", 1, 2, 20, 16, 24, 64, 4)],
+                         ids=lambda w: w.name)
+def test_noalloc_no_text_and_d64(wl):
+    # Without text tokens the call needs no scratch at all; with d = 64 it runs the other kernel
+    # instantiation. Both must equal clear_attn_fwd on two calls in a row, and the oracle.
+    q, k, v = gpu_inputs(wl, seed=11)
+    ref_o, ref_lse = L.clear_attn_fwd(q, k, v, wl.n_text, wl.H, wl.W, wl.r)
+    assert L.clear_attn_check() == 0
+    O, LSE = oracle.clear_attention_forward(q.cpu(), k.cpu(), v.cpu(), wl.n_text, wl.H, wl.W, wl.r)
+    for _ in range(2):
+        o, lse = _noalloc(wl, q, k, v)
+        assert_close(o.float().cpu().numpy(), ref_o.float().cpu().numpy(), f"{wl.name} O vs fwd")
+        assert_close(lse.cpu().numpy(), ref_lse.cpu().numpy(), f"{wl.name} LSE vs fwd", max_abs=LSE_ABS,
+                     mean_abs=LSE_ABS)
+        assert_close(o.float().cpu().numpy(), O, f"{wl.name} O vs oracle")
+        assert_close(lse.cpu().numpy(), LSE, f"{wl.name} LSE vs oracle", max_abs=LSE_ABS, mean_abs=LSE_ABS / 10)
 
 
 @pytest.mark.gpu
