@@ -178,9 +178,8 @@ struct FwdLayout {
   static __host__ __device__ constexpr uint32_t o_col(int half) { return half * 256 + 128; }
 };
 
-// Tiles of a pair each half needs (the producer's last-needed bits). Not inlined: the producer
-// runs it once per pair, and a second tile iterator inline would crowd its small register budget.
-__device__ __noinline__ void pair_need_counts(const Geom& g, const PairItem& it, const int* wtab, int wtn, int* na,
+// Tiles of a pair each half needs (the producer's last-needed bits).
+__device__ __forceinline__ void pair_need_counts(const Geom& g, const PairItem& it, const int* wtab, int wtn, int* na,
                                               int* nb) {
   int nu;
   count_pair_tiles(g, it, wtab, wtn, &nu, na, nb);
@@ -191,7 +190,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_constant__ CUtensorMap tm_q_img,
                  const __grid_constant__ CUtensorMap tm_k_lin, const __grid_constant__ CUtensorMap tm_k_img,
                  const __grid_constant__ CUtensorMap tm_v_lin, const __grid_constant__ CUtensorMap tm_v_img,
-                 const __grid_constant__ FwdParams p) {
+                 const FwdParams p) {
   using L = FwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -646,11 +645,10 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
         // keeps any key (skipped: P = 0, no exponentials), every thread keeps every key (no
         // selects), or partly kept (masked scores set to -inf). The classes are warp-uniform, so the
         // branches do not diverge.
-        uint32_t kw[kFChunk / 32];
-        #pragma unroll
-        for (int c = 0; c < kFChunk / 32; ++c) kw[c] = ~0u;
-        uint32_t cany = (1u << (kFChunk / 32)) - 1u, cfull = cany;
+        constexpr uint32_t kAllChunks = (1u << (kFChunk / 32)) - 1u;
+        uint32_t cany = kAllChunks;
         if (!(t.flags & full_bit)) {
+          uint32_t kw[kFChunk / 32];
           if (t.kind == kLinear) {
             #pragma unroll
             for (int c = 0; c < kFChunk / 32; ++c) {
@@ -680,8 +678,8 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
               kw[c] = word;
             }
           }
+          uint32_t cfull = 0;
           cany = 0;
-          cfull = 0;
           #pragma unroll
           for (int c = 0; c < kFChunk / 32; ++c) {
             cany |= __any_sync(0xffffffffu, kw[c] != 0u) ? (1u << c) : 0u;
@@ -696,7 +694,6 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
           }
         }
         // ---- tile max over the chunks some thread keeps (8 independent chains of 3-input maxima)
-        constexpr uint32_t kAllChunks = (1u << (kFChunk / 32)) - 1u;
         float mx[8];
         if (cany == kAllChunks) {  // straight-line: every chunk
           #pragma unroll
@@ -729,6 +726,8 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
         if (m_used == -INFINITY) {
           m_used = mt_scaled;  // nothing accumulated yet (l == 0)
         } else if (mt_scaled > m_used + kRescaleThreshold) {
+          // Lazy rescale: only when the max grows by more than 2^kRescaleThreshold; the final
+          // O / l and the LSE use the same m_used, so the result stays exact up to rounding.
           alpha = ex2_approx(m_used - mt_scaled);
           l *= alpha;
           m_used = mt_scaled;
@@ -758,7 +757,8 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
             const uint64_t x = f32x2_fma(f32x2_pack(s[c], s[c + 1]), sl2x2, nbase2);
             if (CLEAR_FWD_EXP_BF16X2) {
               const uint32_t pb = ex2_approx_bf16x2(pack_bf16x2(f32x2_lo(x), f32x2_hi(x)));
-              acc2[q & 3] = f32x2_add(acc2[q & 3], f32x2_pack(__uint_as_float(pb << 16), __uint_as_float(pb & 0xFFFF0000u)));
+              acc2[q & 3] =
+                  f32x2_add(acc2[q & 3], f32x2_pack(__uint_as_float(pb << 16), __uint_as_float(pb & 0xFFFF0000u)));
               pw[q] = pb;
             } else {
               float e0, e1;

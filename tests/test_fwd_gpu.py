@@ -135,3 +135,24 @@ def test_outputs_only_16_byte_aligned(d):
     o2, lse2 = L.clear_attn_fwd(q, k, v, wl.n_text, wl.H, wl.W, wl.r, o=o, workspace=ws)
     assert L.clear_attn_check() == 0
     assert torch.equal(o2, ref_o) and torch.equal(lse2, ref_lse)
+
+
+@pytest.mark.parametrize("boost", [3.0, 8.0])
+def test_forward_scores_far_above_the_first_tiles(boost):
+    # A row's exponent base is its running max; a later tile whose scores lie far above it must
+    # raise the base and rescale the stored sum and O without losing exactness. Keys in the bottom
+    # image rows are scaled up and aligned with every query, so for many rows the last tiles carry
+    # scores about 30 (boost 3) or 90 (boost 8) log2 units above the text and upper-window keys
+    # visited first. (Much larger scores, in the thousands, also perturb the tensor core's fp32
+    # accumulation of S at the bf16 tolerance's scale; that is not what this checks.)
+    wl = Workload("late_peak", 1, 2, 40, 24, 32, 128, 6)
+    q, k, v = (t.float() for t in make_inputs(wl, seed=21, dtype=torch.float32))
+    q = q.abs() * 0.5 + 0.2
+    img0 = wl.n_text + 16 * wl.W
+    k[:, :, img0:] = k[:, :, img0:].abs() * boost
+    q, k, v = (t.to(torch.bfloat16).cuda() for t in (q, k, v))
+    o, lse = _run(wl, q, k, v)
+    O, LSE = oracle.clear_attention_forward(q.cpu(), k.cpu(), v.cpu(), wl.n_text, wl.H, wl.W, wl.r)
+    assert_close(o.float().cpu().numpy(), O, f"boost {boost} O")
+    rel = np.abs(lse.cpu().numpy() - LSE) / np.maximum(1.0, np.abs(LSE))
+    assert rel.max() <= LSE_ABS, f"boost {boost} LSE rel {rel.max():.3e}"
