@@ -235,7 +235,7 @@ clear_status_t noalloc_geom(Geom* g) {
   if (g->n_text == 0) return CLEAR_OK;
   for (int cap = g->fS; cap >= 1; --cap) {
     Geom t = *g;
-    choose_splits(t.fnC, kFSplitTargetChunks, cap, &t.fS, &t.fcps);
+    choose_splits(t.fnC, 2 * kSplitTargetChunks, cap, &t.fS, &t.fcps);
     t.n_txt_pairs = (long long)t.BH * t.nTq2 * t.fS;
     if (fwd_workspace_layout(t).total <= kNoAllocScratchBytes) {
       *g = t;

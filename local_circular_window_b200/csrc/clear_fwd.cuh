@@ -8,28 +8,26 @@
 //
 // One CTA per SM, persistent over a static list of pair items (clear_sched.cuh). A pair is two
 // 128-row query tiles ("halves" A and B: the upper and lower 8 x 16 rectangles of a 16 x 16 image
-// block, or two consecutive text tiles) that share every 128-key tile: each K/V tile is loaded once
-// and multiplied by whichever halves reach it. Every product is a full-width tensor-core step:
-// S = Q K^T is M128 N128 (K = d), O += P V is M128 N=d (K = 128 keys), P read from TMEM.
+// block, or two consecutive text tiles) that share every 64-key tile: each K/V tile is loaded once
+// and multiplied by whichever halves reach it.
 //   warps 0-3   softmax / epilogue of half A (thread t owns query row t = TMEM lane t);
 //   warps 4-7   softmax / epilogue of half B;
-//   warp 8      TMA producer: Q of each half (its own buffer, reloaded as soon as that half has
-//               issued its last score product of the pair), K and V tiles into 2-slot rings. It
-//               enumerates each union tile once, publishes its descriptor (kind, origin, per-half
-//               need / full bits, last-of-pair and last-needed-by-half bits, head) in a 16-entry
-//               shared ring that the V stream and both MMA issuers read, and posts each half's
-//               tiles (and the end of each pair) to that half's softmax through a 4-slot mailbox;
-//   warps 9/10  MMA issuers, one per half, in a fixed order per needed tile:
-//               S = Q K^T -> (softmax writes P over S) -> O += P V -> next tile's S. With a single S
-//               buffer per half the two halves alternate on the tensor pipe: one half's P V and
-//               next S run while the other half's softmax works. Tiles a half does not need are
-//               still observed and released by that half, so each half sees every phase of every
-//               ring slot in order, which keeps the parity-based waits exact;
+//   warp 8      TMA producer: Q of both halves once per pair, K and V tiles into 4-slot rings. It
+//               enumerates each union tile once and publishes its descriptor (kind, origin, per-half
+//               need / full bits, last-of-pair bit, head) in a 16-entry shared ring that the V
+//               stream and both MMA issuers read, so nobody else re-runs the enumeration;
+//   warps 9/10  MMA issuers, one per half. Each polls two walks over the pair's union tiles: the
+//               QK walk issues S_j = Q K_j^T into one of two 64-column TMEM buffers (up to one
+//               needed tile ahead of P V) and posts the tile to its softmax through a two-slot
+//               mailbox; the PV walk issues O += P_j V_j once the softmax has written P_j over S_j
+//               (bf16, in TMEM; A operand from TMEM). Tiles a half does not need are still
+//               observed (their "full" phase) and released by that half, so each half sees every
+//               phase of every ring slot in order, which keeps the parity-based waits exact.
+//               Polling (instead of blocking) keeps either walk from holding up the other, so
+//               every wait depends only on earlier tiles. The end of a pair is posted to the
+//               softmax as a mailbox message;
 //   warp 11     idle (it completes the third warpgroup, whose registers go to the softmax).
-// TMEM columns of half h: S (fp32) / P (bf16 pairs, first 64 columns) [256h, 256h+128),
-// O [256h+128, 256h+128+d). Products issued by one thread run in order, so an S product issued
-// after the P V product that reads the same columns never overwrites P early, and the S-full
-// commit of tile j also covers the P V of tile j-1 (the softmax may rescale O once S_j is ready).
+// TMEM columns of half h: S buffers [256h, 256h+64) and [256h+64, 256h+128), O [256h+128, 256h+256).
 // The running max is rescaled lazily: O and l are only rescaled when a row's max grows by more
 // than 2^8, which leaves the result exact up to rounding (the final division uses the same max).
 #pragma once
@@ -41,8 +39,8 @@
 
 namespace clear {
 
-constexpr int kKStages = 2;   // K ring slots (128-key tiles)
-constexpr int kVStages = 2;   // V ring slots
+constexpr int kKStages = 4;   // K ring slots
+constexpr int kVStages = 4;   // V ring slots
 constexpr int kFwdThreads = 384;           // 3 warpgroups: softmax A, softmax B, producer + MMA
 // Launched at 168 registers per thread (65536 / 384, rounded to 8). The producer / MMA warpgroup
 // drops to kRegsLow and the two softmax warpgroups grow to kRegsHigh:
@@ -52,12 +50,7 @@ constexpr uint32_t kRegsHigh = 208;
 static_assert(2 * 128 * kRegsHigh + 128 * kRegsLow <= 384 * 168, "register split exceeds the launch allocation");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kTileRing = 16;              // union tile descriptors in flight (producer -> others)
-// Descriptor ring entry x: kind | flags << 4 | these bits.
-constexpr int kRingLastUnion = 1 << 12;    // last union tile of the pair
-constexpr int kRingLastA = 1 << 13;        // last tile of the pair that half A needs
-constexpr int kRingLastB = 1 << 14;        // last tile of the pair that half B needs
-constexpr int kMsgSlots = 4;               // mailbox slots per half (producer -> softmax)
-// Mailbox message kinds (producer -> softmax); tiles use their KeyKind (kLinear / kRect).
+// Mailbox message kinds (issuer -> softmax); tiles use their KeyKind (kLinear / kRect).
 constexpr int kMsgEndPair = 2;             // the half's last tile of the current pair was posted
 constexpr int kMsgEndAll = 3;              // no more pairs for this CTA
 
@@ -100,41 +93,6 @@ __device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
   return d;
 }
 
-// 2^x on the FMA pipe for two packed fp32 values, to take part of the exponentials off the
-// MUFU unit (16 results per clock per SM, as many clocks per tile as the tensor core needs).
-// Range reduction: x = j + f with j = round-to-nearest(x), |f| <= 1/2; j is read from the low
-// mantissa bits of x + 1.5 * 2^23. 2^f is a degree-3 polynomial whose coefficients minimise the
-// maximum relative error on [-1/2, 1/2] (Remez exchange; fit_exp2_poly.py next to this file),
-// 7.5e-5 (2^-13.7), far below the bf16 rounding P gets next. 2^j is added to the exponent field
-// (j * 2^23 added to the bit pattern). x is clamped below at -125 so that the result stays a
-// normal float: a masked score (-inf) gives 2^-125 ~ 2.4e-38 instead of 0, which changes no
-// sum or product at fp32 / bf16 precision.
-constexpr float kExp2C0 = 0.99992806f, kExp2C1 = 0.69326097f, kExp2C2 = 0.24261113f, kExp2C3 = 0.05517167f;
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
-  const float x0 = fmaxf(f32x2_lo(x), -125.f), x1 = fmaxf(f32x2_hi(x), -125.f);
-  const uint64_t xc = f32x2_pack(x0, x1);
-  const uint64_t t = f32x2_add(xc, f32x2_pack(12582912.f, 12582912.f));    // 1.5 * 2^23: rounds to integer
-  const uint64_t j = f32x2_add(t, f32x2_pack(-12582912.f, -12582912.f));   // round(x), exact
-  const uint64_t f = f32x2_fma(j, f32x2_pack(-1.f, -1.f), xc);             // x - round(x), exact
-  uint64_t q = f32x2_fma(f, f32x2_pack(kExp2C3, kExp2C3), f32x2_pack(kExp2C2, kExp2C2));
-  q = f32x2_fma(q, f, f32x2_pack(kExp2C1, kExp2C1));
-  q = f32x2_fma(q, f, f32x2_pack(kExp2C0, kExp2C0));
-  const uint32_t r0 = __float_as_uint(f32x2_lo(q)) + (__float_as_uint(f32x2_lo(t)) << 23);
-  const uint32_t r1 = __float_as_uint(f32x2_hi(q)) + (__float_as_uint(f32x2_hi(t)) << 23);
-  return f32x2_pack(__uint_as_float(r0), __uint_as_float(r1));
-}
-
-// Which column pairs of each 32-column chunk take the polynomial exp2 instead of MUFU ex2
-// (bit q: columns 2q and 2q + 1).
-#ifndef CLEAR_FWD_EXP2_POLY_PAIRS
-#define CLEAR_FWD_EXP2_POLY_PAIRS 0x0000u
-#endif
-// 1: P = 2^x through the MUFU's packed bf16 form: x rounded to bf16, two results per operation,
-// already the bf16 pair the P V product reads; the row sum adds those bf16 values.
-#ifndef CLEAR_FWD_EXP_BF16X2
-#define CLEAR_FWD_EXP_BF16X2 0
-#endif
-
 // One 32-byte global store (the address must be 32-byte aligned).
 __device__ __forceinline__ void st_global_v8(void* ptr, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                              uint32_t a4, uint32_t a5, uint32_t a6, uint32_t a7) {
@@ -146,43 +104,50 @@ __device__ __forceinline__ void st_global_v8(void* ptr, uint32_t a0, uint32_t a1
 template <int D>
 struct FwdLayout {
   static constexpr int kQTileBytes = kTile * D * 2;      // one 128-row bf16 query tile
-  static constexpr int kKVTileBytes = kFChunk * D * 2;   // one 128-key bf16 tile
-  static constexpr int kBlock = kTile * 128;             // 128 rows x 64 elements (128B-swizzled)
+  static constexpr int kKVTileBytes = kFChunk * D * 2;   // one 64-key bf16 tile
+  static constexpr int kKVBlock = kFChunk * 128;         // 64 rows x 64 elements (128B-swizzled)
   static constexpr int kQ = 0;                           // Q_A, Q_B
   static constexpr int kK = kQ + 2 * kQTileBytes;
   static constexpr int kV = kK + kKStages * kKVTileBytes;
   static constexpr int kBars = kV + kVStages * kKVTileBytes;
   // barrier indices
-  static constexpr int bQFull = 0;                       // + half
-  static constexpr int bQEmpty = bQFull + 2;             // + half
-  static constexpr int bKFull = bQEmpty + 2;             // + slot
+  static constexpr int bQFull = 0, bQEmpty = 1;
+  static constexpr int bKFull = 2;                       // + slot
   static constexpr int bKEmpty = bKFull + kKStages;      // + slot
   static constexpr int bVFull = bKEmpty + kKStages;      // + slot
   static constexpr int bVEmpty = bVFull + kVStages;      // + slot
-  static constexpr int bSFull = bVEmpty + kVStages;      // + half: S = Q K^T of the half's tile ready
-  static constexpr int bPFull = bSFull + 2;              // + half: P written over S
-  static constexpr int bMsgFull = bPFull + 2;            // + kMsgSlots * half + slot: mailbox message posted
-  static constexpr int bMsgEmpty = bMsgFull + 2 * kMsgSlots;  // + kMsgSlots * half + slot: mailbox slot read
-  static constexpr int bODone = bMsgEmpty + 2 * kMsgSlots;    // + half: last P V of the half's pair done
-  static constexpr int bExpDone = bODone + 2;            // + half: the half's exponentials of a shared tile done
-  static constexpr int kNumBars = bExpDone + 2;
-  static constexpr int kMsg = kBars + kNumBars * 8;      // int4[2][kMsgSlots] mailbox: {kind, a, b, flags | ordinal << 8}
-  static constexpr int kRing = kMsg + 2 * kMsgSlots * 16;  // int4[kTileRing]: {x bits, a, b, bh}
+  static constexpr int bSFull = bVEmpty + kVStages;      // + 2 * half + buffer
+  static constexpr int bPFull = bSFull + 4;              // + 2 * half + buffer
+  static constexpr int bMsgFull = bPFull + 4;            // + 2 * half + slot: mailbox message posted
+  static constexpr int bMsgEmpty = bMsgFull + 4;         // + 2 * half + slot: mailbox slot read
+  static constexpr int bODone = bMsgEmpty + 4;           // + half: last P V of the half's pair done
+  static constexpr int bOReady = bODone + 2;             // + half: every P V done (one phase per tile)
+  static constexpr int kNumBars = bOReady + 2;
+  static constexpr int kMsg = kBars + kNumBars * 8;      // int4[2][2] mailbox: {kind, a, b, flags | ordinal << 8}
+  static constexpr int kRing = kMsg + 64;                // int4[kTileRing]: {kind | flags << 4 | last << 12, a, b, bh}
   static constexpr int kMisc = kRing + kTileRing * 16;
   static constexpr int kWTab = kMisc + 16;               // int[kMaxRTable] (tile enumeration)
   static constexpr int kHwTab = kWTab + kMaxRTable * 4;  // int16[hw_table_size(r, H)] (masks)
   static constexpr int kFixed = kHwTab + 1024;           // + slack for 1024-byte alignment
   static __host__ __device__ constexpr int alloc_bytes(int hw_entries) { return kFixed + ((hw_entries * 2 + 15) & ~15); }
   static constexpr uint32_t kTmemCols = 512;
-  static __host__ __device__ constexpr uint32_t s_col(int half) { return half * 256; }
+  static __host__ __device__ constexpr uint32_t s_col(int half, int buf) { return half * 256 + buf * 64; }
   static __host__ __device__ constexpr uint32_t o_col(int half) { return half * 256 + 128; }
 };
 
-// Tiles of a pair each half needs (the producer's last-needed bits).
-__device__ __forceinline__ void pair_need_counts(const Geom& g, const PairItem& it, const int* wtab, int wtn, int* na,
-                                              int* nb) {
-  int nu;
-  count_pair_tiles(g, it, wtab, wtn, &nu, na, nb);
+// Loads one 64-key tile (all 64-element column blocks) of k or v: a 64-token chunk (kind kLinear,
+// first token a) or a 4 x 16 grid rectangle (kind kRect, rows from a, columns from b).
+template <int D>
+__device__ __forceinline__ void load_kv64(uint8_t* dst, const CUtensorMap* lin, const CUtensorMap* img, uint64_t* bar,
+                                          int kind, int a, int b, int bh) {
+  #pragma unroll
+  for (int h = 0; h < D / 64; ++h) {
+    uint8_t* d = dst + h * FwdLayout<D>::kKVBlock;
+    if (kind == kLinear)
+      tma_load_3d(d, lin, bar, h * 64, a, bh);
+    else
+      tma_load_4d(d, img, bar, h * 64, b, a, bh);
+  }
 }
 
 template <int D>
@@ -207,14 +172,8 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
   const Geom& g = p.g;
 
   if (threadIdx.x == 0) {
-    for (int h = 0; h < 2; ++h) {
-      mbar_init(&bars[L::bQFull + h], 1);
-      mbar_init(&bars[L::bQEmpty + h], 1);
-      mbar_init(&bars[L::bSFull + h], 1);
-      mbar_init(&bars[L::bPFull + h], 128);
-      mbar_init(&bars[L::bODone + h], 1);
-      mbar_init(&bars[L::bExpDone + h], 128);
-    }
+    mbar_init(&bars[L::bQFull], 1);
+    mbar_init(&bars[L::bQEmpty], 2);
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(&bars[L::bKFull + s], 1);
       mbar_init(&bars[L::bKEmpty + s], 2);
@@ -223,9 +182,15 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
       mbar_init(&bars[L::bVFull + s], 1);
       mbar_init(&bars[L::bVEmpty + s], 2);
     }
-    for (int i = 0; i < 2 * kMsgSlots; ++i) {
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&bars[L::bSFull + i], 1);
+      mbar_init(&bars[L::bPFull + i], 128);
       mbar_init(&bars[L::bMsgFull + i], 1);
       mbar_init(&bars[L::bMsgEmpty + i], 128);
+    }
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&bars[L::bODone + h], 1);
+      mbar_init(&bars[L::bOReady + h], 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -246,261 +211,249 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
   const int wtn = imin(g.r, kMaxRTable);
   const long long stride = gridDim.x;
 
-  // The producer and issuer warps run their loops with all 32 lanes (warp-uniform state, barrier
-  // results combined by votes) and issue each TMA copy, tcgen05 product or commit from one elected
-  // lane: operands that are warp-uniform can then stay in uniform registers.
   if (warp == 8) {
     // ------------------------------------------------------------------ TMA producer
     regs_dec<kRegsLow>();
-    if (elect_one()) {
+    if (lane == 0) {
       tma_prefetch_desc(&tm_q_lin); tma_prefetch_desc(&tm_q_img);
       tma_prefetch_desc(&tm_k_lin); tma_prefetch_desc(&tm_k_img);
       tma_prefetch_desc(&tm_v_lin); tma_prefetch_desc(&tm_v_img);
-    }
-    __syncwarp();
-    // Q stream of each half: pair index and loads so far.
-    long long wq0 = blockIdx.x, wq1 = blockIdx.x;
-    uint32_t nq0 = 0, nq1 = 0;
-    // K stream: the current union tile and a one-tile lookahead (for the last-of-pair bit), and
-    // the tiles each half still needs in the pair (for its last-needed bit).
-    long long wk = blockIdx.x;
-    PairItem itk{};
-    PairKeyIter kik;
-    KeyTile tcur{}, tnext{};
-    int remA = 0, remB = 0;
-    bool kval = wk < p.n_work, next_in_pair = false;
-    if (kval) {
-      itk = decode_pair(g, wk);
-      pair_need_counts(g, itk, wtab, wtn, &remA, &remB);
-      kik.init(g, itk, wtab, wtn);
-      kik.next(&tcur);
-      next_in_pair = kik.next(&tnext);
-    }
-    uint32_t Gk = 0, Gv = 0;
-    uint32_t nm0 = 0, nm1 = 0;   // mailbox messages posted to each half
-    uint32_t pk = 0;             // pair ordinal of the K stream (this CTA's pairs, in order)
-    bool end0 = false, end1 = false;
-    // Slot n of half h's mailbox is free once the softmax has read the message kMsgSlots posts back.
-    auto slot_free = [&](int h, uint32_t n) -> bool {
-      return mbar_test(&bars[L::bMsgEmpty + kMsgSlots * h + n % kMsgSlots], ((n / kMsgSlots) & 1) ^ 1);
-    };
-    auto post = [&](int h, uint32_t n, int4 m) {  // called by the elected lane
-      msg[kMsgSlots * h + n % kMsgSlots] = m;
-      mbar_arrive(&bars[L::bMsgFull + kMsgSlots * h + n % kMsgSlots]);
-    };
-    PollWatchdog wd;
-    wd.start();
-    while (wq0 < p.n_work || wq1 < p.n_work || kval || Gv < Gk || !end0 || !end1) {
-      bool prog = false;
-      #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        long long& wq = h ? wq1 : wq0;
-        uint32_t& nq = h ? nq1 : nq0;
-        if (wq < p.n_work &&
-            (nq == 0 || __any_sync(0xffffffffu, mbar_test(&bars[L::bQEmpty + h], (nq - 1) & 1)))) {
+      long long wq = blockIdx.x;
+      uint32_t q_loads = 0;
+      // K stream: the current union tile and a one-tile lookahead (for the last-of-pair bit).
+      long long wk = blockIdx.x;
+      PairItem itk{};
+      PairKeyIter kik;
+      KeyTile tcur{}, tnext{};
+      bool kval = wk < p.n_work, next_in_pair = false;
+      if (kval) {
+        itk = decode_pair(g, wk);
+        kik.init(g, itk, wtab, wtn);
+        kik.next(&tcur);
+        next_in_pair = kik.next(&tnext);
+      }
+      uint32_t Gk = 0, Gv = 0;
+      PollWatchdog wd;
+      wd.start();
+      while (wq < p.n_work || kval || Gv < Gk) {
+        bool prog = false;
+        if (wq < p.n_work && (q_loads == 0 || mbar_test(&bars[L::bQEmpty], (q_loads - 1) & 1))) {
           const PairItem it = decode_pair(g, wq);
-          if (elect_one()) {
-            if (h == 0 || it.validB) {
-              mbar_arrive_expect_tx(&bars[L::bQFull + h], L::kQTileBytes);
-              if (it.is_text)
-                load_tile<D>(smem + L::kQ + h * L::kQTileBytes, &tm_q_lin, &tm_q_img, &bars[L::bQFull + h], kLinear,
-                             it.q0 + h * kTile, 0, it.bh);
-              else
-                load_tile<D>(smem + L::kQ + h * L::kQTileBytes, &tm_q_lin, &tm_q_img, &bars[L::bQFull + h], kRect,
-                             it.q0 + h * kQH, it.x0, it.bh);
-            } else {
-              mbar_arrive(&bars[L::bQFull + h]);  // no query rows: the phase completes empty
-            }
+          mbar_arrive_expect_tx(&bars[L::bQFull], (it.validB ? 2 : 1) * L::kQTileBytes);
+          if (it.is_text) {
+            load_tile<D>(smem + L::kQ, &tm_q_lin, &tm_q_img, &bars[L::bQFull], kLinear, it.q0, 0, it.bh);
+            if (it.validB)
+              load_tile<D>(smem + L::kQ + L::kQTileBytes, &tm_q_lin, &tm_q_img, &bars[L::bQFull], kLinear,
+                           it.q0 + kTile, 0, it.bh);
+          } else {
+            load_tile<D>(smem + L::kQ, &tm_q_lin, &tm_q_img, &bars[L::bQFull], kRect, it.q0, it.x0, it.bh);
+            if (it.validB)
+              load_tile<D>(smem + L::kQ + L::kQTileBytes, &tm_q_lin, &tm_q_img, &bars[L::bQFull], kRect,
+                           it.q0 + kQH, it.x0, it.bh);
           }
-          __syncwarp();
-          ++nq;
+          ++q_loads;
           wq += stride;
           prog = true;
         }
-      }
-      if (kval && Gk - Gv < (uint32_t)kTileRing) {
-        const uint32_t ks = Gk % kKStages;
-        const bool needA = tcur.flags & kNeedA, needB = tcur.flags & kNeedB;
-        const bool lastA = needA && remA == 1, lastB = needB && remB == 1;
-        // The K slot and the mailbox slots this tile's messages take (the tile, and the end of the
-        // pair after a half's last tile) must all be free.
-        bool ready = mbar_test(&bars[L::bKEmpty + ks], ((Gk / kKStages) & 1) ^ 1);
-        if (needA) ready = ready && slot_free(0, nm0) && (!lastA || slot_free(0, nm0 + 1));
-        if (needB) ready = ready && slot_free(1, nm1) && (!lastB || slot_free(1, nm1 + 1));
-        if (__all_sync(0xffffffffu, ready)) {
-          int bits = tcur.kind | (tcur.flags << 4) | (next_in_pair ? 0 : kRingLastUnion);
-          if (lastA) bits |= kRingLastA;
-          if (lastB) bits |= kRingLastB;
-          remA -= needA ? 1 : 0;
-          remB -= needB ? 1 : 0;
-          if (elect_one()) {
-            const int4 m = make_int4(tcur.kind, tcur.a, tcur.b, tcur.flags | (int)(pk << 8));
-            if (needA) post(0, nm0, m);
-            if (lastA) post(0, nm0 + 1, make_int4(kMsgEndPair, 0, 0, 0));
-            if (needB) post(1, nm1, m);
-            if (lastB) post(1, nm1 + 1, make_int4(kMsgEndPair, 0, 0, 0));
+        if (kval && Gk - Gv < (uint32_t)kTileRing) {
+          const uint32_t ks = Gk % kKStages;
+          if (mbar_test(&bars[L::bKEmpty + ks], ((Gk / kKStages) & 1) ^ 1)) {
             // Publish the descriptor before the load: the K barrier's completion makes it visible.
-            ring[Gk % kTileRing] = make_int4(bits, tcur.a, tcur.b, itk.bh);
+            ring[Gk % kTileRing] = make_int4(tcur.kind | (tcur.flags << 4) | (next_in_pair ? 0 : (1 << 12)), tcur.a,
+                                             tcur.b, itk.bh);
             mbar_arrive_expect_tx(&bars[L::bKFull + ks], L::kKVTileBytes);
-            load_tile<D>(smem + L::kK + ks * L::kKVTileBytes, &tm_k_lin, &tm_k_img, &bars[L::bKFull + ks], tcur.kind,
+            load_kv64<D>(smem + L::kK + ks * L::kKVTileBytes, &tm_k_lin, &tm_k_img, &bars[L::bKFull + ks], tcur.kind,
                          tcur.a, tcur.b, itk.bh);
-          }
-          __syncwarp();
-          nm0 += (needA ? 1 : 0) + (lastA ? 1 : 0);
-          nm1 += (needB ? 1 : 0) + (lastB ? 1 : 0);
-          ++Gk;
-          if (next_in_pair) {
-            tcur = tnext;
-            next_in_pair = kik.next(&tnext);
-          } else {
-            ++pk;
-            wk += stride;
-            kval = wk < p.n_work;
-            if (kval) {
-              itk = decode_pair(g, wk);
-              pair_need_counts(g, itk, wtab, wtn, &remA, &remB);
-              kik.init(g, itk, wtab, wtn);
-              kik.next(&tcur);
+            ++Gk;
+            if (next_in_pair) {
+              tcur = tnext;
               next_in_pair = kik.next(&tnext);
+            } else {
+              wk += stride;
+              kval = wk < p.n_work;
+              if (kval) {
+                itk = decode_pair(g, wk);
+                kik.init(g, itk, wtab, wtn);
+                kik.next(&tcur);
+                next_in_pair = kik.next(&tnext);
+              }
             }
-          }
-          prog = true;
-        }
-      }
-      if (!kval && (!end0 || !end1)) {  // every tile posted: tell both softmax warpgroups to stop
-        #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          bool& done = h ? end1 : end0;
-          const uint32_t n = h ? nm1 : nm0;
-          if (!done && __all_sync(0xffffffffu, slot_free(h, n))) {
-            if (elect_one()) post(h, n, make_int4(kMsgEndAll, 0, 0, 0));
-            __syncwarp();
-            done = true;
             prog = true;
           }
         }
-      }
-      if (Gv < Gk) {
-        const uint32_t vs = Gv % kVStages;
-        if (__any_sync(0xffffffffu, mbar_test(&bars[L::bVEmpty + vs], ((Gv / kVStages) & 1) ^ 1))) {
-          if (elect_one()) {
+        if (Gv < Gk) {
+          const uint32_t vs = Gv % kVStages;
+          if (mbar_test(&bars[L::bVEmpty + vs], ((Gv / kVStages) & 1) ^ 1)) {
             const int4 e = ring[Gv % kTileRing];
             mbar_arrive_expect_tx(&bars[L::bVFull + vs], L::kKVTileBytes);
-            load_tile<D>(smem + L::kV + vs * L::kKVTileBytes, &tm_v_lin, &tm_v_img, &bars[L::bVFull + vs], e.x & 15,
+            load_kv64<D>(smem + L::kV + vs * L::kKVTileBytes, &tm_v_lin, &tm_v_img, &bars[L::bVFull + vs], e.x & 15,
                          e.y, e.z, e.w);
+            ++Gv;
+            prog = true;
           }
-          __syncwarp();
-          ++Gv;
-          prog = true;
         }
+        if (!wd.tick(prog, abort_flag, kDevTimeoutTmaEmpty, 1, (int)Gk, (int)Gv, (int)q_loads)) break;
       }
-      const bool alive = wd.tick(prog, abort_flag, kDevTimeoutTmaEmpty, 1, (int)Gk, (int)Gv, (int)(nm0 | (nm1 << 16)));
-      if (!__all_sync(0xffffffffu, alive)) break;
     }
+    __syncwarp();
   } else if (warp == 9 || warp == 10) {
     // ------------------------------------------------------------------ MMA issuers (one per half)
     regs_dec<kRegsLow>();
-    constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kFChunk, 0, 0);
-    constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-    const int h = warp - 9;
-    const int need_bit = h == 0 ? kNeedA : kNeedB;
-    const int last_bit = h == 0 ? kRingLastA : kRingLastB;
-    const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
-    const uint32_t s_tm = tm + L::s_col(h);
-    const uint32_t o_tm = tm + L::o_col(h);
-    // Shared-memory matrix descriptors, advanced per 16-element K step with plain adds.
-    const uint64_t qdesc = smem_desc_sw128(smem_u32(smem + L::kQ + h * L::kQTileBytes), 16, 1024);
-    const uint64_t kdesc0 = smem_desc_sw128(smem_u32(smem + L::kK), 16, 1024);
-    const uint64_t vdesc0 = smem_desc_sw128(smem_u32(smem + L::kV), L::kBlock, 1024);
-    const uint32_t n_pairs = (uint32_t)((p.n_work - blockIdx.x + stride - 1) / stride);
-    uint32_t G = 0;     // union tiles observed
-    uint32_t nS = 0;    // tiles this half multiplied (S / P phases)
-    bool ok = true;
-    // Bounded wait by every lane; the warp goes on only if all of them saw the phase.
-    auto wait_all = [&](uint64_t* bar, uint32_t parity, int site) -> bool {
-      const bool r = mbar_wait(bar, parity, abort_flag, kDevTimeoutMma, site, (int)G, (int)nS);
-      return __all_sync(0xffffffffu, r);
-    };
-    for (uint32_t pair = 0; ok && pair < n_pairs; ++pair) {
-      // Every half observes every Q phase (a half without query rows gets an empty phase).
-      if (!wait_all(&bars[L::bQFull + h], pair & 1, 4 + h)) {
-        ok = false;
-        break;
-      }
-      bool had = false, q_released = false, o_done = false;
-      while (true) {
-        const uint32_t ks = G % kKStages, vs = G % kVStages;
-        if (!wait_all(&bars[L::bKFull + ks], (G / kKStages) & 1, 6 + h)) {
-          ok = false;
-          break;
-        }
-        const int ex = __shfl_sync(0xffffffffu, ring[G % kTileRing].x, 0);
-        const int flags = (ex >> 4) & 255;
-        const bool last_union = (ex & kRingLastUnion) != 0;
-        if (flags & need_bit) {
-          const bool last_h = (ex & last_bit) != 0;
-          const uint64_t kd = kdesc0 + (uint64_t)((ks * L::kKVTileBytes) >> 4);
-          if (elect_one()) {
-            tc_fence_after();
-            #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = ((kk >> 2) * L::kBlock + (kk & 3) * 32) >> 4;
-              umma_ss(s_tm, qdesc + off, kd + off, idesc_qk, kk > 0);
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kFChunk, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+      const int h = warp - 9;
+      const int need_bit = h == 0 ? kNeedA : kNeedB;
+      const uint32_t q_addr = smem_u32(smem + L::kQ + h * L::kQTileBytes);
+      const uint32_t o_tm = tmem + L::o_col(h);
+      // Shared-memory matrix descriptors, advanced per 16-element K step with plain adds.
+      const uint64_t qdesc = smem_desc_sw128(q_addr, 16, 1024);
+      const uint64_t kdesc0 = smem_desc_sw128(smem_u32(smem + L::kK), 16, 1024);
+      const uint64_t vdesc0 = smem_desc_sw128(smem_u32(smem + L::kV), L::kKVBlock, 1024);
+      const uint32_t n_pairs = (uint32_t)((p.n_work - blockIdx.x + stride - 1) / stride);
+      // QK walk over the union tiles (union index Gq); pairs are observed in order.
+      uint32_t pair = 0, Gq = 0, nqk = 0, nmsg = 0;
+      bool q_seen = false, had = false, end_pending = false, all_posted = false;
+      // PV walk: union index Gp; up to two needed tiles whose Q K^T is issued and P V is not.
+      uint32_t Gp = 0, npv = 0;
+      // The pending tiles form a two-entry FIFO kept in registers (head h*, tail t*): union index,
+      // and flags (bit 0: first of the pair, overwrite O; bit 1: commit o_done after its P V).
+      uint32_t hG = 0, tG = 0;
+      int hF = 0, tF = 0;
+      int pend = 0;
+      PollWatchdog wd;
+      wd.start();
+      while (!all_posted || Gp < Gq || pend > 0) {
+        bool prog = false;
+        // ---- PV walk step (tiles the QK walk has passed, in order). It goes first: a ready P V
+        // frees the S buffer the next Q K^T needs.
+        if (Gp < Gq) {
+          const uint32_t vs = Gp % kVStages;
+          const bool needed = pend > 0 && hG == Gp;
+          if (!needed) {
+            if (mbar_test(&bars[L::bVFull + vs], (Gp / kVStages) & 1)) {
+              mbar_arrive(&bars[L::bVEmpty + vs]);  // observed and released
+              ++Gp;
+              prog = true;
             }
-            umma_commit(&bars[L::bSFull + h]);
-            umma_commit(&bars[L::bKEmpty + ks]);
-            if (last_h) umma_commit(&bars[L::bQEmpty + h]);  // the half's Q may be reloaded for its next pair
+          } else {
+            const uint32_t b = npv & 1;
+            const bool pr = mbar_test(&bars[L::bPFull + 2 * h + b], (npv >> 1) & 1);
+            const bool vr = mbar_test(&bars[L::bVFull + vs], (Gp / kVStages) & 1);
+            if (pr && vr) {
+              tc_fence_after();
+              const uint64_t vd = vdesc0 + (uint64_t)((vs * L::kKVTileBytes) >> 4);
+              const uint32_t s_tm = tmem + L::s_col(h, b);
+              const bool first = hF & 1;
+              #pragma unroll
+              for (int kk = 0; kk < kFChunk / 16; ++kk)
+                umma_ts(o_tm, s_tm + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv,
+                        (!first || kk > 0) ? 1u : 0u);
+              umma_commit(&bars[L::bVEmpty + vs]);
+              umma_commit(&bars[L::bOReady + h]);
+              if (hF & 2) umma_commit(&bars[L::bODone + h]);
+              ++npv;
+              --pend;
+              hG = tG;
+              hF = tF;
+              ++Gp;
+              prog = true;
+            }
           }
-          __syncwarp();
-          q_released |= last_h;
-          if (!wait_all(&bars[L::bVFull + vs], (G / kVStages) & 1, 8 + h) ||
-              !wait_all(&bars[L::bPFull + h], nS & 1, 18 + h)) {
-            ok = false;
-            break;
-          }
-          const uint64_t vd = vdesc0 + (uint64_t)((vs * L::kKVTileBytes) >> 4);
-          if (elect_one()) {
-            tc_fence_after();
-            #pragma unroll
-            for (int kk = 0; kk < kFChunk / 16; ++kk)
-              umma_ts(o_tm, s_tm + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv, (had || kk > 0) ? 1u : 0u);
-            umma_commit(&bars[L::bVEmpty + vs]);
-            if (last_h) umma_commit(&bars[L::bODone + h]);
-          }
-          __syncwarp();
-          had = true;
-          ++nS;
-          o_done |= last_h;
-        } else {
-          // Not needed by this half: observed and released (after its V load, so the slot's
-          // phases stay in step with the other half).
-          if (elect_one()) mbar_arrive(&bars[L::bKEmpty + ks]);
-          __syncwarp();
-          if (!wait_all(&bars[L::bVFull + vs], (G / kVStages) & 1, 8 + h)) {
-            ok = false;
-            break;
-          }
-          if (elect_one()) mbar_arrive(&bars[L::bVEmpty + vs]);
-          __syncwarp();
         }
-        ++G;
-        if (last_union) break;
-      }
-      if (!ok) break;
-      if (!q_released) {
-        if (elect_one()) {
-          if (had)
-            umma_commit(&bars[L::bQEmpty + h]);
-          else
-            mbar_arrive(&bars[L::bQEmpty + h]);
+        // ---- QK walk step
+        if (end_pending || (pair >= n_pairs && !all_posted)) {
+          // Post an end-of-pair (or end-of-work) message once the mailbox slot is free.
+          const uint32_t ms = nmsg & 1;
+          if (mbar_test(&bars[L::bMsgEmpty + 2 * h + ms], ((nmsg >> 1) & 1) ^ 1)) {
+            msg[2 * h + ms] = make_int4(end_pending ? kMsgEndPair : kMsgEndAll, 0, 0, 0);
+            mbar_arrive(&bars[L::bMsgFull + 2 * h + ms]);
+            ++nmsg;
+            if (end_pending) end_pending = false; else all_posted = true;
+            prog = true;
+          }
+        } else if (pair < n_pairs) {
+          if (!q_seen) {
+            if (mbar_test(&bars[L::bQFull], pair & 1)) {  // every half observes every Q phase
+              q_seen = true;
+              had = false;
+              prog = true;
+            }
+          } else {
+            const uint32_t ks = Gq % kKStages;
+            const uint32_t ms = nmsg & 1;
+            // The K barrier, the ring entry and the mailbox are read back to back so their
+            // latencies overlap; the test's acquire orders the ring read, and the entry is used
+            // only once the test has passed.
+            const bool kr = mbar_test(&bars[L::bKFull + ks], (Gq / kKStages) & 1);
+            const int4 e = ring[Gq % kTileRing];
+            const bool mr = mbar_test(&bars[L::bMsgEmpty + 2 * h + ms], ((nmsg >> 1) & 1) ^ 1);
+            if (kr) {
+              const int flags = (e.x >> 4) & 255;
+              const bool last_of_pair = (e.x >> 12) & 1;
+              const bool needed = (flags & need_bit) != 0;
+              bool done_tile = false;
+              if (!needed) {
+                mbar_arrive(&bars[L::bKEmpty + ks]);  // observed and released
+                done_tile = true;
+              } else if (pend < 2 && mr) {
+                const uint32_t b = nqk & 1;
+                msg[2 * h + ms] = make_int4(e.x & 15, e.y, e.z, flags | (int)(pair << 8));
+                mbar_arrive(&bars[L::bMsgFull + 2 * h + ms]);
+                ++nmsg;
+                tc_fence_after();
+                const uint64_t kd = kdesc0 + (uint64_t)((ks * L::kKVTileBytes) >> 4);
+                #pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                  const uint32_t qoff = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+                  const uint32_t koff = ((kk >> 2) * L::kKVBlock + (kk & 3) * 32) >> 4;
+                  umma_ss(tmem + L::s_col(h, b), qdesc + qoff, kd + koff, idesc_qk, kk > 0);
+                }
+                umma_commit(&bars[L::bSFull + 2 * h + b]);
+                umma_commit(&bars[L::bKEmpty + ks]);
+                if (pend == 0) {
+                  hG = Gq;
+                  hF = had ? 0 : 1;
+                } else {
+                  tG = Gq;
+                  tF = had ? 0 : 1;
+                }
+                ++pend;
+                ++nqk;
+                had = true;
+                done_tile = true;
+              }
+              if (done_tile) {
+                ++Gq;
+                prog = true;
+                if (last_of_pair) {
+                  // Pair finished for this half: release Q, arrange o_done, tell the softmax.
+                  if (had) {
+                    umma_commit(&bars[L::bQEmpty]);
+                    // o_done follows this half's last P V of the pair: mark it if still pending
+                    // (it is the most recent needed tile), else commit now.
+                    if (pend == 2)
+                      tF |= 2;
+                    else if (pend == 1)
+                      hF |= 2;
+                    else
+                      umma_commit(&bars[L::bODone + h]);
+                    end_pending = true;
+                  } else {
+                    mbar_arrive(&bars[L::bQEmpty]);
+                  }
+                  ++pair;
+                  q_seen = false;
+                }
+              }
+            }
+          }
         }
-        __syncwarp();
-      }
-      if (had && !o_done) {  // not reached: the producer marks every half's last tile of a pair
-        if (elect_one()) umma_commit(&bars[L::bODone + h]);
-        __syncwarp();
+        if (!wd.tick(prog, abort_flag, kDevTimeoutMma, 2 + h, (int)Gq, (int)(Gp | (npv << 16)),
+                     pend | (end_pending ? 4 : 0) | (all_posted ? 8 : 0) | (q_seen ? 16 : 0) | ((int)pair << 8))) break;
       }
     }
+    __syncwarp();
   } else if (warp == 11) {
     regs_dec<kRegsLow>();
   } else {
@@ -510,10 +463,8 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
     const int row = threadIdx.x & 127;       // TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t o_tm = tmem + lane_base + L::o_col(half);
-    const uint32_t s_tm = tmem + lane_base + L::s_col(half);
     const int full_bit = half == 0 ? kFullA : kFullB;
     uint32_t nq = 0, n_out = 0, nmsg = 0;
-    uint32_t nboth = 0;  // tiles both halves multiply, seen so far (exponential-phase turns)
     const float sl2 = p.scale_log2;
     // Per-pair state, set up at the pair's first tile.
     PairItem it{};
@@ -524,12 +475,12 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
     float l = 0.f;
     int j = 0;
     while (true) {
-      const uint32_t ms = nmsg % kMsgSlots;
-      if (!mbar_wait(&bars[L::bMsgFull + kMsgSlots * half + ms], (nmsg / kMsgSlots) & 1, abort_flag,
-                     kDevTimeoutSoftmax, 10 + half, (int)nmsg, j))
+      const uint32_t ms = nmsg & 1;
+      if (!mbar_wait(&bars[L::bMsgFull + 2 * half + ms], (nmsg >> 1) & 1, abort_flag, kDevTimeoutSoftmax, 10 + half,
+                     (int)nmsg, j))
         goto softmax_done;
-      const int4 mv = msg[kMsgSlots * half + ms];
-      mbar_arrive(&bars[L::bMsgEmpty + kMsgSlots * half + ms]);
+      const int4 mv = msg[2 * half + ms];
+      mbar_arrive(&bars[L::bMsgEmpty + 2 * half + ms]);
       ++nmsg;
       if (mv.x == kMsgEndAll) break;
       if (mv.x == kMsgEndPair) {
@@ -542,7 +493,7 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
         if (it.is_text) {
           const size_t prow = ((size_t)it.split * g.BH + it.bh) * g.n_text + (row_valid ? tq : 0);
           float* dst = p.opart + prow * D;
-          // Two TMEM loads per wait; each row's run is written 32 (or 16) bytes at a time.
+          // Two TMEM loads per wait; each row's 512-byte run is written 32 (or 16) bytes at a time.
           #pragma unroll
           for (int c = 0; c < D / 32; c += 2) {
             uint32_t ov[2][32];
@@ -628,97 +579,52 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
         l = 0.f;
       }
       {
-        if (!mbar_wait(&bars[L::bSFull + half], nq & 1, abort_flag, kDevTimeoutSoftmax, 12 + half, (int)nq, j))
+        const uint32_t b = nq & 1, ph = (nq >> 1) & 1;
+        if (!mbar_wait(&bars[L::bSFull + 2 * half + b], ph, abort_flag, kDevTimeoutSoftmax, 12 + half, (int)nq, j))
           goto softmax_done;
         tc_fence_after();
+        const uint32_t s_tm = tmem + lane_base + L::s_col(half, b);
         float s[kFChunk];
         {
-          uint32_t sr[kFChunk / 32][32];
-          #pragma unroll
-          for (int c = 0; c < kFChunk / 32; ++c) tmem_ld32(s_tm + c * 32, sr[c]);
+          uint32_t sr[2][32];
+          tmem_ld32(s_tm + 0, sr[0]);
+          tmem_ld32(s_tm + 32, sr[1]);
           tmem_wait_ld();
           #pragma unroll
           for (int c = 0; c < kFChunk; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
         }
-        // ---- mask. kw[c]: keep bits of this row's columns 32c .. 32c+31 (a rectangle's key rows
-        // 2c and 2c+1, 16 bits each). Each 32-column chunk is then classed over the warp: no thread
-        // keeps any key (skipped: P = 0, no exponentials), every thread keeps every key (no
-        // selects), or partly kept (masked scores set to -inf). The classes are warp-uniform, so the
-        // branches do not diverge.
-        constexpr uint32_t kAllChunks = (1u << (kFChunk / 32)) - 1u;
-        uint32_t cany = kAllChunks;
+        // ---- mask (branch-free selects; full tiles skip it)
         if (!(t.flags & full_bit)) {
-          uint32_t kw[kFChunk / 32];
           if (t.kind == kLinear) {
+            const int lim = t.b;
             #pragma unroll
-            for (int c = 0; c < kFChunk / 32; ++c) {
-              const int n = t.b - 32 * c;  // valid keys of the chunk
-              kw[c] = n >= 32 ? ~0u : (n <= 0 ? 0u : ((1u << n) - 1u));
-            }
+            for (int c = 0; c < kFChunk; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
           } else {
-            // Row ky keeps columns [xc - w, xc + w] of the grid, w = half-width at |ky - yc|
-            // (none when |ky - yc| >= r or ky is past the grid): clipped to the rectangle's 16
-            // columns and the grid, as a 16-bit run.
-            const int xr = xc - t.b;
-            const int hi_lim = imin(g.W - 1 - t.b, kKW - 1);
+            // keep bits: word q holds key rows 2q (bits 0-15) and 2q+1 (bits 16-31)
+            uint32_t keep[kFKH / 2];
             #pragma unroll
-            for (int c = 0; c < kFChunk / 32; ++c) {
-              uint32_t word = 0;
-              #pragma unroll
-              for (int u = 0; u < 2; ++u) {
-                const int ky = t.a + 2 * c + u;
-                const int dy = ky - yc;
-                const int ady = dy < 0 ? -dy : dy;
-                int w = hwtab[imin(ady, hwn - 1)];
-                w = (ady < hwn && ky < g.H) ? w : -1;
-                const int lo = imin(imax(xr - w, 0), kKW);
-                const int hi = imax(imin(xr + w, hi_lim), -1);
-                word |= ((0xFFFFu >> (15 - hi)) & (0xFFFFu << lo) & 0xFFFFu) << (16 * u);
-              }
-              kw[c] = word;
+            for (int q = 0; q < kFKH / 2; ++q) {
+              int lo0, hi0, lo1, hi1;
+              row_range_tab(g, hwtab, hwn, yc, xc, t.a + 2 * q, t.b, &lo0, &hi0);
+              row_range_tab(g, hwtab, hwn, yc, xc, t.a + 2 * q + 1, t.b, &lo1, &hi1);
+              const int n0 = imax(hi0 - lo0 + 1, 0), n1 = imax(hi1 - lo1 + 1, 0);
+              keep[q] = (((1u << n0) - 1u) << (lo0 & 15)) | ((((1u << n1) - 1u) << (lo1 & 15)) << 16);
             }
-          }
-          uint32_t cfull = 0;
-          cany = 0;
-          #pragma unroll
-          for (int c = 0; c < kFChunk / 32; ++c) {
-            cany |= __any_sync(0xffffffffu, kw[c] != 0u) ? (1u << c) : 0u;
-            cfull |= __all_sync(0xffffffffu, kw[c] == ~0u) ? (1u << c) : 0u;
-          }
-          #pragma unroll
-          for (int c = 0; c < kFChunk / 32; ++c) {
-            if (((cany & ~cfull) >> c) & 1u) {
-              #pragma unroll
-              for (int e = 0; e < 32; ++e) s[32 * c + e] = ((kw[c] >> e) & 1u) ? s[32 * c + e] : -INFINITY;
-            }
+            #pragma unroll
+            for (int c = 0; c < kFChunk; ++c)
+              s[c] = (keep[c >> 5] & (1u << (c & 31))) ? s[c] : -INFINITY;
           }
         }
-        // ---- tile max over the chunks some thread keeps (8 independent chains of 3-input maxima)
+        // ---- tile max (8 independent chains of 3-input maxima)
         float mx[8];
-        if (cany == kAllChunks) {  // straight-line: every chunk
-          #pragma unroll
-          for (int u = 0; u < 8; ++u) mx[u] = fmax3(s[u], s[u + 8], s[u + 16]);
-          #pragma unroll
-          for (int c = 24; c + 16 <= kFChunk - 8; c += 16) {
-            #pragma unroll
-            for (int u = 0; u < 8; ++u) mx[u] = fmax3(mx[u], s[c + u], s[c + 8 + u]);
-          }
-          #pragma unroll
-          for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], s[kFChunk - 8 + u]);
-        } else {
-          #pragma unroll
-          for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
-          #pragma unroll
-          for (int c = 0; c < kFChunk / 32; ++c) {
-            if ((cany >> c) & 1u) {
-              #pragma unroll
-              for (int u = 0; u < 8; ++u) {
-                mx[u] = fmax3(mx[u], s[32 * c + u], s[32 * c + 8 + u]);
-                mx[u] = fmax3(mx[u], s[32 * c + 16 + u], s[32 * c + 24 + u]);
-              }
-            }
-          }
-        }
+        #pragma unroll
+        for (int u = 0; u < 8; ++u) mx[u] = fmax3(s[u], s[u + 8], s[u + 16]);
+        #pragma unroll
+        for (int u = 0; u < 8; ++u) mx[u] = fmax3(mx[u], s[u + 24], s[u + 32]);
+        #pragma unroll
+        for (int u = 0; u < 8; ++u) mx[u] = fmax3(mx[u], s[u + 40], s[u + 48]);
+        #pragma unroll
+        for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], s[u + 56]);
         const float mt = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(fmax3(mx[3], mx[4], mx[5]), mx[6], mx[7]));
         const float mt_scaled = mt * sl2;
         float alpha = 1.f;
@@ -726,82 +632,17 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
         if (m_used == -INFINITY) {
           m_used = mt_scaled;  // nothing accumulated yet (l == 0)
         } else if (mt_scaled > m_used + kRescaleThreshold) {
-          // Lazy rescale: only when the max grows by more than 2^kRescaleThreshold; the final
-          // O / l and the LSE use the same m_used, so the result stays exact up to rounding.
           alpha = ex2_approx(m_used - mt_scaled);
           l *= alpha;
           m_used = mt_scaled;
           need_rescale = true;
         }
-        // ---- The two halves take turns at the exponentials of a tile both of them multiply: half A
-        // after half B's previous such tile, half B after half A's same tile. Each half then has
-        // the MUFU unit to itself while the tensor core runs the other half's products, instead of
-        // both halves computing at once and both waiting for the tensor core afterwards.
-        const bool both = (t.flags & (kNeedA | kNeedB)) == (kNeedA | kNeedB);
-        if (both && (half == 1 || nboth > 0)) {
-          const uint32_t ph = half == 0 ? ((nboth - 1) & 1) : (nboth & 1);
-          if (!mbar_wait(&bars[L::bExpDone + (half ^ 1)], ph, abort_flag, kDevTimeoutSoftmax, 20 + half, (int)nboth,
-                         (int)nq))
-            goto softmax_done;
-        }
-        // ---- P = 2^(s * scale_log2 - m), row sum, bf16 pairs written over S in TMEM
-        const float base = (m_used == -INFINITY) ? 0.f : m_used;
-        const uint64_t sl2x2 = f32x2_pack(sl2, sl2), nbase2 = f32x2_pack(-base, -base);
-        uint64_t acc2[4] = {0, 0, 0, 0};
-        // P for columns 32c .. 32c+31: 16 bf16 pairs, row-sum terms into acc2, stored over S.
-        auto exp_chunk = [&](int c4) {
-          uint32_t pw[16];
-          #pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            const int c = 32 * c4 + 2 * q;
-            const uint64_t x = f32x2_fma(f32x2_pack(s[c], s[c + 1]), sl2x2, nbase2);
-            if (CLEAR_FWD_EXP_BF16X2) {
-              const uint32_t pb = ex2_approx_bf16x2(pack_bf16x2(f32x2_lo(x), f32x2_hi(x)));
-              acc2[q & 3] =
-                  f32x2_add(acc2[q & 3], f32x2_pack(__uint_as_float(pb << 16), __uint_as_float(pb & 0xFFFF0000u)));
-              pw[q] = pb;
-            } else {
-              float e0, e1;
-              if ((CLEAR_FWD_EXP2_POLY_PAIRS >> q) & 1u) {
-                const uint64_t e = exp2_poly_x2(x);
-                e0 = f32x2_lo(e);
-                e1 = f32x2_hi(e);
-              } else {
-                e0 = ex2_approx(f32x2_lo(x));
-                e1 = ex2_approx(f32x2_hi(x));
-              }
-              acc2[q & 3] = f32x2_add(acc2[q & 3], f32x2_pack(e0, e1));
-              pw[q] = pack_bf16x2(e0, e1);
-            }
-          }
-          tmem_st16(s_tm + c4 * 16, pw);
-        };
-        if (cany == kAllChunks) {  // straight-line: every chunk
-          #pragma unroll
-          for (int c4 = 0; c4 < kFChunk / 32; ++c4) exp_chunk(c4);
-        } else {
-          #pragma unroll
-          for (int c4 = 0; c4 < kFChunk / 32; ++c4) {
-            if ((cany >> c4) & 1u) {
-              exp_chunk(c4);
-            } else {  // no thread keeps a key of this chunk: P = 0
-              uint32_t pw[16];
-              #pragma unroll
-              for (int q = 0; q < 16; ++q) pw[q] = 0u;
-              tmem_st16(s_tm + c4 * 16, pw);
-            }
-          }
-        }
-        if (both) {
-          mbar_arrive(&bars[L::bExpDone + half]);
-          ++nboth;
-        }
-        l += ((f32x2_lo(acc2[0]) + f32x2_hi(acc2[0])) + (f32x2_lo(acc2[1]) + f32x2_hi(acc2[1]))) +
-             ((f32x2_lo(acc2[2]) + f32x2_hi(acc2[2])) + (f32x2_lo(acc2[3]) + f32x2_hi(acc2[3])));
         if (j > 0 && __any_sync(0xffffffffu, need_rescale)) {
-          // O holds P V up to tile j-1, complete: the S-full commit of this tile was issued after
-          // it. Rescale O in place; P V of this tile waits for the P-full signal below. (Done
-          // after P is written, when the score registers are free.)
+          // O holds P V up to tile j-1: wait for that product (the one for tile j cannot start
+          // before this tile's P is signalled), then rescale O in place.
+          if (!mbar_wait(&bars[L::bOReady + half], (nq - 1) & 1, abort_flag, kDevTimeoutSoftmax, 14 + half, (int)nq, j))
+            goto softmax_done;
+          tc_fence_after();
           #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t ov[32];
@@ -812,9 +653,25 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
             tmem_st32(o_tm + c * 32, ov);
           }
         }
+        // ---- P = 2^(s * scale_log2 - m), row sum, bf16 pairs written over S in TMEM
+        const float base = (m_used == -INFINITY) ? 0.f : m_used;
+        const uint64_t sl2x2 = f32x2_pack(sl2, sl2), nbase2 = f32x2_pack(-base, -base);
+        uint64_t acc2[4] = {0, 0, 0, 0};
+        uint32_t pw[32];
+        #pragma unroll
+        for (int q = 0; q < 32; ++q) {
+          const uint64_t x = f32x2_fma(f32x2_pack(s[2 * q], s[2 * q + 1]), sl2x2, nbase2);
+          const float e0 = ex2_approx(f32x2_lo(x));
+          const float e1 = ex2_approx(f32x2_hi(x));
+          acc2[q & 3] = f32x2_add(acc2[q & 3], f32x2_pack(e0, e1));
+          pw[q] = pack_bf16x2(e0, e1);
+        }
+        tmem_st32(s_tm, pw);
+        l += ((f32x2_lo(acc2[0]) + f32x2_hi(acc2[0])) + (f32x2_lo(acc2[1]) + f32x2_hi(acc2[1]))) +
+             ((f32x2_lo(acc2[2]) + f32x2_hi(acc2[2])) + (f32x2_lo(acc2[3]) + f32x2_hi(acc2[3])));
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars[L::bPFull + half]);
+        mbar_arrive(&bars[L::bPFull + 2 * half + b]);
         ++nq;
         ++j;
       }

@@ -42,10 +42,10 @@ constexpr int kQW = 16;     // image query tile columns
 constexpr int kKH = 8;      // image key tile rows
 constexpr int kKW = 16;     // image key tile columns
 constexpr int kTile = 128;  // rows per query tile, keys per key tile
-// The forward pairs two query tiles that share 128-key tiles: 8 x 16 grid rectangles or 128-token
-// chunks, so every score product is a full-width M128 N128 tensor-core step.
-constexpr int kFKH = 8;       // forward key rectangle rows
-constexpr int kFChunk = 128;  // forward keys per tile
+// The forward pairs two query tiles and visits 64-key tiles: 4 x 16 grid rectangles or 64-token
+// chunks (half-size key tiles let each half double-buffer S in tensor memory).
+constexpr int kFKH = 4;       // forward key rectangle rows
+constexpr int kFChunk = 64;   // forward keys per tile
 
 enum KeyKind : int { kLinear = 0, kRect = 1 };
 enum KeyFlags : int { kNeedsMask = 0, kFull = 1 };
@@ -75,12 +75,12 @@ struct Geom {
   int cps;           // chunks per split
   long long n_txt_items, n_img_items;
   // Forward pairs: two query tiles share every key tile they visit (a 16 x 16 image block, or
-  // two consecutive 128-row text tiles); key tiles are kFChunk keys.
+  // two consecutive 128-row text tiles); key tiles are 64 keys.
   int nqy2, nQ2;     // image blocks per (b, h): ceil(H/16) x ceil(W/16)
   int nTq2;          // text tile pairs: ceil(nTq / 2)
-  int fnC;           // forward key chunks (kFChunk tokens) over all T tokens
-  int fnTk;          // forward key chunks over the text tokens
-  int fS, fcps;      // forward text splits and key chunks per split
+  int fnC;           // 64-key chunks over all T tokens
+  int fnTk;          // 64-key chunks over the text tokens
+  int fS, fcps;      // forward text splits and 64-key chunks per split
   long long n_txt_pairs, n_img_pairs;
 };
 
@@ -131,7 +131,6 @@ CLEAR_HD void choose_splits(int nC, int target, int max_splits, int* S, int* cps
 }
 
 constexpr int kSplitTargetChunks = 64;
-constexpr int kFSplitTargetChunks = 8192 / kFChunk;  // forward: about 8192 keys per split
 constexpr int kMaxSplits = 32;
 
 CLEAR_HD Geom make_geom(int B, int heads, int n_text, int H, int W, int d, int r, int window = kCircle) {
@@ -154,7 +153,7 @@ CLEAR_HD Geom make_geom(int B, int heads, int n_text, int H, int W, int d, int r
   g.nTq2 = cdiv(g.nTq, 2);
   g.fnC = cdiv(g.T, kFChunk);
   g.fnTk = cdiv(n_text, kFChunk);
-  choose_splits(g.fnC, kFSplitTargetChunks, kMaxSplits, &g.fS, &g.fcps);
+  choose_splits(g.fnC, 2 * kSplitTargetChunks, kMaxSplits, &g.fS, &g.fcps);
   g.n_txt_pairs = (long long)g.BH * g.nTq2 * g.fS;
   g.n_img_pairs = (long long)g.BH * g.nQ2;
   return g;
@@ -330,16 +329,10 @@ CLEAR_HD PairItem decode_pair(const Geom& g, long long w) {
   return it;
 }
 
-// Union key tiles of a pair (kFChunk keys each), with per-half need / full flags. Image blocks visit
-// the text chunks, then the 16-column rectangles (kFKH key rows each) covering the union of both
-// halves' windows; a tile is needed by a half iff some (query of that half, key of the tile) pair
-// is kept. Rectangles neither half reaches are skipped.
-//
-// Band order: the top bands are reached by half A only and the bottom bands by half B only, so
-// bands are taken from both ends inward (0 with n-1, then 1 with n-2, ...), and within such a band
-// pair the tiles alternate between the two bands (top column 0, bottom column 0, top column 1, ...).
-// Consecutive tiles then tend to feed different halves, so neither half waits long for the other
-// on the shared K/V ring.
+// Union key tiles of a pair (64 keys each), with per-half need / full flags. Image blocks visit the
+// 64-token text chunks, then band by band (4 key rows) the 16-column rectangles covering the union
+// of both halves' windows; a tile is needed by a half iff some (query of that half, key of the
+// tile) pair is kept.
 struct PairKeyIter {
   const int* wtab;
   int wtab_n;
@@ -348,23 +341,20 @@ struct PairKeyIter {
   int yA0, yAl, yB0, yBl;     // half rows (clipped); B rows only if validB
   int ky_begin, ky_end;
   int lin_next, lin_end;
-  int n_bands, next_pair;     // band pairs (t, n_bands-1-t) are loaded in order of t
-  // Current top (t) and bottom (b) band of the pair: first key row, next column, last column.
-  // (Plain fields, not arrays: a runtime-indexed array would live in local memory on the device.)
-  int ky_t, kx_t, kxe_t, ky_b, kx_b, kxe_b;
-  int side;                   // band the next tile is taken from: 0 top, 1 bottom
+  int band_ky, kx, kx_end;
+  int band_step, n_bands;     // bands are visited ends-inward: 0, n-1, 1, n-2, ...
 
   CLEAR_HD void init(const Geom& g, const PairItem& it, const int* table = nullptr, int table_n = 0) {
     wtab = table;
     wtab_n = table_n;
     is_text = it.is_text; r = g.r; window = g.window; H = g.H; W = g.W; n_text = g.n_text; T = g.T;
     validB = it.validB;
-    ky_t = ky_b = 0; kx_t = kx_b = 1; kxe_t = kxe_b = 0; side = 0;
     if (is_text) {
       lin_next = it.c_begin;
       lin_end = it.c_end;
-      y0 = x0 = xl = yA0 = yAl = yB0 = yBl = 0; ky_begin = 0; ky_end = -1;
-      n_bands = next_pair = 0;
+      band_ky = 1; ky_end = 0; kx = 1; kx_end = 0;
+      y0 = x0 = xl = yA0 = yAl = yB0 = yBl = 0; ky_begin = 0;
+      band_step = n_bands = 0;
       return;
     }
     lin_next = 0;
@@ -383,47 +373,42 @@ struct PairKeyIter {
     ky_begin = imax(0, y0 - (r - 1));
     ky_end = imin(H - 1, ylast + (r - 1));
     n_bands = (ky_end - ky_begin) / kFKH + 1;
-    next_pair = 0;
+    band_step = 0;
+    band_ky = ky_begin;
+    kx = 1; kx_end = 0;
   }
 
   CLEAR_HD int hw(int dy) const { return (dy < wtab_n) ? wtab[dy] : half_width(r, dy, window); }
 
-  // Column range of band k (key rows from ky_begin + k*kFKH) that some query of the block reaches;
-  // an empty range (kx > kx_end) when none does.
-  CLEAR_HD void band_cols(int k, int* kyy, int* kxx, int* kxe) const {
+  // Next band with kept columns. The first and last bands are reached by one half only (the
+  // top ones by half A, the bottom ones by half B); alternating from both ends keeps both halves
+  // busy instead of leaving one idle at the start of the pair and the other at its end.
+  CLEAR_HD bool advance_band() {
     const int ylast = validB ? yBl : yAl;
-    *kyy = ky_begin + k * kFKH;
-    const int band_last = imin(*kyy + kFKH - 1, H - 1);
-    const int dmin = imax(0, imax(y0 - band_last, *kyy - ylast));
-    const int w = hw(dmin);
-    *kxx = 1; *kxe = 0;
-    if (w < 0) return;
-    *kxx = imax(0, x0 - w);
-    *kxe = imin(W - 1, xl + w);
-  }
-
-  // Loads the next band pair with at least one column; false when none is left.
-  CLEAR_HD bool advance_bands() {
     while (true) {
-      const int t = next_pair, b = n_bands - 1 - next_pair;
-      if (t > b) return false;
-      ++next_pair;
-      band_cols(t, &ky_t, &kx_t, &kxe_t);
-      if (b != t) band_cols(b, &ky_b, &kx_b, &kxe_b); else { kx_b = 1; kxe_b = 0; }
-      side = 0;
-      if (kx_t <= kxe_t || kx_b <= kxe_b) return true;
+      if (band_step >= n_bands) return false;
+      const int k = (band_step & 1) ? n_bands - 1 - (band_step >> 1) : (band_step >> 1);
+      ++band_step;
+      band_ky = ky_begin + k * kFKH;
+      const int band_last = imin(band_ky + kFKH - 1, H - 1);
+      const int dmin = imax(0, imax(y0 - band_last, band_ky - ylast));
+      const int w = hw(dmin);
+      if (w < 0) continue;
+      kx = imax(0, x0 - w);
+      kx_end = imin(W - 1, xl + w);
+      if (kx <= kx_end) return true;
     }
   }
 
-  // need / full of rectangle [ky, ky+kFKH) x [kx, kx+16) for query rows [qa, qb], columns [x0, xl].
-  CLEAR_HD int half_flags(int kyy, int kxx, int qa, int qb, int need_bit, int full_bit) const {
-    const int kyl = imin(kyy + kFKH - 1, H - 1);
+  // need / full of rectangle [ky, ky+4) x [kx, kx+16) for query rows [qa, qb], columns [x0, xl].
+  CLEAR_HD int half_flags(int ky, int kxx, int qa, int qb, int need_bit, int full_bit) const {
+    const int kyl = imin(ky + kFKH - 1, H - 1);
     const int kxl = imin(kxx + kKW - 1, W - 1);
-    const int dy = imax(0, imax(qa - kyl, kyy - qb));
+    const int dy = imax(0, imax(qa - kyl, ky - qb));
     const int dx = imax(0, imax(x0 - kxl, kxx - xl));
     if (!within(r, window, dx, dy)) return 0;
-    const bool inside = (kyy + kFKH - 1 <= H - 1) && (kxx + kKW - 1 <= W - 1);
-    const int mdy = imax(kyy + kFKH - 1 - qa, qb - kyy);
+    const bool inside = (ky + kFKH - 1 <= H - 1) && (kxx + kKW - 1 <= W - 1);
+    const int mdy = imax(ky + kFKH - 1 - qa, qb - ky);
     const int mdx = imax(kxx + kKW - 1 - x0, xl - kxx);
     return need_bit | ((inside && within(r, window, mdx, mdy)) ? full_bit : 0);
   }
@@ -442,22 +427,17 @@ struct PairKeyIter {
     }
     if (is_text) return false;
     while (true) {
-      if (kx_t > kxe_t && kx_b > kxe_b) {
-        if (!advance_bands()) return false;
+      if (kx > kx_end) {
+        if (!advance_band()) return false;
       }
-      const bool bottom = side ? (kx_b <= kxe_b) : !(kx_t <= kxe_t);
-      side = bottom ? 0 : 1;
-      const int kyy = bottom ? ky_b : ky_t, kxx = bottom ? kx_b : kx_t;
-      if (bottom) kx_b += kKW; else kx_t += kKW;
-      const int f = half_flags(kyy, kxx, yA0, yAl, kNeedA, kFullA) |
-                    (validB ? half_flags(kyy, kxx, yB0, yBl, kNeedB, kFullB) : 0);
-      if (f & (kNeedA | kNeedB)) {
-        t->kind = kRect;
-        t->a = kyy;
-        t->b = kxx;
-        t->flags = f;
-        return true;
-      }
+      const int f = half_flags(band_ky, kx, yA0, yAl, kNeedA, kFullA) |
+                    (validB ? half_flags(band_ky, kx, yB0, yBl, kNeedB, kFullB) : 0);
+      t->kind = kRect;
+      t->a = band_ky;
+      t->b = kx;
+      t->flags = f;
+      kx += kKW;
+      if (f & (kNeedA | kNeedB)) return true;  // rectangles neither half reaches are skipped
     }
   }
 };

@@ -9,8 +9,8 @@ import pytest
 import local_circular_window_b200 as L
 import oracle
 
-KQH, KQW, KKH, KKW, TILE = 8, 16, 8, 16, 128
-KCHUNK = 128  # forward key tiles: 128-token chunks or 8 x 16 rectangles
+KQH, KQW, KKH, KKW, TILE = 8, 16, 4, 16, 128
+KCHUNK = 64  # forward key tiles: 64-token chunks or 4 x 16 rectangles
 
 
 def _keys_of_tile(tile, n_text, H, W, T):
@@ -138,5 +138,5 @@ def test_split_shape_at_8k():
     p = L.make_params(1, 24, 512, 512, 512, 128, 8)
     n_txt_items, n_img_items, S, cps = L.forward_shape(p)
     assert n_img_items == 24 * (512 // 16) * (512 // 16)
-    assert S * cps >= (512 + 512 * 512 + 127) // 128 and S <= 32
+    assert S * cps >= (512 + 512 * 512 + 63) // 64 and S <= 32
     assert n_txt_items == 24 * 2 * S
