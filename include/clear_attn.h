@@ -104,6 +104,30 @@ CLEAR_API clear_status_t clear_attn_fwd(const clear_attn_params_t* params, const
                               const void* v, void* o, float* lse, void* workspace,
                               size_t workspace_bytes, void* stream);
 
+/* Element strides of q, k, v and o for clear_attn_fwd_strided: {batch, head, token} for each
+ * tensor, in elements (not bytes). The d elements of one token row are contiguous. */
+typedef struct {
+  long long q[3], k[3], v[3], o[3];
+} clear_attn_strides_t;
+
+/*
+ * Forward on strided tensors: the same operation and results as clear_attn_fwd (bit for bit: the
+ * arithmetic and its order are the same), but element (b, h, t, i) of q is read at
+ *   q + b * strides->q[0] + h * strides->q[1] + t * strides->q[2] + i
+ * (likewise k, v), and row (b, h, t) of o is written at the same place of o with strides->o. This
+ * reads, e.g., a packed [B, T, 3, heads, d] qkv buffer (q = buf, k = buf + heads*d,
+ * v = buf + 2*heads*d, strides {T*3*heads*d, d, 3*heads*d}) and writes o as [B, T, heads, d], with
+ * no copy. The paper has no counterpart (its model feeds attention from such a packed projection).
+ *   strides  every stride a positive multiple of 8 elements (16 bytes, as TMA requires) and below
+ *            2^39, else CLEAR_ERR_UNSUPPORTED; NULL is CLEAR_ERR_INVALID_ARG. Overlapping o rows
+ *            are the caller's error (results undefined).
+ *   lse      fp32 [B, heads, T], contiguous, as in clear_attn_fwd.
+ *   Pointers 16-byte aligned; workspace as for clear_attn_fwd (same size query).
+ */
+CLEAR_API clear_status_t clear_attn_fwd_strided(const clear_attn_params_t* params, const clear_attn_strides_t* strides,
+                                                const void* q, const void* k, const void* v, void* o, float* lse,
+                                                void* workspace, size_t workspace_bytes, void* stream);
+
 /*
  * Forward for callers that cannot allocate device memory: same inputs, outputs and results as
  * clear_attn_fwd (up to the summation order of the text rows), but no workspace argument. The

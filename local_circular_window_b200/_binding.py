@@ -26,6 +26,12 @@ STATUS_NAMES = {0: "CLEAR_OK", 1: "CLEAR_ERR_INVALID_ARG", 2: "CLEAR_ERR_UNSUPPO
                 4: "CLEAR_ERR_CUDA", 5: "CLEAR_ERR_DEVICE_TIMEOUT"}
 
 
+class ClearStrides(ctypes.Structure):
+    """Mirror of clear_attn_strides_t: {batch, head, token} element strides of q, k, v and o."""
+    _fields_ = [("q", ctypes.c_longlong * 3), ("k", ctypes.c_longlong * 3), ("v", ctypes.c_longlong * 3),
+                ("o", ctypes.c_longlong * 3)]
+
+
 class ClearParams(ctypes.Structure):
     """Mirror of clear_attn_params_t."""
     _fields_ = [("B", ctypes.c_int), ("heads", ctypes.c_int), ("n_text", ctypes.c_int), ("H", ctypes.c_int),
@@ -59,6 +65,9 @@ _lib.clear_attn_bwd_workspace_size.restype = ctypes.c_size_t
 _lib.clear_attn_bwd_workspace_size.argtypes = [_P, ctypes.POINTER(_i)]
 _lib.clear_attn_fwd.restype = _i
 _lib.clear_attn_fwd.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+_lib.clear_attn_fwd_strided.restype = _i
+_lib.clear_attn_fwd_strided.argtypes = [_P, ctypes.POINTER(ClearStrides), _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t,
+                                        _vp]
 _lib.clear_attn_fwd_noalloc.restype = _i
 _lib.clear_attn_fwd_noalloc.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.clear_attn_fwd_host_workspace_size.restype = ctypes.c_size_t
@@ -199,6 +208,43 @@ def clear_attn_fwd(q, k, v, n_text: int, H: int, W: int, r: int, o=None, lse=Non
                              _stream_ptr(stream))
     if st != CLEAR_OK:
         raise ClearError(st, "clear_attn_fwd")
+    return o, lse
+
+
+def _bht_strides(t):
+    return (t.stride(0), t.stride(1), t.stride(2))
+
+
+def clear_attn_fwd_strided(q, k, v, n_text: int, H: int, W: int, r: int, o=None, lse=None, workspace=None,
+                           stream=None, window="circle"):
+    """CLEAR attention forward on strided [B, heads, T, d] views (each token row contiguous), e.g.
+    q = qkv[:, :, 0].permute(0, 2, 1, 3) of a packed [B, T, 3, heads, d] buffer, through
+    clear_attn_fwd_strided: nothing is copied. o may be any such view (allocated contiguous if None).
+    Returns (o, lse)."""
+    B, heads, T, d = q.shape
+    if T != n_text + H * W:
+        raise ValueError("T must equal n_text + H * W")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and tuple(t.shape) == tuple(q.shape) and t.stride(3) == 1):
+            raise ValueError(f"{name} must be a CUDA bf16 view of shape {tuple(q.shape)} with contiguous rows")
+    p = make_params(B, heads, n_text, H, W, d, r, window)
+    if o is None:
+        o = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    if not (o.is_cuda and o.dtype == torch.bfloat16 and tuple(o.shape) == tuple(q.shape) and o.stride(3) == 1):
+        raise ValueError(f"o must be a CUDA bf16 view of shape {tuple(q.shape)} with contiguous rows")
+    if lse is None:
+        lse = torch.empty((B, heads, T), dtype=torch.float32, device=q.device)
+    st = ClearStrides((ctypes.c_longlong * 3)(*_bht_strides(q)), (ctypes.c_longlong * 3)(*_bht_strides(k)),
+                      (ctypes.c_longlong * 3)(*_bht_strides(v)), (ctypes.c_longlong * 3)(*_bht_strides(o)))
+    ws_bytes = fwd_workspace_size(p)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    status = _lib.clear_attn_fwd_strided(ctypes.byref(p), ctypes.byref(st), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                         _ptr(lse), _ptr(workspace),
+                                         0 if workspace is None else workspace.numel() * workspace.element_size(),
+                                         _stream_ptr(stream))
+    if status != CLEAR_OK:
+        raise ClearError(status, "clear_attn_fwd_strided")
     return o, lse
 
 

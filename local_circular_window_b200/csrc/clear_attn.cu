@@ -163,15 +163,81 @@ bool make_qkv_maps(QKVMaps* m, const void* q, const void* k, const void* v, cons
          make_linear_map(&m->v_lin, v, g) && make_image_map(&m->v_img, v, g);
 }
 
-// Forward maps: 128-row query tiles, 64-key K/V tiles (64-token chunks and 4 x 16 rectangles).
-bool make_fwd_maps(QKVMaps* m, const void* q, const void* k, const void* v, const Geom& g) {
-  return make_linear_map(&m->q_lin, q, g) && make_image_map(&m->q_img, q, g) &&
-         make_linear_map(&m->k_lin, k, g, kFChunk) && make_image_map(&m->k_img, k, g, kFKH) &&
-         make_linear_map(&m->v_lin, v, g, kFChunk) && make_image_map(&m->v_img, v, g, kFKH);
+// Element strides of one [B, heads, T, d] view: batch, head, token (d is contiguous).
+struct TensorStrides {
+  long long sb, sh, st;
+};
+
+TensorStrides contiguous_strides(const Geom& g) {
+  return TensorStrides{(long long)g.heads * g.T * g.d, (long long)g.T * g.d, (long long)g.d};
 }
 
-template <int D>
-clear_status_t launch_fwd(const Geom& g, const QKVMaps& m, void* o, float* lse, void* ws,
+// Whether b*heads+h can be one axis of stride sh (then the forward uses the flat maps).
+bool flat_bh(const TensorStrides& t, const Geom& g) { return g.B == 1 || t.sb == (long long)g.heads * t.sh; }
+
+// Forward view of q, k or v. Flat: linear (d, T, B*heads) with box 64 x rows x 1 and image
+// (d, W, H, B*heads) from token n_text with box 64 x 16 x rows x 1. Split: the same with separate
+// head and batch axes, (d, T, heads, B) and (d, W, H, heads, B).
+bool make_fwd_tensor_maps(CUtensorMap* lin, CUtensorMap* img, const void* base, const TensorStrides& t, const Geom& g,
+                          int lin_rows, int img_rows, bool split) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t e = 2;  // bytes per element
+  if (!split) {
+    cuuint64_t dims[3] = {(cuuint64_t)g.d, (cuuint64_t)g.T, (cuuint64_t)g.BH};
+    cuuint64_t strides[2] = {(cuuint64_t)t.st * e, (cuuint64_t)t.sh * e};
+    cuuint32_t box[3] = {64, (cuuint32_t)lin_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(lin, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+    const char* ib = static_cast<const char*>(base) + (size_t)g.n_text * t.st * e;
+    cuuint64_t idims[4] = {(cuuint64_t)g.d, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.BH};
+    cuuint64_t istrides[3] = {(cuuint64_t)t.st * e, (cuuint64_t)g.W * t.st * e, (cuuint64_t)t.sh * e};
+    cuuint32_t ibox[4] = {64, (cuuint32_t)kKW, (cuuint32_t)img_rows, 1};
+    cuuint32_t iestr[4] = {1, 1, 1, 1};
+    return enc(img, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<char*>(ib), idims, istrides, ibox, iestr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
+  {
+    cuuint64_t dims[4] = {(cuuint64_t)g.d, (cuuint64_t)g.T, (cuuint64_t)g.heads, (cuuint64_t)g.B};
+    cuuint64_t strides[3] = {(cuuint64_t)t.st * e, (cuuint64_t)t.sh * e, (cuuint64_t)t.sb * e};
+    cuuint32_t box[4] = {64, (cuuint32_t)lin_rows, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (enc(lin, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  const char* ib = static_cast<const char*>(base) + (size_t)g.n_text * t.st * e;
+  cuuint64_t dims[5] = {(cuuint64_t)g.d, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.heads, (cuuint64_t)g.B};
+  cuuint64_t strides[4] = {(cuuint64_t)t.st * e, (cuuint64_t)g.W * t.st * e, (cuuint64_t)t.sh * e, (cuuint64_t)t.sb * e};
+  cuuint32_t box[5] = {64, (cuuint32_t)kKW, (cuuint32_t)img_rows, 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return enc(img, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<char*>(ib), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Forward maps: 128-row query tiles, 64-key K/V tiles (64-token chunks and 4 x 16 rectangles).
+bool make_fwd_maps(QKVMaps* m, const void* q, const void* k, const void* v, const TensorStrides* st,
+                   const Geom& g, bool split) {
+  return make_fwd_tensor_maps(&m->q_lin, &m->q_img, q, st[0], g, kTile, kQH, split) &&
+         make_fwd_tensor_maps(&m->k_lin, &m->k_img, k, st[1], g, kFChunk, kFKH, split) &&
+         make_fwd_tensor_maps(&m->v_lin, &m->v_img, v, st[2], g, kFChunk, kFKH, split);
+}
+
+// Strides the forward accepts: positive multiples of 8 elements (16 bytes, the TMA stride rule), so
+// that every token row starts 16-byte aligned when the base is.
+bool strides_ok(const TensorStrides& t) {
+  return t.sb > 0 && t.sh > 0 && t.st > 0 && t.sb % 8 == 0 && t.sh % 8 == 0 && t.st % 8 == 0 &&
+         t.sb < (1ll << 39) && t.sh < (1ll << 39) && t.st < (1ll << 39);
+}
+
+template <int D, bool kSplit>
+clear_status_t launch_fwd(const Geom& g, const QKVMaps& m, void* o, const TensorStrides& os, float* lse, void* ws,
                           int num_sms, cudaStream_t stream) {
   using L = FwdLayout<D>;
   const int smem_bytes = L::alloc_bytes(hw_table_size(g.r, g.H));
@@ -180,24 +246,27 @@ clear_status_t launch_fwd(const Geom& g, const QKVMaps& m, void* o, float* lse, 
   p.g = g;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   p.o = static_cast<__nv_bfloat16*>(o);
+  p.o_sb = os.sb;
+  p.o_sh = os.sh;
+  p.o_st = os.st;
   p.lse = lse;
   const FwdWorkspace wl = fwd_workspace_layout(g);
   p.opart = g.n_text ? reinterpret_cast<float*>(static_cast<char*>(ws) + wl.opart_off) : nullptr;
-  p.wide_o = (reinterpret_cast<uintptr_t>(o) & 31u) == 0;
+  p.wide_o = (reinterpret_cast<uintptr_t>(o) & 31u) == 0 && os.sb % 16 == 0 && os.sh % 16 == 0 && os.st % 16 == 0;
   p.wide_part = (reinterpret_cast<uintptr_t>(p.opart) & 31u) == 0;
   p.ml = g.n_text ? reinterpret_cast<float2*>(static_cast<char*>(ws) + wl.ml_off) : nullptr;
   p.n_work = g.n_txt_pairs + g.n_img_pairs;
-  if (cudaFuncSetAttribute(clear_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(clear_fwd_kernel<D, kSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smem_bytes) != cudaSuccess)
     return CLEAR_ERR_CUDA;
   const long long grid = p.n_work < num_sms ? p.n_work : num_sms;
-  clear_fwd_kernel<D><<<(unsigned)grid, kFwdThreads, smem_bytes, stream>>>(
+  clear_fwd_kernel<D, kSplit><<<(unsigned)grid, kFwdThreads, smem_bytes, stream>>>(
       m.q_lin, m.q_img, m.k_lin, m.k_img, m.v_lin, m.v_img, p);
   if (cudaGetLastError() != cudaSuccess) return CLEAR_ERR_CUDA;
   if (g.n_text > 0) {
     const long long rows = (long long)g.BH * g.n_text;
     const int wpb = 8;
-    clear_fwd_combine_kernel<D><<<(unsigned)((rows + wpb - 1) / wpb), wpb * 32, 0, stream>>>(p);
+    clear_fwd_combine_kernel<D, kSplit><<<(unsigned)((rows + wpb - 1) / wpb), wpb * 32, 0, stream>>>(p);
     if (cudaGetLastError() != cudaSuccess) return CLEAR_ERR_CUDA;
   }
   return CLEAR_OK;
@@ -347,6 +416,22 @@ clear_status_t copy_streams(cudaStream_t* h2d, cudaStream_t* d2h) {
   return CLEAR_OK;
 }
 
+// The forward on tensors with the given strides (q, k, v, o), once the arguments are checked.
+clear_status_t run_fwd(const Geom& g, const TensorStrides* st4, const void* q, const void* k, const void* v, void* o,
+                       float* lse, void* workspace, cudaStream_t s) {
+  int num_sms = 0;
+  const clear_status_t st = check_device(&num_sms);
+  if (st != CLEAR_OK) return st;
+  const bool split = !(flat_bh(st4[0], g) && flat_bh(st4[1], g) && flat_bh(st4[2], g) && flat_bh(st4[3], g));
+  QKVMaps maps;
+  if (!make_fwd_maps(&maps, q, k, v, st4, g, split)) return CLEAR_ERR_CUDA;
+  if (split)
+    return g.d == 128 ? launch_fwd<128, true>(g, maps, o, st4[3], lse, workspace, num_sms, s)
+                      : launch_fwd<64, true>(g, maps, o, st4[3], lse, workspace, num_sms, s);
+  return g.d == 128 ? launch_fwd<128, false>(g, maps, o, st4[3], lse, workspace, num_sms, s)
+                    : launch_fwd<64, false>(g, maps, o, st4[3], lse, workspace, num_sms, s);
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------------------------------------
@@ -392,14 +477,27 @@ clear_status_t clear_attn_fwd(const clear_attn_params_t* params, const void* q, 
     return CLEAR_ERR_INVALID_ARG;
   const size_t need = fwd_workspace_layout(c.g).total;
   if (need > 0 && (workspace_bytes < need || !aligned16(workspace))) return CLEAR_ERR_WORKSPACE;
-  int num_sms = 0;
-  clear_status_t st = check_device(&num_sms);
-  if (st != CLEAR_OK) return st;
-  QKVMaps maps;
-  if (!make_fwd_maps(&maps, q, k, v, c.g)) return CLEAR_ERR_CUDA;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return c.g.d == 128 ? launch_fwd<128>(c.g, maps, o, lse, workspace, num_sms, s)
-                      : launch_fwd<64>(c.g, maps, o, lse, workspace, num_sms, s);
+  const TensorStrides cs = contiguous_strides(c.g);
+  const TensorStrides st4[4] = {cs, cs, cs, cs};
+  return run_fwd(c.g, st4, q, k, v, o, lse, workspace, static_cast<cudaStream_t>(stream));
+}
+
+clear_status_t clear_attn_fwd_strided(const clear_attn_params_t* params, const clear_attn_strides_t* strides,
+                                      const void* q, const void* k, const void* v, void* o, float* lse,
+                                      void* workspace, size_t workspace_bytes, void* stream) {
+  const Checked c = check_params(params);
+  if (c.st != CLEAR_OK) return c.st;
+  if (!strides || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return CLEAR_ERR_INVALID_ARG;
+  const TensorStrides st4[4] = {{strides->q[0], strides->q[1], strides->q[2]},
+                                {strides->k[0], strides->k[1], strides->k[2]},
+                                {strides->v[0], strides->v[1], strides->v[2]},
+                                {strides->o[0], strides->o[1], strides->o[2]}};
+  for (const TensorStrides& t : st4)
+    if (!strides_ok(t)) return CLEAR_ERR_UNSUPPORTED;
+  const size_t need = fwd_workspace_layout(c.g).total;
+  if (need > 0 && (workspace_bytes < need || !aligned16(workspace))) return CLEAR_ERR_WORKSPACE;
+  return run_fwd(c.g, st4, q, k, v, o, lse, workspace, static_cast<cudaStream_t>(stream));
 }
 
 clear_status_t clear_attn_fwd_noalloc(const clear_attn_params_t* params, const void* q, const void* k,
@@ -417,11 +515,9 @@ clear_status_t clear_attn_fwd_noalloc(const clear_attn_params_t* params, const v
   void* scratch = nullptr;
   st = noalloc_scratch(&scratch);
   if (st != CLEAR_OK) return st;
-  QKVMaps maps;
-  if (!make_fwd_maps(&maps, q, k, v, g)) return CLEAR_ERR_CUDA;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return g.d == 128 ? launch_fwd<128>(g, maps, o, lse, scratch, num_sms, s)
-                    : launch_fwd<64>(g, maps, o, lse, scratch, num_sms, s);
+  const TensorStrides cs = contiguous_strides(g);
+  const TensorStrides st4[4] = {cs, cs, cs, cs};
+  return run_fwd(g, st4, q, k, v, o, lse, scratch, static_cast<cudaStream_t>(stream));
 }
 
 size_t clear_attn_fwd_host_workspace_size(const clear_attn_params_t* params, clear_status_t* status) {

@@ -57,7 +57,10 @@ constexpr int kMsgEndAll = 3;              // no more pairs for this CTA
 struct FwdParams {
   Geom g;
   float scale_log2;           // (1/sqrt(d)) * log2(e)
-  __nv_bfloat16* o;           // [BH, T, d]
+  __nv_bfloat16* o;           // row (b, h, t) at o + b * o_sb + h * o_sh + t * o_st (elements)
+  long long o_sb, o_sh, o_st;
+  // The kernel's kSplit parameter: q, k, v maps (and o) have separate head and batch axes; without
+  // it one flat b*heads+h axis, and row (bh, t) of o sits at o + bh * o_sh + t * o_st.
   float* lse;                 // [BH, T]
   float* opart;               // [fS, BH, n_text, d] unnormalised partial O of text rows
   float2* ml;                 // [fS, BH, n_text] (running max in scaled log2 units, sum)
@@ -135,22 +138,55 @@ struct FwdLayout {
   static __host__ __device__ constexpr uint32_t o_col(int half) { return half * 256 + 128; }
 };
 
+// The forward's tensor maps view q, k, v with one flat b*heads+h axis when the layout allows it
+// (batch stride = heads x head stride, or B = 1): linear (d, T, B*heads) and image (d, W, H,
+// B*heads) maps. Otherwise (split_bh) they have separate head and batch axes, so any token, head and
+// batch strides (multiples of 16 bytes) are read in place: (d, T, heads, B) and (d, W, H, heads, B),
+// and a tile's (head, batch) coordinates come from its bh = b * heads + h.
 // Loads one 64-key tile (all 64-element column blocks) of k or v: a 64-token chunk (kind kLinear,
 // first token a) or a 4 x 16 grid rectangle (kind kRect, rows from a, columns from b).
-template <int D>
+template <int D, bool kSplit>
 __device__ __forceinline__ void load_kv64(uint8_t* dst, const CUtensorMap* lin, const CUtensorMap* img, uint64_t* bar,
-                                          int kind, int a, int b, int bh) {
+                                          int kind, int a, int b, int bh, int heads) {
   #pragma unroll
   for (int h = 0; h < D / 64; ++h) {
     uint8_t* d = dst + h * FwdLayout<D>::kKVBlock;
-    if (kind == kLinear)
-      tma_load_3d(d, lin, bar, h * 64, a, bh);
-    else
-      tma_load_4d(d, img, bar, h * 64, b, a, bh);
+    if (!kSplit) {
+      if (kind == kLinear)
+        tma_load_3d(d, lin, bar, h * 64, a, bh);
+      else
+        tma_load_4d(d, img, bar, h * 64, b, a, bh);
+    } else {
+      const int hh = bh % heads, bb = bh / heads;
+      if (kind == kLinear)
+        tma_load_4d(d, lin, bar, h * 64, a, hh, bb);
+      else
+        tma_load_5d(d, img, bar, h * 64, b, a, hh, bb);
+    }
   }
 }
 
-template <int D>
+// Loads one 128-row query tile (all 64-element column blocks): 128 tokens from a (kind kLinear) or
+// an 8 x 16 grid rectangle (kind kRect, rows from a, columns from b).
+template <int D, bool kSplit>
+__device__ __forceinline__ void load_q128(uint8_t* dst, const CUtensorMap* lin, const CUtensorMap* img, uint64_t* bar,
+                                          int kind, int a, int b, int bh, int heads) {
+  if (!kSplit) {
+    load_tile<D>(dst, lin, img, bar, kind, a, b, bh);
+    return;
+  }
+  const int hh = bh % heads, bb = bh / heads;
+  #pragma unroll
+  for (int h = 0; h < D / 64; ++h) {
+    uint8_t* d = dst + h * kHalfBytes;
+    if (kind == kLinear)
+      tma_load_4d(d, lin, bar, h * 64, a, hh, bb);
+    else
+      tma_load_5d(d, img, bar, h * 64, b, a, hh, bb);
+  }
+}
+
+template <int D, bool kSplit>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_constant__ CUtensorMap tm_q_img,
                  const __grid_constant__ CUtensorMap tm_k_lin, const __grid_constant__ CUtensorMap tm_k_img,
@@ -241,15 +277,15 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
           const PairItem it = decode_pair(g, wq);
           mbar_arrive_expect_tx(&bars[L::bQFull], (it.validB ? 2 : 1) * L::kQTileBytes);
           if (it.is_text) {
-            load_tile<D>(smem + L::kQ, &tm_q_lin, &tm_q_img, &bars[L::bQFull], kLinear, it.q0, 0, it.bh);
+            load_q128<D, kSplit>(smem + L::kQ, &tm_q_lin, &tm_q_img, &bars[L::bQFull], kLinear, it.q0, 0, it.bh, g.heads);
             if (it.validB)
-              load_tile<D>(smem + L::kQ + L::kQTileBytes, &tm_q_lin, &tm_q_img, &bars[L::bQFull], kLinear,
-                           it.q0 + kTile, 0, it.bh);
+              load_q128<D, kSplit>(smem + L::kQ + L::kQTileBytes, &tm_q_lin, &tm_q_img, &bars[L::bQFull], kLinear,
+                           it.q0 + kTile, 0, it.bh, g.heads);
           } else {
-            load_tile<D>(smem + L::kQ, &tm_q_lin, &tm_q_img, &bars[L::bQFull], kRect, it.q0, it.x0, it.bh);
+            load_q128<D, kSplit>(smem + L::kQ, &tm_q_lin, &tm_q_img, &bars[L::bQFull], kRect, it.q0, it.x0, it.bh, g.heads);
             if (it.validB)
-              load_tile<D>(smem + L::kQ + L::kQTileBytes, &tm_q_lin, &tm_q_img, &bars[L::bQFull], kRect,
-                           it.q0 + kQH, it.x0, it.bh);
+              load_q128<D, kSplit>(smem + L::kQ + L::kQTileBytes, &tm_q_lin, &tm_q_img, &bars[L::bQFull], kRect,
+                           it.q0 + kQH, it.x0, it.bh, g.heads);
           }
           ++q_loads;
           wq += stride;
@@ -262,8 +298,8 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
             ring[Gk % kTileRing] = make_int4(tcur.kind | (tcur.flags << 4) | (next_in_pair ? 0 : (1 << 12)), tcur.a,
                                              tcur.b, itk.bh);
             mbar_arrive_expect_tx(&bars[L::bKFull + ks], L::kKVTileBytes);
-            load_kv64<D>(smem + L::kK + ks * L::kKVTileBytes, &tm_k_lin, &tm_k_img, &bars[L::bKFull + ks], tcur.kind,
-                         tcur.a, tcur.b, itk.bh);
+            load_kv64<D, kSplit>(smem + L::kK + ks * L::kKVTileBytes, &tm_k_lin, &tm_k_img, &bars[L::bKFull + ks], tcur.kind,
+                         tcur.a, tcur.b, itk.bh, g.heads);
             ++Gk;
             if (next_in_pair) {
               tcur = tnext;
@@ -286,8 +322,8 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
           if (mbar_test(&bars[L::bVEmpty + vs], ((Gv / kVStages) & 1) ^ 1)) {
             const int4 e = ring[Gv % kTileRing];
             mbar_arrive_expect_tx(&bars[L::bVFull + vs], L::kKVTileBytes);
-            load_kv64<D>(smem + L::kV + vs * L::kKVTileBytes, &tm_v_lin, &tm_v_img, &bars[L::bVFull + vs], e.x & 15,
-                         e.y, e.z, e.w);
+            load_kv64<D, kSplit>(smem + L::kV + vs * L::kKVTileBytes, &tm_v_lin, &tm_v_img, &bars[L::bVFull + vs], e.x & 15,
+                         e.y, e.z, e.w, g.heads);
             ++Gv;
             prog = true;
           }
@@ -521,9 +557,11 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
           }
           if (row_valid) p.ml[prow] = make_float2(m_used, l);
         } else {
-          const size_t orow = (size_t)it.bh * g.T + g.n_text + (size_t)yq * g.W + xq;
+          const size_t orow = (size_t)it.bh * g.T + g.n_text + (size_t)yq * g.W + xq;  // lse row
           const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-          __nv_bfloat16* dst = p.o + orow * D;
+          __nv_bfloat16* dst = p.o + (long long)(g.n_text + yq * g.W + xq) * p.o_st +
+                               (kSplit ? (long long)(it.bh / g.heads) * p.o_sb + (long long)(it.bh % g.heads) * p.o_sh
+                                       : (long long)it.bh * p.o_sh);
           #pragma unroll
           for (int c = 0; c < D / 32; c += 2) {
             uint32_t ov[2][32];
@@ -690,7 +728,7 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
 
 // Merges the split partials of the text rows: m = max_s m_s, l = sum_s 2^(m_s - m) l_s,
 // O = sum_s 2^(m_s - m) O_s / l, LSE = (m + log2 l) ln 2. One warp per text row.
-template <int D>
+template <int D, bool kSplit>
 __global__ void clear_fwd_combine_kernel(const FwdParams p) {
   const Geom& g = p.g;
   const int warps_per_block = blockDim.x / 32;
@@ -720,8 +758,10 @@ __global__ void clear_fwd_combine_kernel(const FwdParams p) {
     for (int e = 0; e < kPer; ++e) acc[e] += f * src[lane * kPer + e];
   }
   const float inv_l = 1.f / l;
-  const size_t orow = (size_t)bh * g.T + tq;
-  __nv_bfloat16* dst = p.o + orow * D + lane * kPer;
+  const size_t orow = (size_t)bh * g.T + tq;  // lse row
+  __nv_bfloat16* dst = p.o + (long long)tq * p.o_st + lane * kPer +
+                       (kSplit ? (long long)(bh / g.heads) * p.o_sb + (long long)(bh % g.heads) * p.o_sh
+                               : (long long)bh * p.o_sh);
   #pragma unroll
   for (int e = 0; e < kPer; ++e) dst[e] = __float2bfloat16_rn(acc[e] * inv_l);
   if (lane == 0) p.lse[orow] = (m + log2f(l)) * 0.69314718055994530942f;
