@@ -12,4 +12,6 @@ from .clear_attention import (  # noqa: F401
     window_pairs,
     kept_pairs,
     useful_flops_fwd,
+    clear_attention_stripe,
+    clear_text_rows_patch_average,
 )

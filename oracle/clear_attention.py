@@ -37,6 +37,11 @@ Revs Pre-Trained Diffusion Transformers Up"):
    image pair (i, j) kept iff |y_j - cy(y_i)| < r and |x_j - cx(x_i)| < r with the centre clamped,
    cy(y) = min(max(y, r-1), H-r) (likewise cx); it needs H, W >= 2r-1. window="shifted".
 
+7. Patch-parallel inference [pith review, "If this is right" (adjacent patches exchange only
+   O(r x W) boundary tokens) and "What carries the argument" (Eq. 7)]: `clear_attention_stripe`
+   gives one stripe's rows (image rows of its own grid rows, text rows over the keys it is given),
+   and `clear_text_rows_patch_average` the patch-wise average of Eq. 7 for the text rows.
+
 Readings where the pages leave a step open (each listed with its reason in the design notes):
 strict "<" in the radius test; image tokens in row-major order t = n_text + y*W + x; windows are
 clipped at the grid border (border queries see fewer keys); text queries attend to every token
@@ -249,3 +254,70 @@ def useful_flops_fwd(B: int, heads: int, n_text: int, H: int, W: int, r: int, d:
                      window: str = "circle") -> int:
     """Forward FLOPs on kept pairs only: 2*d for q.k plus 2*d for p*v, per kept (q, k) pair."""
     return 4 * d * B * heads * kept_pairs(n_text, H, W, r, window)
+
+
+# ----------------------------------------------------------------------------------------------
+# Patch-parallel inference: stripes of the grid and the patch-wise text approximation
+# ----------------------------------------------------------------------------------------------
+
+def clear_attention_stripe(q, k, v, n_text: int, H: int, W: int, r: int, q_row0: int, q_row1: int,
+                           key_row0: int, key_row1: int, text_keys: bool, scale=None, window: str = "circle"):
+    """Forward of one stripe of a patch-parallel split [pith review, "If this is right": adjacent
+    patches exchange only O(r x W) boundary tokens].
+
+    The problem (q, k, v, n_text, H, W) is the stripe itself: text tokens, then its H grid rows
+    (halo rows included). Image query rows [q_row0, q_row1) get the ordinary CLEAR rows of this
+    problem (mask of the stripe grid). Text query rows get one softmax over the keys the stripe
+    names: the text tokens if text_keys, and the image tokens of rows [key_row0, key_row1).
+    Returns (O_text [B, heads, n_text, d], LSE_text [B, heads, n_text],
+             O_img [B, heads, (q_row1 - q_row0) * W, d], LSE_img [B, heads, (q_row1 - q_row0) * W]).
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    B, Hh, T, d = q.shape
+    assert T == n_text + H * W
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    img_rows = list(range(n_text + q_row0 * W, n_text + q_row1 * W))
+    M_img = clear_mask(n_text, H, W, r, rows=img_rows, window=window)
+    keep_txt = np.zeros(T, dtype=bool)
+    if text_keys:
+        keep_txt[:n_text] = True
+    keep_txt[n_text + key_row0 * W:n_text + key_row1 * W] = True
+    Ot = np.empty((B, Hh, n_text, d))
+    Lt = np.empty((B, Hh, n_text))
+    Oi = np.empty((B, Hh, len(img_rows), d))
+    Li = np.empty((B, Hh, len(img_rows)))
+    for b in range(B):
+        for h in range(Hh):
+            if n_text:
+                S = (q[b, h, :n_text] @ k[b, h].T) * scale
+                P, lse = _masked_softmax_rows(S, np.broadcast_to(keep_txt, S.shape))
+                Ot[b, h], Lt[b, h] = P @ v[b, h], lse
+            S = (q[b, h, img_rows] @ k[b, h].T) * scale
+            P, lse = _masked_softmax_rows(S, M_img)
+            Oi[b, h], Li[b, h] = P @ v[b, h], lse
+    return Ot, Lt, Oi, Li
+
+
+def clear_text_rows_patch_average(q, k, v, n_text: int, H: int, W: int, row_bounds, scale=None):
+    """The patch-wise text approximation of Eq. 7 [pith review, "What carries the argument"]: text
+    query rows averaged over N patches, O_text = (1/N) sum_p softmax(Q_text K_p^T * scale) V_p.
+
+    Patch p holds grid rows [row_bounds[p], row_bounds[p+1]). The pages leave open whether K_p, V_p
+    hold the text tokens too (the review's referee comment on Eq. 7); read here as yes: each GPU of
+    a patch-parallel run holds the text tokens and its own image rows, so K_p, V_p are the text
+    tokens followed by patch p's image tokens. Returns O_text [B, heads, n_text, d] in float64.
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    B, Hh, T, d = q.shape
+    assert T == n_text + H * W and row_bounds[0] == 0 and row_bounds[-1] == H
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    n = len(row_bounds) - 1
+    O = np.zeros((B, Hh, n_text, d))
+    for p in range(n):
+        cols = list(range(n_text)) + list(range(n_text + row_bounds[p] * W, n_text + row_bounds[p + 1] * W))
+        for b in range(B):
+            for h in range(Hh):
+                S = (q[b, h, :n_text] @ k[b, h, cols].T) * scale
+                P, _ = _masked_softmax_rows(S, np.ones_like(S, dtype=bool))
+                O[b, h] += P @ v[b, h, cols]
+    return O / n
