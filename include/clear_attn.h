@@ -128,6 +128,58 @@ CLEAR_API clear_status_t clear_attn_fwd_strided(const clear_attn_params_t* param
                                                 const void* q, const void* k, const void* v, void* o, float* lse,
                                                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------------------------
+ * Patch-parallel inference (pith.science review of the CLEAR paper, "If this is right": adjacent
+ * patches exchange only O(r x W) boundary tokens; "What carries the argument": Eq. 7). Each GPU
+ * holds the text tokens and a stripe of image rows; a circular window of radius r reaches r - 1
+ * rows, so a stripe extended by r - 1 halo rows on each side holds every key its own image
+ * queries keep. Its text queries see a disjoint share of the keys, and the shares' text-row
+ * outputs are merged exactly (log-sum-exp weights) or by the paper's patch-wise average.
+ * --------------------------------------------------------------------------------------------- */
+
+/* A stripe of the problem given in clear_attn_params_t (whose H x W grid is the stripe,
+ * halo rows included). Rows are grid rows of the stripe. */
+typedef struct {
+  int q_row0, q_row1;     /* image query rows computed and written: [q_row0, q_row1), 0 <= q_row0 < q_row1 <= H */
+  int key_row0, key_row1; /* image keys the text query rows see: rows [key_row0, key_row1) (may be empty) */
+  int text_keys;          /* 1: text query rows also see the n_text text keys; 0: they do not */
+} clear_attn_stripe_t;
+
+/* Workspace bytes clear_attn_fwd_stripe needs (the text rows' split partials for this key set). */
+CLEAR_API size_t clear_attn_fwd_stripe_workspace_size(const clear_attn_params_t* params,
+                                                      const clear_attn_stripe_t* stripe, clear_status_t* status);
+
+/*
+ * Forward of one stripe. q, k, v, o: bf16 [B, heads, n_text + H*W, d] of the stripe (text tokens,
+ * then the stripe's rows, halos included); lse fp32 [B, heads, n_text + H*W]. Image query rows
+ * [q_row0, q_row1) attend, as in clear_attn_fwd, to all text keys and to the image keys of the
+ * stripe within their window (windows are clipped at the stripe's edges, which halos of r - 1 rows
+ * keep away from the computed rows). Text query rows attend to the keys the stripe names (see
+ * clear_attn_stripe_t) and are normalised over them, with their lse. Only these rows of o and lse
+ * are written; the halo rows are left untouched. The circle and square windows are offered; the
+ * shifted window is CLEAR_ERR_UNSUPPORTED (its centre clamping needs the whole grid). Invalid row
+ * ranges, or text rows left without any key, are CLEAR_ERR_INVALID_ARG. Otherwise as clear_attn_fwd.
+ */
+CLEAR_API clear_status_t clear_attn_fwd_stripe(const clear_attn_params_t* params, const clear_attn_stripe_t* stripe,
+                                               const void* q, const void* k, const void* v, void* o, float* lse,
+                                               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Merges the text query rows of n_parts stripe forwards. params gives B, heads, n_text, d (H, W, r
+ * are only checked). o_parts: bf16 [n_parts, B, heads, n_text, d] and lse_parts: fp32
+ * [n_parts, B, heads, n_text], part p's text rows (normalised over its keys, and their lse); o: bf16
+ * [B, heads, n_text, d], lse: fp32 [B, heads, n_text].
+ *   mode 0: exact. lse = log sum_p exp(lse_p), o = sum_p exp(lse_p - lse) o_p: the softmax over the
+ *           union of the parts' keys, which must be disjoint (text keys in exactly one part).
+ *   mode 1: Eq. 7 of the paper, o = (1/n_parts) sum_p o_p, each part's keys being the text tokens
+ *           and its own image rows; lse is written as in mode 0.
+ * A part without keys (lse_p = -inf) has weight 0 in mode 0. CLEAR_ERR_INVALID_ARG for n_parts
+ * outside [1, 4096], another mode, n_text = 0 or misaligned pointers.
+ */
+CLEAR_API clear_status_t clear_attn_text_merge(const clear_attn_params_t* params, int n_parts, int mode,
+                                               const void* o_parts, const float* lse_parts, void* o, float* lse,
+                                               void* stream);
+
 /*
  * Forward for callers that cannot allocate device memory: same inputs, outputs and results as
  * clear_attn_fwd (up to the summation order of the text rows), but no workspace argument. The
@@ -245,6 +297,17 @@ CLEAR_API clear_status_t clear_sched_forward_shape(const clear_attn_params_t* pa
  * holds real queries}. Writes at most max_tiles tiles; the total count goes to *n_tiles. */
 CLEAR_API clear_status_t clear_sched_item_tiles(const clear_attn_params_t* params, long long item,
                                       int* q_info, int* tiles, int max_tiles, int* n_tiles);
+
+/* clear_sched_forward_shape and clear_sched_item_tiles for the forward of a stripe (see
+ * clear_attn_fwd_stripe): image pairs cover query rows [q_row0, q_row1); text pairs visit the
+ * stripe's text-row key ranges (the text tokens if text_keys, then rows [key_row0, key_row1), each
+ * range in 64-token chunks from its own first token). */
+CLEAR_API clear_status_t clear_sched_stripe_forward_shape(const clear_attn_params_t* params,
+                                                          const clear_attn_stripe_t* stripe, long long* n_text_items,
+                                                          long long* n_image_items, int* splits, int* chunks_per_split);
+CLEAR_API clear_status_t clear_sched_stripe_item_tiles(const clear_attn_params_t* params,
+                                                       const clear_attn_stripe_t* stripe, long long item, int* q_info,
+                                                       int* tiles, int max_tiles, int* n_tiles);
 
 /* Useful (kept-pair) and executed (padded-tile) multiply-add pair counts of one forward call,
  * summed over B and heads: useful = number of ones in the mask; executed = 128 x 64 per tile

@@ -10,7 +10,7 @@ import importlib
 _EXPORTS = {
     "CLEAR_OK", "ClearError", "ClearParams", "LIB_PATH", "bwd_workspace_size", "clear_attn_bwd",
     "clear_attn_check", "clear_attn_fwd", "clear_attn_fwd_host", "clear_attn_fwd_strided", "ClearStrides",
-    "device_diag", "forward_shape",
+    "device_diag", "forward_shape", "ClearStripe", "make_stripe", "clear_attn_fwd_stripe", "clear_attn_text_merge",
     "fwd_host_workspace_size", "fwd_workspace_size", "header_functions", "item_tiles", "lib", "make_params",
     "pair_counts", "selftest_expiry", "status_string", "version",
 }

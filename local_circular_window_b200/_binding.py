@@ -32,6 +32,12 @@ class ClearStrides(ctypes.Structure):
                 ("o", ctypes.c_longlong * 3)]
 
 
+class ClearStripe(ctypes.Structure):
+    """Mirror of clear_attn_stripe_t."""
+    _fields_ = [("q_row0", ctypes.c_int), ("q_row1", ctypes.c_int), ("key_row0", ctypes.c_int),
+                ("key_row1", ctypes.c_int), ("text_keys", ctypes.c_int)]
+
+
 class ClearParams(ctypes.Structure):
     """Mirror of clear_attn_params_t."""
     _fields_ = [("B", ctypes.c_int), ("heads", ctypes.c_int), ("n_text", ctypes.c_int), ("H", ctypes.c_int),
@@ -68,6 +74,19 @@ _lib.clear_attn_fwd.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_
 _lib.clear_attn_fwd_strided.restype = _i
 _lib.clear_attn_fwd_strided.argtypes = [_P, ctypes.POINTER(ClearStrides), _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t,
                                         _vp]
+_S = ctypes.POINTER(ClearStripe)
+_lib.clear_attn_fwd_stripe_workspace_size.restype = ctypes.c_size_t
+_lib.clear_attn_fwd_stripe_workspace_size.argtypes = [_P, _S, ctypes.POINTER(_i)]
+_lib.clear_attn_fwd_stripe.restype = _i
+_lib.clear_attn_fwd_stripe.argtypes = [_P, _S, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+_lib.clear_attn_text_merge.restype = _i
+_lib.clear_attn_text_merge.argtypes = [_P, _i, _i, _vp, _vp, _vp, _vp, _vp]
+_lib.clear_sched_stripe_forward_shape.restype = _i
+_lib.clear_sched_stripe_forward_shape.argtypes = [_P, _S, ctypes.POINTER(_ll), ctypes.POINTER(_ll), ctypes.POINTER(_i),
+                                                  ctypes.POINTER(_i)]
+_lib.clear_sched_stripe_item_tiles.restype = _i
+_lib.clear_sched_stripe_item_tiles.argtypes = [_P, _S, _ll, ctypes.POINTER(_i), ctypes.POINTER(_i), _i,
+                                               ctypes.POINTER(_i)]
 _lib.clear_attn_fwd_noalloc.restype = _i
 _lib.clear_attn_fwd_noalloc.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.clear_attn_fwd_host_workspace_size.restype = ctypes.c_size_t
@@ -138,26 +157,36 @@ def bwd_workspace_size(p: ClearParams) -> int:
     return n
 
 
-def forward_shape(p: ClearParams):
+def make_stripe(q_row0: int, q_row1: int, key_row0: int, key_row1: int, text_keys: bool) -> ClearStripe:
+    return ClearStripe(q_row0, q_row1, key_row0, key_row1, 1 if text_keys else 0)
+
+
+def _stripe_ref(stripe):
+    return None if stripe is None else ctypes.byref(stripe)
+
+
+def forward_shape(p: ClearParams, stripe: ClearStripe = None):
+    """(text pairs, image pairs, text splits, chunks per split) of the forward (of a stripe if given)."""
     nt, ni, s, c = _ll(0), _ll(0), _i(0), _i(0)
-    st = _lib.clear_sched_forward_shape(ctypes.byref(p), ctypes.byref(nt), ctypes.byref(ni), ctypes.byref(s),
-                                        ctypes.byref(c))
+    st = _lib.clear_sched_stripe_forward_shape(ctypes.byref(p), _stripe_ref(stripe), ctypes.byref(nt),
+                                               ctypes.byref(ni), ctypes.byref(s), ctypes.byref(c))
     if st != CLEAR_OK:
-        raise ClearError(st, "clear_sched_forward_shape")
+        raise ClearError(st, "clear_sched_stripe_forward_shape")
     return nt.value, ni.value, s.value, c.value
 
 
-def item_tiles(p: ClearParams, item: int):
-    """(q_info, tiles) of one forward work item; tiles is a list of (kind, a, b, flags)."""
+def item_tiles(p: ClearParams, item: int, stripe: ClearStripe = None):
+    """(q_info, tiles) of one forward work item (of a stripe if given); tiles: (kind, a, b, flags)."""
     q = (_i * 5)()
     n = _i(0)
-    st = _lib.clear_sched_item_tiles(ctypes.byref(p), item, q, None, 0, ctypes.byref(n))
+    st = _lib.clear_sched_stripe_item_tiles(ctypes.byref(p), _stripe_ref(stripe), item, q, None, 0, ctypes.byref(n))
     if st != CLEAR_OK:
-        raise ClearError(st, "clear_sched_item_tiles")
+        raise ClearError(st, "clear_sched_stripe_item_tiles")
     buf = (_i * (4 * max(1, n.value)))()
-    st = _lib.clear_sched_item_tiles(ctypes.byref(p), item, q, buf, n.value, ctypes.byref(n))
+    st = _lib.clear_sched_stripe_item_tiles(ctypes.byref(p), _stripe_ref(stripe), item, q, buf, n.value,
+                                            ctypes.byref(n))
     if st != CLEAR_OK:
-        raise ClearError(st, "clear_sched_item_tiles")
+        raise ClearError(st, "clear_sched_stripe_item_tiles")
     tiles = [tuple(buf[4 * i:4 * i + 4]) for i in range(n.value)]
     return tuple(q), tiles
 
@@ -245,6 +274,60 @@ def clear_attn_fwd_strided(q, k, v, n_text: int, H: int, W: int, r: int, o=None,
                                          _stream_ptr(stream))
     if status != CLEAR_OK:
         raise ClearError(status, "clear_attn_fwd_strided")
+    return o, lse
+
+
+def clear_attn_fwd_stripe(q, k, v, n_text: int, H: int, W: int, r: int, stripe: ClearStripe, o=None, lse=None,
+                          workspace=None, stream=None, window="circle"):
+    """Forward of one stripe of a patch-parallel split through clear_attn_fwd_stripe: q, k, v are the
+    stripe's contiguous [B, heads, n_text + H*W, d] tensors (halo rows included). Only the text rows
+    and image rows [q_row0, q_row1) of o and lse are written. Returns (o, lse)."""
+    B, heads, T, d = q.shape
+    if T != n_text + H * W:
+        raise ValueError("T must equal n_text + H * W")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_qkv(name, t, q.shape)
+    p = make_params(B, heads, n_text, H, W, d, r, window)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, heads, T), dtype=torch.float32, device=q.device)
+    st = _i(0)
+    ws_bytes = _lib.clear_attn_fwd_stripe_workspace_size(ctypes.byref(p), ctypes.byref(stripe), ctypes.byref(st))
+    if st.value != CLEAR_OK:
+        raise ClearError(st.value, "clear_attn_fwd_stripe_workspace_size")
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    status = _lib.clear_attn_fwd_stripe(ctypes.byref(p), ctypes.byref(stripe), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                        _ptr(lse), _ptr(workspace),
+                                        0 if workspace is None else workspace.numel() * workspace.element_size(),
+                                        _stream_ptr(stream))
+    if status != CLEAR_OK:
+        raise ClearError(status, "clear_attn_fwd_stripe")
+    return o, lse
+
+
+TEXT_MERGE_MODES = {"exact": 0, "eq7": 1}
+
+
+def clear_attn_text_merge(o_parts, lse_parts, mode="exact", o=None, lse=None, stream=None):
+    """Merges the text rows of P stripes through clear_attn_text_merge. o_parts: bf16
+    [P, B, heads, n_text, d]; lse_parts: fp32 [P, B, heads, n_text] (contiguous CUDA tensors).
+    mode "exact" (disjoint key shares, log-sum-exp weights) or "eq7" (the paper's patch-wise
+    average). Returns (o [B, heads, n_text, d], lse [B, heads, n_text])."""
+    P, B, heads, n_text, d = o_parts.shape
+    if not (o_parts.is_cuda and o_parts.dtype == torch.bfloat16 and o_parts.is_contiguous()):
+        raise ValueError("o_parts must be a contiguous CUDA bf16 tensor")
+    if not (lse_parts.is_cuda and lse_parts.dtype == torch.float32 and lse_parts.is_contiguous()
+            and tuple(lse_parts.shape) == (P, B, heads, n_text)):
+        raise ValueError("lse_parts must be a contiguous CUDA fp32 tensor [P, B, heads, n_text]")
+    p = make_params(B, heads, n_text, 1, 1, d, 1)
+    o = torch.empty((B, heads, n_text, d), dtype=torch.bfloat16, device=o_parts.device) if o is None else o
+    lse = torch.empty((B, heads, n_text), dtype=torch.float32, device=o_parts.device) if lse is None else lse
+    status = _lib.clear_attn_text_merge(ctypes.byref(p), P, TEXT_MERGE_MODES[mode], _ptr(o_parts), _ptr(lse_parts),
+                                        _ptr(o), _ptr(lse), _stream_ptr(stream))
+    if status != CLEAR_OK:
+        raise ClearError(status, "clear_attn_text_merge")
     return o, lse
 
 

@@ -75,6 +75,29 @@ Checked check_params(const clear_attn_params_t* p) {
 
 bool aligned16(const void* ptr) { return ptr && (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
+// The forward restricted to a stripe of the grid (patch-parallel inference): image query rows
+// [q_row0, q_row1); text query rows see grid rows [key_row0, key_row1) and, if text_keys, the text
+// tokens. The shifted window is not offered (its centre clamping would need the whole grid).
+Checked check_stripe(const clear_attn_params_t* p, const clear_attn_stripe_t* s) {
+  Checked c = check_params(p);
+  if (c.st != CLEAR_OK) return c;
+  c.st = CLEAR_ERR_INVALID_ARG;
+  if (!s) return c;
+  if (p->window == kShifted) {
+    c.st = CLEAR_ERR_UNSUPPORTED;
+    return c;
+  }
+  if (s->q_row0 < 0 || s->q_row0 >= s->q_row1 || s->q_row1 > p->H) return c;
+  if (s->key_row0 < 0 || s->key_row0 > s->key_row1 || s->key_row1 > p->H) return c;
+  if (s->text_keys != 0 && s->text_keys != 1) return c;
+  if (p->n_text > 0 && !s->text_keys && s->key_row0 == s->key_row1) return c;  // text rows without keys
+  const int tk_lo = p->n_text + s->key_row0 * p->W, tk_hi = p->n_text + s->key_row1 * p->W;
+  set_text_key_ranges(&c.g, s->text_keys, tk_lo, tk_hi);
+  set_forward_work(&c.g, s->q_row0, s->q_row1);
+  c.st = CLEAR_OK;
+  return c;
+}
+
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct FwdWorkspace {
@@ -500,6 +523,51 @@ clear_status_t clear_attn_fwd_strided(const clear_attn_params_t* params, const c
   return run_fwd(c.g, st4, q, k, v, o, lse, workspace, static_cast<cudaStream_t>(stream));
 }
 
+size_t clear_attn_fwd_stripe_workspace_size(const clear_attn_params_t* params, const clear_attn_stripe_t* stripe,
+                                            clear_status_t* status) {
+  const Checked c = check_stripe(params, stripe);
+  if (status) *status = c.st;
+  if (c.st != CLEAR_OK) return 0;
+  return fwd_workspace_layout(c.g).total;
+}
+
+clear_status_t clear_attn_fwd_stripe(const clear_attn_params_t* params, const clear_attn_stripe_t* stripe,
+                                     const void* q, const void* k, const void* v, void* o, float* lse, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  const Checked c = check_stripe(params, stripe);
+  if (c.st != CLEAR_OK) return c.st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return CLEAR_ERR_INVALID_ARG;
+  const size_t need = fwd_workspace_layout(c.g).total;
+  if (need > 0 && (workspace_bytes < need || !aligned16(workspace))) return CLEAR_ERR_WORKSPACE;
+  const TensorStrides cs = contiguous_strides(c.g);
+  const TensorStrides st4[4] = {cs, cs, cs, cs};
+  return run_fwd(c.g, st4, q, k, v, o, lse, workspace, static_cast<cudaStream_t>(stream));
+}
+
+clear_status_t clear_attn_text_merge(const clear_attn_params_t* params, int n_parts, int mode, const void* o_parts,
+                                     const float* lse_parts, void* o, float* lse, void* stream) {
+  const Checked c = check_params(params);
+  if (c.st != CLEAR_OK) return c.st;
+  if (n_parts < 1 || n_parts > 4096 || (mode != 0 && mode != 1) || c.g.n_text == 0) return CLEAR_ERR_INVALID_ARG;
+  if (!aligned16(o_parts) || !aligned16(lse_parts) || !aligned16(o) || !aligned16(lse)) return CLEAR_ERR_INVALID_ARG;
+  const long long rows = (long long)c.g.BH * c.g.n_text;
+  if (rows * n_parts >= (1ll << 31)) return CLEAR_ERR_INVALID_ARG;
+  int num_sms = 0;
+  const clear_status_t st = check_device(&num_sms);
+  if (st != CLEAR_OK) return st;
+  const int wpb = 8;
+  const unsigned blocks = (unsigned)((rows + wpb - 1) / wpb);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const __nv_bfloat16* op = static_cast<const __nv_bfloat16*>(o_parts);
+  __nv_bfloat16* oo = static_cast<__nv_bfloat16*>(o);
+  if (c.g.d == 128)
+    clear_text_merge_kernel<128><<<blocks, wpb * 32, 0, s>>>((int)rows, n_parts, mode, op, lse_parts, oo, lse);
+  else
+    clear_text_merge_kernel<64><<<blocks, wpb * 32, 0, s>>>((int)rows, n_parts, mode, op, lse_parts, oo, lse);
+  return cudaGetLastError() == cudaSuccess ? CLEAR_OK : CLEAR_ERR_CUDA;
+}
+
 clear_status_t clear_attn_fwd_noalloc(const clear_attn_params_t* params, const void* q, const void* k,
                                       const void* v, void* o, float* lse, void* stream) {
   const Checked c = check_params(params);
@@ -674,7 +742,13 @@ clear_status_t clear_attn_selftest_expiry(int limit_ms, void* stream) {
 clear_status_t clear_sched_forward_shape(const clear_attn_params_t* params, long long* n_text_items,
                                          long long* n_image_items, int* splits,
                                          int* chunks_per_split) {
-  const Checked c = check_params(params);
+  return clear_sched_stripe_forward_shape(params, nullptr, n_text_items, n_image_items, splits, chunks_per_split);
+}
+
+clear_status_t clear_sched_stripe_forward_shape(const clear_attn_params_t* params, const clear_attn_stripe_t* stripe,
+                                                long long* n_text_items, long long* n_image_items, int* splits,
+                                                int* chunks_per_split) {
+  const Checked c = stripe ? check_stripe(params, stripe) : check_params(params);
   if (c.st != CLEAR_OK) return c.st;
   if (n_text_items) *n_text_items = c.g.n_txt_pairs;
   if (n_image_items) *n_image_items = c.g.n_img_pairs;
@@ -685,7 +759,12 @@ clear_status_t clear_sched_forward_shape(const clear_attn_params_t* params, long
 
 clear_status_t clear_sched_item_tiles(const clear_attn_params_t* params, long long item, int* q_info,
                                       int* tiles, int max_tiles, int* n_tiles) {
-  const Checked c = check_params(params);
+  return clear_sched_stripe_item_tiles(params, nullptr, item, q_info, tiles, max_tiles, n_tiles);
+}
+
+clear_status_t clear_sched_stripe_item_tiles(const clear_attn_params_t* params, const clear_attn_stripe_t* stripe,
+                                             long long item, int* q_info, int* tiles, int max_tiles, int* n_tiles) {
+  const Checked c = stripe ? check_stripe(params, stripe) : check_params(params);
   if (c.st != CLEAR_OK) return c.st;
   if (item < 0 || item >= c.g.n_txt_pairs + c.g.n_img_pairs || max_tiles < 0) return CLEAR_ERR_INVALID_ARG;
   const PairItem it = decode_pair(c.g, item);

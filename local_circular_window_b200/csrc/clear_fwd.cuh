@@ -609,7 +609,7 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
         } else {
           yq = it.q0 + half * kQH + (row >> 4);
           xq = it.x0 + (row & 15);
-          row_valid = (yq < g.H) && (xq < g.W);
+          row_valid = (yq < g.qy1) && (xq < g.W);
           yc = window_center(yq, g.r, g.H, g.window);
           xc = window_center(xq, g.r, g.W, g.window);
         }
@@ -765,6 +765,49 @@ __global__ void clear_fwd_combine_kernel(const FwdParams p) {
   #pragma unroll
   for (int e = 0; e < kPer; ++e) dst[e] = __float2bfloat16_rn(acc[e] * inv_l);
   if (lane == 0) p.lse[orow] = (m + log2f(l)) * 0.69314718055994530942f;
+}
+
+}  // namespace clear
+
+namespace clear {
+
+// Merges text query rows computed by P patches (parts) of a patch-parallel forward. Part p gives
+// its rows normalised over its own keys, O_p, and their log-sum-exp L_p (natural log).
+//   mode 0 (exact): L = log sum_p exp(L_p), O = sum_p exp(L_p - L) O_p: the softmax over the union
+//                   of the parts' key sets, which must be disjoint;
+//   mode 1 (the patch-wise average of Eq. 7 in the CLEAR paper): O = (1/P) sum_p O_p, each part's
+//                   keys being the text tokens plus that patch's image tokens; L is written as in
+//                   mode 0.
+// One warp per text row; parts with no key (L_p = -inf) carry no weight.
+template <int D>
+__global__ void clear_text_merge_kernel(int rows, int parts, int mode, const __nv_bfloat16* __restrict__ o_parts,
+                                        const float* __restrict__ lse_parts, __nv_bfloat16* __restrict__ o,
+                                        float* __restrict__ lse) {
+  const int warps_per_block = blockDim.x / 32;
+  const long long row = (long long)blockIdx.x * warps_per_block + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  float m = -INFINITY;
+  for (int pp = 0; pp < parts; ++pp) m = fmaxf(m, lse_parts[(size_t)pp * rows + row]);
+  constexpr int kPer = D / 32;
+  float acc[kPer];
+  #pragma unroll
+  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+  float z = 0.f;
+  for (int pp = 0; pp < parts; ++pp) {
+    const float lp = lse_parts[(size_t)pp * rows + row];
+    const float w = (lp == -INFINITY) ? 0.f : expf(lp - m);
+    z += w;
+    const float f = mode == 0 ? w : 1.f;
+    const __nv_bfloat16* src = o_parts + ((size_t)pp * rows + row) * D + lane * kPer;
+    #pragma unroll
+    for (int e = 0; e < kPer; ++e) acc[e] += f * __bfloat162float(src[e]);
+  }
+  const float inv = mode == 0 ? 1.f / z : 1.f / (float)parts;
+  __nv_bfloat16* dst = o + (size_t)row * D + lane * kPer;
+  #pragma unroll
+  for (int e = 0; e < kPer; ++e) dst[e] = __float2bfloat16_rn(acc[e] * inv);
+  if (lane == 0) lse[row] = m + logf(z);
 }
 
 }  // namespace clear

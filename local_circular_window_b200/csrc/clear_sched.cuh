@@ -76,12 +76,18 @@ struct Geom {
   long long n_txt_items, n_img_items;
   // Forward pairs: two query tiles share every key tile they visit (a 16 x 16 image block, or
   // two consecutive 128-row text tiles); key tiles are 64 keys.
-  int nqy2, nQ2;     // image blocks per (b, h): ceil(H/16) x ceil(W/16)
+  int nqy2, nQ2;     // image blocks per (b, h): ceil((qy1 - qy0)/16) x ceil(W/16)
   int nTq2;          // text tile pairs: ceil(nTq / 2)
-  int fnC;           // 64-key chunks over all T tokens
+  int fnC;           // 64-key chunks a text query row visits (both key ranges below)
   int fnTk;          // 64-key chunks over the text tokens
   int fS, fcps;      // forward text splits and 64-key chunks per split
   long long n_txt_pairs, n_img_pairs;
+  // Stripe mode (patch-parallel inference; the defaults are the whole problem): image query rows
+  // are rows [qy0, qy1) of the grid only, and text query rows see the keys of token ranges
+  // [ta_lo, ta_hi) and [tb_lo, tb_hi) (fnC = nca + ncb chunks of 64 keys, each range chunked from
+  // its own start).
+  int qy0, qy1;
+  int ta_lo, ta_hi, tb_lo, tb_hi, nca;
 };
 
 CLEAR_HD int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -133,6 +139,31 @@ CLEAR_HD void choose_splits(int nC, int target, int max_splits, int* S, int* cps
 constexpr int kSplitTargetChunks = 64;
 constexpr int kMaxSplits = 32;
 
+// Text rows' key ranges: the text tokens (when text_keys) and image tokens [tk_lo, tk_hi); one range
+// when they are adjacent.
+CLEAR_HD void set_text_key_ranges(Geom* g, int text_keys, int tk_lo, int tk_hi) {
+  if (text_keys && tk_lo == g->n_text) {
+    g->ta_lo = 0; g->ta_hi = tk_hi; g->tb_lo = g->tb_hi = tk_hi;
+  } else if (text_keys) {
+    g->ta_lo = 0; g->ta_hi = g->n_text; g->tb_lo = tk_lo; g->tb_hi = tk_hi;
+  } else {
+    g->ta_lo = tk_lo; g->ta_hi = tk_hi; g->tb_lo = g->tb_hi = tk_hi;
+  }
+  g->nca = cdiv(g->ta_hi - g->ta_lo, kFChunk);
+  g->fnC = g->nca + cdiv(g->tb_hi - g->tb_lo, kFChunk);
+}
+
+// Work counts that depend on the query rows and text-row key ranges (after set_text_key_ranges).
+CLEAR_HD void set_forward_work(Geom* g, int qy0, int qy1) {
+  g->qy0 = qy0;
+  g->qy1 = qy1;
+  g->nqy2 = cdiv(qy1 - qy0, 2 * kQH);
+  g->nQ2 = g->nqy2 * g->nqx;
+  choose_splits(g->fnC, 2 * kSplitTargetChunks, kMaxSplits, &g->fS, &g->fcps);
+  g->n_txt_pairs = (long long)g->BH * g->nTq2 * g->fS;
+  g->n_img_pairs = (long long)g->BH * g->nQ2;
+}
+
 CLEAR_HD Geom make_geom(int B, int heads, int n_text, int H, int W, int d, int r, int window = kCircle) {
   Geom g;
   g.B = B; g.heads = heads; g.n_text = n_text; g.H = H; g.W = W; g.d = d; g.r = r;
@@ -148,14 +179,10 @@ CLEAR_HD Geom make_geom(int B, int heads, int n_text, int H, int W, int d, int r
   choose_splits(g.nC, kSplitTargetChunks, kMaxSplits, &g.S, &g.cps);
   g.n_txt_items = (long long)g.BH * g.nTq * g.S;
   g.n_img_items = (long long)g.BH * g.nQ;
-  g.nqy2 = cdiv(H, 2 * kQH);
-  g.nQ2 = g.nqy2 * g.nqx;
   g.nTq2 = cdiv(g.nTq, 2);
-  g.fnC = cdiv(g.T, kFChunk);
   g.fnTk = cdiv(n_text, kFChunk);
-  choose_splits(g.fnC, 2 * kSplitTargetChunks, kMaxSplits, &g.fS, &g.fcps);
-  g.n_txt_pairs = (long long)g.BH * g.nTq2 * g.fS;
-  g.n_img_pairs = (long long)g.BH * g.nQ2;
+  set_text_key_ranges(&g, 1, n_text, g.T);
+  set_forward_work(&g, 0, H);
   return g;
 }
 
@@ -319,9 +346,9 @@ CLEAR_HD PairItem decode_pair(const Geom& g, long long w) {
     int blk = (int)(u % g.nQ2);
     it.is_text = 0;
     it.bh = (int)(u / g.nQ2);
-    it.q0 = (blk / g.nqx) * (2 * kQH);
+    it.q0 = g.qy0 + (blk / g.nqx) * (2 * kQH);
     it.x0 = (blk % g.nqx) * kQW;
-    it.validB = (it.q0 + kQH) < g.H;
+    it.validB = (it.q0 + kQH) < g.qy1;
     it.split = 0;
     it.c_begin = 0;
     it.c_end = 0;
@@ -337,6 +364,7 @@ struct PairKeyIter {
   const int* wtab;
   int wtab_n;
   int is_text, r, window, H, W, n_text, T, validB;
+  int ta_lo, ta_hi, tb_lo, tb_hi, nca;  // text rows' key ranges (chunk i < nca: range a)
   int y0, x0, xl;             // block origin, last column
   int yA0, yAl, yB0, yBl;     // half rows (clipped); B rows only if validB
   int ky_begin, ky_end;
@@ -349,6 +377,7 @@ struct PairKeyIter {
     wtab_n = table_n;
     is_text = it.is_text; r = g.r; window = g.window; H = g.H; W = g.W; n_text = g.n_text; T = g.T;
     validB = it.validB;
+    ta_lo = g.ta_lo; ta_hi = g.ta_hi; tb_lo = g.tb_lo; tb_hi = g.tb_hi; nca = g.nca;
     if (is_text) {
       lin_next = it.c_begin;
       lin_end = it.c_end;
@@ -361,8 +390,8 @@ struct PairKeyIter {
     lin_end = g.fnTk;
     y0 = it.q0; x0 = it.x0;
     xl = imin(x0 + kQW - 1, W - 1);
-    yA0 = y0; yAl = imin(y0 + kQH - 1, H - 1);
-    yB0 = y0 + kQH; yBl = imin(y0 + 2 * kQH - 1, H - 1);
+    yA0 = y0; yAl = imin(y0 + kQH - 1, g.qy1 - 1);
+    yB0 = y0 + kQH; yBl = imin(y0 + 2 * kQH - 1, g.qy1 - 1);
     if (window == kShifted) {  // clamping is monotone: a query rectangle maps to a centre rectangle
       x0 = window_center(x0, r, W, window); xl = window_center(xl, r, W, window);
       yA0 = window_center(yA0, r, H, window); yAl = window_center(yAl, r, H, window);
@@ -415,8 +444,13 @@ struct PairKeyIter {
 
   CLEAR_HD bool next(KeyTile* t) {
     if (lin_next < lin_end) {
-      const int a = lin_next * kFChunk;
-      const int lim = is_text ? T : n_text;
+      // Image blocks: the text keys from token 0. Text rows: chunk i of range a, or of range b.
+      int a = lin_next * kFChunk, lim = n_text;
+      if (is_text) {
+        const bool in_a = lin_next < nca;
+        a = in_a ? ta_lo + lin_next * kFChunk : tb_lo + (lin_next - nca) * kFChunk;
+        lim = in_a ? ta_hi : tb_hi;
+      }
       t->kind = kLinear;
       t->a = a;
       t->b = imin(kFChunk, lim - a);

@@ -30,7 +30,7 @@ def _rank_main(rank, world, port, out):
 
 def test_whole_job_takes_slowest_rank_and_sums_work():
     world = 2
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True)
     for rank in range(world):
         ms, value = out[rank]
