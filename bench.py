@@ -391,10 +391,12 @@ def run_clear(args):
     configs = None
     if not args.no_configs:
         configs = {}
-        for name in FORWARD_CONFIGS:
-            if name == wl.name:
-                continue
-            configs[name] = time_forward_config(L, WORKLOADS[name], peak, stream, seed=3000 + rank)
+        with ClockSampler(local) as cfg_clk:
+            for name in FORWARD_CONFIGS:
+                if name == wl.name:
+                    continue
+                configs[name] = time_forward_config(L, WORKLOADS[name], peak, stream, seed=3000 + rank)
+        configs["clocks"] = cfg_clk.summary()
         torch.cuda.empty_cache()
 
     cpu = None

@@ -181,6 +181,31 @@ CLEAR_API clear_status_t clear_attn_text_merge(const clear_attn_params_t* params
                                                void* stream);
 
 /*
+ * Mixed-resolution batch forward: n_items problems of their own (n_text, H, W) in ONE launch (their
+ * pairs form one work list), e.g. a batch holding 1024^2 and 2048^2 images at once. Each item is the
+ * CLEAR forward of clear_attn_fwd (pith.science review of "CLEAR: Conv-Like Linearization Revs
+ * Pre-Trained Diffusion Transformers Up", "Core claim": text rows and text keys global, image keys
+ * within radius r on the item's own grid); items never attend to each other.
+ *   params: heads, d, r and window are shared by every item; B, n_text, H and W are not used.
+ *   item_shapes: host int[3 * n_items], item i = (n_text_i, H_i, W_i), each checked as clear_attn_fwd
+ *     checks its params (n_items in [1, 4096]).
+ *   q, k, v, o: bf16 [heads, T_total, d] with T_total = sum_i (n_text_i + H_i * W_i); item i's tokens
+ *     (text first, then its grid row-major) start at token sum_{j<i} T_j. lse: fp32 [heads, T_total].
+ *   workspace: device memory of clear_attn_fwd_varlen_workspace_size bytes, 256-byte aligned; the
+ *     call copies the items' geometry and tensor maps into it (an asynchronous copy on `stream`)
+ *     before launching, so a workspace must not be shared by calls that overlap on the GPU.
+ * The radius is clamped once, to the largest full-grid radius among the items (an item whose own
+ * grid is smaller keeps all its pairs either way). Results equal clear_attn_fwd on each item alone.
+ * CLEAR_ERR_INVALID_ARG for a bad item or count, misaligned pointers or T_total > 2^30;
+ * CLEAR_ERR_WORKSPACE for a short or misaligned workspace.
+ */
+CLEAR_API size_t clear_attn_fwd_varlen_workspace_size(const clear_attn_params_t* params, int n_items,
+                                                      const int* item_shapes, clear_status_t* status);
+CLEAR_API clear_status_t clear_attn_fwd_varlen(const clear_attn_params_t* params, int n_items, const int* item_shapes,
+                                               const void* q, const void* k, const void* v, void* o, float* lse,
+                                               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Forward for callers that cannot allocate device memory: same inputs, outputs and results as
  * clear_attn_fwd (up to the summation order of the text rows), but no workspace argument. The
  * paper has no counterpart; this entry point exists for integration. Some callers cannot call

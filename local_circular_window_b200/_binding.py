@@ -79,6 +79,10 @@ _lib.clear_attn_fwd_stripe_workspace_size.restype = ctypes.c_size_t
 _lib.clear_attn_fwd_stripe_workspace_size.argtypes = [_P, _S, ctypes.POINTER(_i)]
 _lib.clear_attn_fwd_stripe.restype = _i
 _lib.clear_attn_fwd_stripe.argtypes = [_P, _S, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+_lib.clear_attn_fwd_varlen_workspace_size.restype = ctypes.c_size_t
+_lib.clear_attn_fwd_varlen_workspace_size.argtypes = [_P, _i, ctypes.POINTER(_i), ctypes.POINTER(_i)]
+_lib.clear_attn_fwd_varlen.restype = _i
+_lib.clear_attn_fwd_varlen.argtypes = [_P, _i, ctypes.POINTER(_i), _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 _lib.clear_attn_text_merge.restype = _i
 _lib.clear_attn_text_merge.argtypes = [_P, _i, _i, _vp, _vp, _vp, _vp, _vp]
 _lib.clear_sched_stripe_forward_shape.restype = _i
@@ -304,6 +308,58 @@ def clear_attn_fwd_stripe(q, k, v, n_text: int, H: int, W: int, r: int, stripe: 
                                         _stream_ptr(stream))
     if status != CLEAR_OK:
         raise ClearError(status, "clear_attn_fwd_stripe")
+    return o, lse
+
+
+def _item_array(items):
+    flat = [int(x) for it in items for x in it]
+    if not items or any(len(it) != 3 for it in items):
+        raise ValueError("items must be a non-empty sequence of (n_text, H, W)")
+    return (_i * len(flat))(*flat)
+
+
+def varlen_tokens(items):
+    """Token count of a packed mixed-resolution batch and each item's first token."""
+    starts, t = [], 0
+    for n_text, H, W in items:
+        starts.append(t)
+        t += n_text + H * W
+    return t, starts
+
+
+def varlen_workspace_size(heads: int, d: int, r: int, items, window="circle") -> int:
+    p = make_params(1, heads, 0, 1, 1, d, r, window)
+    st = _i(0)
+    n = _lib.clear_attn_fwd_varlen_workspace_size(ctypes.byref(p), len(items), _item_array(items), ctypes.byref(st))
+    if st.value != CLEAR_OK:
+        raise ClearError(st.value, "clear_attn_fwd_varlen_workspace_size")
+    return n
+
+
+def clear_attn_fwd_varlen(q, k, v, items, r: int, o=None, lse=None, workspace=None, stream=None, window="circle"):
+    """Mixed-resolution batch forward through clear_attn_fwd_varlen: one launch over items of their
+    own (n_text, H, W). q, k, v: contiguous bf16 CUDA [heads, T_total, d], the items packed along the
+    token axis in order (varlen_tokens gives each item's first token). Returns (o, lse) with o like q
+    and lse fp32 [heads, T_total]."""
+    heads, T, d = q.shape
+    total, _ = varlen_tokens(items)
+    if T != total:
+        raise ValueError("q's token axis must hold every item's n_text + H * W tokens")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_qkv(name, t, q.shape)
+    p = make_params(1, heads, 0, 1, 1, d, r, window)
+    shapes = _item_array(items)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((heads, T), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(varlen_workspace_size(heads, d, r, items, window), dtype=torch.uint8, device=q.device)
+    status = _lib.clear_attn_fwd_varlen(ctypes.byref(p), len(items), shapes, _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                        _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                        _stream_ptr(stream))
+    if status != CLEAR_OK:
+        raise ClearError(status, "clear_attn_fwd_varlen")
     return o, lse
 
 

@@ -9,6 +9,7 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <vector>
 
 #include "clear_attn.h"
 #include "clear_bwd.cuh"
@@ -279,11 +280,11 @@ clear_status_t launch_fwd(const Geom& g, const QKVMaps& m, void* o, const Tensor
   p.wide_part = (reinterpret_cast<uintptr_t>(p.opart) & 31u) == 0;
   p.ml = g.n_text ? reinterpret_cast<float2*>(static_cast<char*>(ws) + wl.ml_off) : nullptr;
   p.n_work = g.n_txt_pairs + g.n_img_pairs;
-  if (cudaFuncSetAttribute(clear_fwd_kernel<D, kSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(clear_fwd_kernel<D, kSplit, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smem_bytes) != cudaSuccess)
     return CLEAR_ERR_CUDA;
   const long long grid = p.n_work < num_sms ? p.n_work : num_sms;
-  clear_fwd_kernel<D, kSplit><<<(unsigned)grid, kFwdThreads, smem_bytes, stream>>>(
+  clear_fwd_kernel<D, kSplit, false><<<(unsigned)grid, kFwdThreads, smem_bytes, stream>>>(
       m.q_lin, m.q_img, m.k_lin, m.k_img, m.v_lin, m.v_img, p);
   if (cudaGetLastError() != cudaSuccess) return CLEAR_ERR_CUDA;
   if (g.n_text > 0) {
@@ -455,6 +456,158 @@ clear_status_t run_fwd(const Geom& g, const TensorStrides* st4, const void* q, c
                     : launch_fwd<64, false>(g, maps, o, st4[3], lse, workspace, num_sms, s);
 }
 
+// ------------------------------------------------------------------------------------------------
+// Mixed-resolution batch: items of their own (n_text, H, W) packed along the token axis of
+// [heads, tok_total, d] tensors, all of them in one forward launch.
+// ------------------------------------------------------------------------------------------------
+constexpr int kMaxVarlenItems = 4096;
+
+struct VarlenPlan {
+  std::vector<Geom> items;
+  std::vector<long long> wbound;  // 2 * n + 1 pair bounds (text pairs of each item, then image pairs, then the total)
+  Geom shared;                    // what the items share, with the largest H (the half-width table's size)
+  long long n_pairs = 0, text_rows = 0, part_rows = 0;
+  size_t maps_off = 0, bound_off = 0, opart_off = 0, ml_off = 0, staged = 0, total = 0;
+};
+
+clear_status_t plan_varlen(const clear_attn_params_t* p, int n_items, const int* shapes, VarlenPlan* v) {
+  if (!p || !shapes || n_items < 1 || n_items > kMaxVarlenItems) return CLEAR_ERR_INVALID_ARG;
+  // One radius for every item: the request clamped to the largest full-grid radius among them. An
+  // item whose own full radius is smaller keeps all its pairs either way.
+  int rmax_full = 1;
+  long long tok = 0;
+  int max_h = 1;
+  for (int i = 0; i < n_items; ++i) {
+    clear_attn_params_t ip = *p;
+    ip.B = 1;
+    ip.n_text = shapes[3 * i];
+    ip.H = shapes[3 * i + 1];
+    ip.W = shapes[3 * i + 2];
+    const Checked c = check_params(&ip);
+    if (c.st != CLEAR_OK) return c.st;
+    if (p->window != kShifted) {
+      const int rf = full_radius(ip.H, ip.W, p->window);
+      rmax_full = rf > rmax_full ? rf : rmax_full;
+    }
+    tok += c.g.T;
+    max_h = ip.H > max_h ? ip.H : max_h;
+  }
+  if (tok > (1ll << 30) || (long long)p->heads * tok * p->d >= (1ll << 40)) return CLEAR_ERR_INVALID_ARG;
+  const int r = p->window == kShifted ? p->r : (p->r < rmax_full ? p->r : rmax_full);
+  if (hw_table_size(r, max_h) > kMaxHwTable) return CLEAR_ERR_UNSUPPORTED;
+  v->items.resize(n_items);
+  v->wbound.assign(2 * (size_t)n_items + 1, 0);
+  long long t0 = 0, part = 0, crow = 0, wt = 0;
+  for (int i = 0; i < n_items; ++i) {
+    Geom g = make_geom(1, p->heads, shapes[3 * i], shapes[3 * i + 1], shapes[3 * i + 2], p->d, r, p->window);
+    g.t0 = (int)t0;
+    g.tok_total = tok;
+    g.part_row0 = part;
+    g.crow0 = crow;
+    t0 += g.T;
+    part += (long long)g.fS * g.BH * g.n_text;
+    crow += (long long)g.BH * g.n_text;
+    v->wbound[i] = wt;
+    wt += g.n_txt_pairs;
+    v->items[i] = g;
+  }
+  for (int i = 0; i < n_items; ++i) {
+    v->wbound[n_items + i] = wt;
+    wt += v->items[i].n_img_pairs;
+  }
+  v->wbound[2 * n_items] = wt;
+  v->n_pairs = wt;
+  v->text_rows = crow;
+  v->part_rows = part;
+  v->shared = make_geom(1, p->heads, 0, max_h, 1, p->d, r, p->window);
+  v->shared.tok_total = tok;
+  // Workspace: the item geometries, the image tensor maps (q, k, v per item), the pair bounds (all
+  // three copied from the host before the launch), then the text rows' split partials.
+  v->maps_off = align256(sizeof(Geom) * n_items);
+  v->bound_off = align256(v->maps_off + sizeof(CUtensorMap) * 3 * (size_t)n_items);
+  v->staged = v->bound_off + sizeof(long long) * v->wbound.size();
+  v->opart_off = align256(v->staged);
+  v->ml_off = align256(v->opart_off + (size_t)part * p->d * sizeof(float));
+  v->total = align256(v->ml_off + (size_t)part * sizeof(float2));
+  return CLEAR_OK;
+}
+
+template <int D>
+clear_status_t launch_fwd_varlen(const VarlenPlan& v, const QKVMaps& maps, void* o, float* lse, void* ws, int num_sms,
+                                 cudaStream_t stream) {
+  using L = FwdLayout<D>;
+  const Geom& g = v.shared;
+  const int smem_bytes = L::alloc_bytes(hw_table_size(g.r, g.H));
+  if (smem_bytes > 232448) return CLEAR_ERR_UNSUPPORTED;
+  FwdParams p{};
+  p.g = g;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.o_sh = g.tok_total * D;
+  p.o_sb = (long long)g.heads * p.o_sh;
+  p.o_st = D;
+  p.lse = lse;
+  char* w = static_cast<char*>(ws);
+  p.opart = v.part_rows ? reinterpret_cast<float*>(w + v.opart_off) : nullptr;
+  p.ml = v.part_rows ? reinterpret_cast<float2*>(w + v.ml_off) : nullptr;
+  p.wide_o = (reinterpret_cast<uintptr_t>(o) & 31u) == 0;
+  p.wide_part = (reinterpret_cast<uintptr_t>(p.opart) & 31u) == 0;
+  p.n_work = v.n_pairs;
+  p.items = reinterpret_cast<const Geom*>(w);
+  p.item_maps = reinterpret_cast<const CUtensorMap*>(w + v.maps_off);
+  p.wbound = reinterpret_cast<const long long*>(w + v.bound_off);
+  p.n_items = (int)v.items.size();
+  if (cudaFuncSetAttribute(clear_fwd_kernel<D, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem_bytes) != cudaSuccess)
+    return CLEAR_ERR_CUDA;
+  const long long grid = p.n_work < num_sms ? p.n_work : num_sms;
+  clear_fwd_kernel<D, false, true><<<(unsigned)grid, kFwdThreads, smem_bytes, stream>>>(
+      maps.q_lin, maps.q_img, maps.k_lin, maps.k_img, maps.v_lin, maps.v_img, p);
+  if (cudaGetLastError() != cudaSuccess) return CLEAR_ERR_CUDA;
+  if (v.text_rows > 0) {
+    const int wpb = 8;
+    clear_fwd_combine_varlen_kernel<D><<<(unsigned)((v.text_rows + wpb - 1) / wpb), wpb * 32, 0, stream>>>(p, v.text_rows);
+    if (cudaGetLastError() != cudaSuccess) return CLEAR_ERR_CUDA;
+  }
+  return CLEAR_OK;
+}
+
+clear_status_t run_fwd_varlen(const VarlenPlan& v, const void* q, const void* k, const void* v_ptr, void* o,
+                              float* lse, void* workspace, cudaStream_t s) {
+  int num_sms = 0;
+  const clear_status_t st = check_device(&num_sms);
+  if (st != CLEAR_OK) return st;
+  const Geom& g = v.shared;
+  // Token-axis (linear) maps over the whole batch: a problem of one grid row of tok_total tokens.
+  const Geom gl = make_geom(1, g.heads, 0, 1, (int)g.tok_total, g.d, 1, kCircle);
+  const TensorStrides ts = contiguous_strides(gl);
+  const TensorStrides st4[4] = {ts, ts, ts, ts};
+  QKVMaps maps;
+  if (!make_fwd_maps(&maps, q, k, v_ptr, st4, gl, false)) return CLEAR_ERR_CUDA;
+  // Staged part of the workspace: geometries, per-item image maps, pair bounds.
+  const size_t n = v.items.size();
+  std::vector<unsigned char> host(v.staged, 0);
+  std::memcpy(host.data(), v.items.data(), sizeof(Geom) * n);
+  CUtensorMap* hm = reinterpret_cast<CUtensorMap*>(host.data() + v.maps_off);
+  const void* bases[3] = {q, k, v_ptr};
+  const int img_rows[3] = {kQH, kFKH, kFKH};
+  const int lin_rows[3] = {kTile, kFChunk, kFChunk};
+  for (size_t i = 0; i < n; ++i) {
+    const Geom& gi = v.items[i];
+    for (int t = 0; t < 3; ++t) {
+      CUtensorMap lin_unused;
+      const char* base = static_cast<const char*>(bases[t]) + (size_t)gi.t0 * g.d * 2;
+      if (!make_fwd_tensor_maps(&lin_unused, &hm[3 * i + t], base, ts, gi, lin_rows[t], img_rows[t], false))
+        return CLEAR_ERR_CUDA;
+    }
+  }
+  std::memcpy(host.data() + v.bound_off, v.wbound.data(), sizeof(long long) * v.wbound.size());
+  if (cudaMemcpyAsync(workspace, host.data(), host.size(), cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return CLEAR_ERR_CUDA;
+  return g.d == 128 ? launch_fwd_varlen<128>(v, maps, o, lse, workspace, num_sms, s)
+                    : launch_fwd_varlen<64>(v, maps, o, lse, workspace, num_sms, s);
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------------------------------------
@@ -543,6 +696,27 @@ clear_status_t clear_attn_fwd_stripe(const clear_attn_params_t* params, const cl
   const TensorStrides cs = contiguous_strides(c.g);
   const TensorStrides st4[4] = {cs, cs, cs, cs};
   return run_fwd(c.g, st4, q, k, v, o, lse, workspace, static_cast<cudaStream_t>(stream));
+}
+
+size_t clear_attn_fwd_varlen_workspace_size(const clear_attn_params_t* params, int n_items, const int* item_shapes,
+                                            clear_status_t* status) {
+  VarlenPlan v;
+  const clear_status_t st = plan_varlen(params, n_items, item_shapes, &v);
+  if (status) *status = st;
+  return st == CLEAR_OK ? v.total : 0;
+}
+
+clear_status_t clear_attn_fwd_varlen(const clear_attn_params_t* params, int n_items, const int* item_shapes,
+                                     const void* q, const void* k, const void* v, void* o, float* lse, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  VarlenPlan plan;
+  const clear_status_t st = plan_varlen(params, n_items, item_shapes, &plan);
+  if (st != CLEAR_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return CLEAR_ERR_INVALID_ARG;
+  if (workspace_bytes < plan.total || !workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return CLEAR_ERR_WORKSPACE;
+  return run_fwd_varlen(plan, q, k, v, o, lse, workspace, static_cast<cudaStream_t>(stream));
 }
 
 clear_status_t clear_attn_text_merge(const clear_attn_params_t* params, int n_parts, int mode, const void* o_parts,

@@ -66,7 +66,30 @@ struct FwdParams {
   float2* ml;                 // [fS, BH, n_text] (running max in scaled log2 units, sum)
   long long n_work;           // pair items
   int wide_o, wide_part;      // o / opart are 32-byte aligned: the epilogue may store 32 bytes at once
+  // Mixed-resolution batch (the kernel's kVar parameter): per-item geometry (Geom::t0, tok_total,
+  // part_row0 and crow0 place the item in the packed tensors) and image tensor maps (q, k, v for
+  // each item), in device memory; the batch's pairs are every item's text pairs, then every item's
+  // image pairs: wbound[i] is the first pair of item i's text pairs, wbound[n_items + i] of its
+  // image pairs, wbound[2 * n_items] the total. p.g then carries what the items share (heads, d,
+  // r, window) and the largest H (the half-width table's size).
+  const Geom* items;
+  const CUtensorMap* item_maps;
+  const long long* wbound;
+  int n_items;
 };
+
+// Item of pair w of a mixed-resolution batch, and w's index among the item's own pairs.
+__device__ __forceinline__ int locate_pair(const FwdParams& p, long long w, long long* local) {
+  int lo = 0, hi = 2 * p.n_items - 1;  // last k with wbound[k] <= w
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(p.wbound + mid) <= w) lo = mid; else hi = mid - 1;
+  }
+  const int item = lo < p.n_items ? lo : lo - p.n_items;
+  const long long off = w - __ldg(p.wbound + lo);
+  *local = lo < p.n_items ? off : p.items[item].n_txt_pairs + off;
+  return item;
+}
 
 // Packed fp32 pairs (one 64-bit register, low word first): fma.rn.f32x2 / add.rn.f32x2 do two
 // correctly rounded fp32 operations per instruction, with the same results as two fmaf / fadd.
@@ -186,7 +209,7 @@ __device__ __forceinline__ void load_q128(uint8_t* dst, const CUtensorMap* lin, 
   }
 }
 
-template <int D, bool kSplit>
+template <int D, bool kSplit, bool kVar>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_constant__ CUtensorMap tm_q_img,
                  const __grid_constant__ CUtensorMap tm_k_lin, const __grid_constant__ CUtensorMap tm_k_img,
@@ -262,29 +285,40 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
       PairKeyIter kik;
       KeyTile tcur{}, tnext{};
       bool kval = wk < p.n_work, next_in_pair = false;
-      if (kval) {
-        itk = decode_pair(g, wk);
-        kik.init(g, itk, wtab, wtn);
+      int ik = 0;  // the K stream's batch item (mixed-resolution batches)
+      auto start_k_pair = [&]() {
+        long long lw = wk;
+        if constexpr (kVar) ik = locate_pair(p, wk, &lw);
+        const Geom& gk = kVar ? p.items[ik] : g;
+        itk = decode_pair(gk, lw);
+        kik.init(gk, itk, wtab, wtn);
         kik.next(&tcur);
         next_in_pair = kik.next(&tnext);
-      }
+      };
+      if (kval) start_k_pair();
       uint32_t Gk = 0, Gv = 0;
       PollWatchdog wd;
       wd.start();
       while (wq < p.n_work || kval || Gv < Gk) {
         bool prog = false;
         if (wq < p.n_work && (q_loads == 0 || mbar_test(&bars[L::bQEmpty], (q_loads - 1) & 1))) {
-          const PairItem it = decode_pair(g, wq);
+          long long lw = wq;
+          int iq = 0;
+          if constexpr (kVar) iq = locate_pair(p, wq, &lw);
+          const Geom& gq = kVar ? p.items[iq] : g;
+          const CUtensorMap* qimg = kVar ? p.item_maps + 3 * iq : &tm_q_img;
+          const int t0 = kVar ? gq.t0 : 0;  // the item's first token in the packed batch
+          const PairItem it = decode_pair(gq, lw);
           mbar_arrive_expect_tx(&bars[L::bQFull], (it.validB ? 2 : 1) * L::kQTileBytes);
           if (it.is_text) {
-            load_q128<D, kSplit>(smem + L::kQ, &tm_q_lin, &tm_q_img, &bars[L::bQFull], kLinear, it.q0, 0, it.bh, g.heads);
+            load_q128<D, kSplit>(smem + L::kQ, &tm_q_lin, qimg, &bars[L::bQFull], kLinear, t0 + it.q0, 0, it.bh, g.heads);
             if (it.validB)
-              load_q128<D, kSplit>(smem + L::kQ + L::kQTileBytes, &tm_q_lin, &tm_q_img, &bars[L::bQFull], kLinear,
-                           it.q0 + kTile, 0, it.bh, g.heads);
+              load_q128<D, kSplit>(smem + L::kQ + L::kQTileBytes, &tm_q_lin, qimg, &bars[L::bQFull], kLinear,
+                           t0 + it.q0 + kTile, 0, it.bh, g.heads);
           } else {
-            load_q128<D, kSplit>(smem + L::kQ, &tm_q_lin, &tm_q_img, &bars[L::bQFull], kRect, it.q0, it.x0, it.bh, g.heads);
+            load_q128<D, kSplit>(smem + L::kQ, &tm_q_lin, qimg, &bars[L::bQFull], kRect, it.q0, it.x0, it.bh, g.heads);
             if (it.validB)
-              load_q128<D, kSplit>(smem + L::kQ + L::kQTileBytes, &tm_q_lin, &tm_q_img, &bars[L::bQFull], kRect,
+              load_q128<D, kSplit>(smem + L::kQ + L::kQTileBytes, &tm_q_lin, qimg, &bars[L::bQFull], kRect,
                            it.q0 + kQH, it.x0, it.bh, g.heads);
           }
           ++q_loads;
@@ -295,11 +329,13 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
           const uint32_t ks = Gk % kKStages;
           if (mbar_test(&bars[L::bKEmpty + ks], ((Gk / kKStages) & 1) ^ 1)) {
             // Publish the descriptor before the load: the K barrier's completion makes it visible.
-            ring[Gk % kTileRing] = make_int4(tcur.kind | (tcur.flags << 4) | (next_in_pair ? 0 : (1 << 12)), tcur.a,
-                                             tcur.b, itk.bh);
+            // Linear tiles carry item-local tokens; bits 16+ of the first word hold the batch item.
+            ring[Gk % kTileRing] = make_int4(tcur.kind | (tcur.flags << 4) | (next_in_pair ? 0 : (1 << 12)) | (ik << 16),
+                                             tcur.a, tcur.b, itk.bh);
             mbar_arrive_expect_tx(&bars[L::bKFull + ks], L::kKVTileBytes);
-            load_kv64<D, kSplit>(smem + L::kK + ks * L::kKVTileBytes, &tm_k_lin, &tm_k_img, &bars[L::bKFull + ks], tcur.kind,
-                         tcur.a, tcur.b, itk.bh, g.heads);
+            load_kv64<D, kSplit>(smem + L::kK + ks * L::kKVTileBytes, &tm_k_lin,
+                                 kVar ? p.item_maps + 3 * ik + 1 : &tm_k_img, &bars[L::bKFull + ks], tcur.kind,
+                                 tcur.kind == kLinear && kVar ? p.items[ik].t0 + tcur.a : tcur.a, tcur.b, itk.bh, g.heads);
             ++Gk;
             if (next_in_pair) {
               tcur = tnext;
@@ -307,12 +343,7 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
             } else {
               wk += stride;
               kval = wk < p.n_work;
-              if (kval) {
-                itk = decode_pair(g, wk);
-                kik.init(g, itk, wtab, wtn);
-                kik.next(&tcur);
-                next_in_pair = kik.next(&tnext);
-              }
+              if (kval) start_k_pair();
             }
             prog = true;
           }
@@ -321,9 +352,11 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
           const uint32_t vs = Gv % kVStages;
           if (mbar_test(&bars[L::bVEmpty + vs], ((Gv / kVStages) & 1) ^ 1)) {
             const int4 e = ring[Gv % kTileRing];
+            const int iv = e.x >> 16;
             mbar_arrive_expect_tx(&bars[L::bVFull + vs], L::kKVTileBytes);
-            load_kv64<D, kSplit>(smem + L::kV + vs * L::kKVTileBytes, &tm_v_lin, &tm_v_img, &bars[L::bVFull + vs], e.x & 15,
-                         e.y, e.z, e.w, g.heads);
+            load_kv64<D, kSplit>(smem + L::kV + vs * L::kKVTileBytes, &tm_v_lin,
+                                 kVar ? p.item_maps + 3 * iv + 2 : &tm_v_img, &bars[L::bVFull + vs], e.x & 15,
+                                 (e.x & 15) == kLinear && kVar ? p.items[iv].t0 + e.y : e.y, e.z, e.w, g.heads);
             ++Gv;
             prog = true;
           }
@@ -502,7 +535,10 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
     const int full_bit = half == 0 ? kFullA : kFullB;
     uint32_t nq = 0, n_out = 0, nmsg = 0;
     const float sl2 = p.scale_log2;
-    // Per-pair state, set up at the pair's first tile.
+    // Per-pair state, set up at the pair's first tile. gs: the pair's geometry (its batch item's in a
+    // mixed-resolution batch).
+    Geom gv = g;
+    const Geom& gs = kVar ? gv : g;
     PairItem it{};
     int yq = 0, xq = 0, tq = 0;
     int yc = 0, xc = 0;  // the window's centre: (yq, xq), clamped inside the grid for shifted windows
@@ -527,7 +563,7 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
         ++n_out;
         tc_fence_after();
         if (it.is_text) {
-          const size_t prow = ((size_t)it.split * g.BH + it.bh) * g.n_text + (row_valid ? tq : 0);
+          const size_t prow = (size_t)gs.part_row0 + ((size_t)it.split * gs.BH + it.bh) * gs.n_text + (row_valid ? tq : 0);
           float* dst = p.opart + prow * D;
           // Two TMEM loads per wait; each row's 512-byte run is written 32 (or 16) bytes at a time.
           #pragma unroll
@@ -557,9 +593,10 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
           }
           if (row_valid) p.ml[prow] = make_float2(m_used, l);
         } else {
-          const size_t orow = (size_t)it.bh * g.T + g.n_text + (size_t)yq * g.W + xq;  // lse row
+          const long long tok = (long long)gs.t0 + gs.n_text + (long long)yq * gs.W + xq;  // token in the batch
+          const size_t orow = (size_t)it.bh * gs.tok_total + tok;                            // lse row
           const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-          __nv_bfloat16* dst = p.o + (long long)(g.n_text + yq * g.W + xq) * p.o_st +
+          __nv_bfloat16* dst = p.o + tok * p.o_st +
                                (kSplit ? (long long)(it.bh / g.heads) * p.o_sb + (long long)(it.bh % g.heads) * p.o_sh
                                        : (long long)it.bh * p.o_sh);
           #pragma unroll
@@ -602,16 +639,18 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
       t.b = mv.z;
       t.flags = mv.w & 255;
       if (j == 0) {  // first tile of a pair: its geometry, fresh statistics
-        it = decode_pair(g, blockIdx.x + (long long)(mv.w >> 8) * stride);
+        long long lw = blockIdx.x + (long long)(mv.w >> 8) * stride;
+        if constexpr (kVar) gv = p.items[locate_pair(p, lw, &lw)];
+        it = decode_pair(gs, lw);
         if (it.is_text) {
           tq = it.q0 + half * kTile + row;
-          row_valid = tq < g.n_text;
+          row_valid = tq < gs.n_text;
         } else {
           yq = it.q0 + half * kQH + (row >> 4);
           xq = it.x0 + (row & 15);
-          row_valid = (yq < g.qy1) && (xq < g.W);
-          yc = window_center(yq, g.r, g.H, g.window);
-          xc = window_center(xq, g.r, g.W, g.window);
+          row_valid = (yq < gs.qy1) && (xq < gs.W);
+          yc = window_center(yq, gs.r, gs.H, gs.window);
+          xc = window_center(xq, gs.r, gs.W, gs.window);
         }
         m_used = -INFINITY;
         l = 0.f;
@@ -643,8 +682,8 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
             #pragma unroll
             for (int q = 0; q < kFKH / 2; ++q) {
               int lo0, hi0, lo1, hi1;
-              row_range_tab(g, hwtab, hwn, yc, xc, t.a + 2 * q, t.b, &lo0, &hi0);
-              row_range_tab(g, hwtab, hwn, yc, xc, t.a + 2 * q + 1, t.b, &lo1, &hi1);
+              row_range_tab(gs, hwtab, hwn, yc, xc, t.a + 2 * q, t.b, &lo0, &hi0);
+              row_range_tab(gs, hwtab, hwn, yc, xc, t.a + 2 * q + 1, t.b, &lo1, &hi1);
               const int n0 = imax(hi0 - lo0 + 1, 0), n1 = imax(hi1 - lo1 + 1, 0);
               keep[q] = (((1u << n0) - 1u) << (lo0 & 15)) | ((((1u << n1) - 1u) << (lo1 & 15)) << 16);
             }
@@ -727,19 +766,13 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
 }
 
 // Merges the split partials of the text rows: m = max_s m_s, l = sum_s 2^(m_s - m) l_s,
-// O = sum_s 2^(m_s - m) O_s / l, LSE = (m + log2 l) ln 2. One warp per text row.
+// O = sum_s 2^(m_s - m) O_s / l, LSE = (m + log2 l) ln 2. One warp per text row: text row tq of
+// head bh of the problem (or batch item) g.
 template <int D, bool kSplit>
-__global__ void clear_fwd_combine_kernel(const FwdParams p) {
-  const Geom& g = p.g;
-  const int warps_per_block = blockDim.x / 32;
-  const long long row_id = (long long)blockIdx.x * warps_per_block + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row_id >= (long long)g.BH * g.n_text) return;
-  const int bh = (int)(row_id / g.n_text);
-  const int tq = (int)(row_id % g.n_text);
+__device__ __forceinline__ void combine_text_row(const FwdParams& p, const Geom& g, int bh, int tq, int lane) {
   float m = -INFINITY;
   for (int s = 0; s < g.fS; ++s) {
-    const float2 v = p.ml[((size_t)s * g.BH + bh) * g.n_text + tq];
+    const float2 v = p.ml[(size_t)g.part_row0 + ((size_t)s * g.BH + bh) * g.n_text + tq];
     if (v.y > 0.f) m = fmaxf(m, v.x);
   }
   constexpr int kPer = D / 32;
@@ -748,7 +781,7 @@ __global__ void clear_fwd_combine_kernel(const FwdParams p) {
   for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
   float l = 0.f;
   for (int s = 0; s < g.fS; ++s) {
-    const size_t prow = ((size_t)s * g.BH + bh) * g.n_text + tq;
+    const size_t prow = (size_t)g.part_row0 + ((size_t)s * g.BH + bh) * g.n_text + tq;
     const float2 v = p.ml[prow];
     if (!(v.y > 0.f)) continue;
     const float f = exp2f(v.x - m);
@@ -758,13 +791,40 @@ __global__ void clear_fwd_combine_kernel(const FwdParams p) {
     for (int e = 0; e < kPer; ++e) acc[e] += f * src[lane * kPer + e];
   }
   const float inv_l = 1.f / l;
-  const size_t orow = (size_t)bh * g.T + tq;  // lse row
-  __nv_bfloat16* dst = p.o + (long long)tq * p.o_st + lane * kPer +
+  const long long tok = (long long)g.t0 + tq;       // token in the (packed) tensors
+  const size_t orow = (size_t)bh * g.tok_total + tok;  // lse row
+  __nv_bfloat16* dst = p.o + tok * p.o_st + lane * kPer +
                        (kSplit ? (long long)(bh / g.heads) * p.o_sb + (long long)(bh % g.heads) * p.o_sh
                                : (long long)bh * p.o_sh);
   #pragma unroll
   for (int e = 0; e < kPer; ++e) dst[e] = __float2bfloat16_rn(acc[e] * inv_l);
   if (lane == 0) p.lse[orow] = (m + log2f(l)) * 0.69314718055994530942f;
+}
+
+template <int D, bool kSplit>
+__global__ void clear_fwd_combine_kernel(const FwdParams p) {
+  const Geom& g = p.g;
+  const int warps_per_block = blockDim.x / 32;
+  const long long row_id = (long long)blockIdx.x * warps_per_block + (threadIdx.x >> 5);
+  if (row_id >= (long long)g.BH * g.n_text) return;
+  combine_text_row<D, kSplit>(p, g, (int)(row_id / g.n_text), (int)(row_id % g.n_text), threadIdx.x & 31);
+}
+
+// The same merge for every text row of a mixed-resolution batch (rows of item i: [crow0_i,
+// crow0_i + BH * n_text_i)).
+template <int D>
+__global__ void clear_fwd_combine_varlen_kernel(const FwdParams p, long long rows) {
+  const int warps_per_block = blockDim.x / 32;
+  const long long row_id = (long long)blockIdx.x * warps_per_block + (threadIdx.x >> 5);
+  if (row_id >= rows) return;
+  int lo = 0, hi = p.n_items - 1;  // last item with crow0 <= row_id (items without text rows share the next one's)
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.items[mid].crow0 <= row_id) lo = mid; else hi = mid - 1;
+  }
+  const Geom& g = p.items[lo];
+  const long long r0 = row_id - g.crow0;
+  combine_text_row<D, false>(p, g, (int)(r0 / g.n_text), (int)(r0 % g.n_text), threadIdx.x & 31);
 }
 
 }  // namespace clear

@@ -88,6 +88,12 @@ struct Geom {
   // its own start).
   int qy0, qy1;
   int ta_lo, ta_hi, tb_lo, tb_hi, nca;
+  // Place in a packed batch (a mixed-resolution forward; the defaults are a problem of its own):
+  // the item's tokens start at token t0 of rows that are tok_total tokens long, its text rows'
+  // split partials start at partial row part_row0, and its text rows are rows
+  // [crow0, crow0 + BH * n_text) of the batch's combine pass.
+  int t0;
+  long long tok_total, part_row0, crow0;
 };
 
 CLEAR_HD int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -183,6 +189,10 @@ CLEAR_HD Geom make_geom(int B, int heads, int n_text, int H, int W, int d, int r
   g.fnTk = cdiv(n_text, kFChunk);
   set_text_key_ranges(&g, 1, n_text, g.T);
   set_forward_work(&g, 0, H);
+  g.t0 = 0;
+  g.tok_total = g.T;
+  g.part_row0 = 0;
+  g.crow0 = 0;
   return g;
 }
 

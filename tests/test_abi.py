@@ -184,3 +184,26 @@ def test_host_forward_binding_checks_tensors():
             L.clear_attn_fwd_host(ok, bad, ok, n_text, H, W, 2, o=ok.clone(), lse=lse)
     with pytest.raises(ValueError):  # lse of the wrong dtype
         L.clear_attn_fwd_host(ok, ok, ok, n_text, H, W, 2, o=ok.clone(), lse=lse.double())
+
+
+@pytest.mark.parametrize("items,expected", [
+    ([], 1), ([(1, 0, 4)], 1), ([(-1, 4, 4)], 1), ([(3, 4, 4), (2, 5, 0)], 1), ([(0, 1 << 15, 1 << 15)], 1),
+])
+def test_varlen_workspace_query_rejects_bad_items(items, expected):
+    with pytest.raises(L.ClearError) as e:
+        if not items:
+            p = L.make_params(1, 2, 0, 1, 1, 64, 3)
+            st = ctypes.c_int(0)
+            n = Bd._lib.clear_attn_fwd_varlen_workspace_size(ctypes.byref(p), 0, None, ctypes.byref(st))
+            assert n == 0
+            raise L.ClearError(st.value, "clear_attn_fwd_varlen_workspace_size")
+        L.varlen_workspace_size(2, 64, 3, items)
+    assert e.value.status == expected
+
+
+def test_varlen_workspace_grows_with_text_rows():
+    a = L.varlen_workspace_size(2, 128, 4, [(0, 16, 16), (0, 8, 8)])
+    b = L.varlen_workspace_size(2, 128, 4, [(128, 16, 16), (0, 8, 8)])
+    assert b > a > 0 and a % 256 == 0 and b % 256 == 0
+    with pytest.raises(L.ClearError):
+        L.varlen_workspace_size(2, 128, 4, [(1, 2, 2)] * 4097)
