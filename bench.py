@@ -39,7 +39,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # dram__bytes_write.sum) on the 8K r=8 shape cut to 2 heads (the full 24-head launch is too large
 # to capture), per head; heads are independent, so a full launch moves heads x this. Valid only
 # for the kernel sources it was taken on (hash below); any change to them reports null.
-FWD_TRAFFIC = {"8k_r8": {"bytes_per_head": (728.350208e6 + 134.553344e6) / 2, "src": "9de5e3a11f674246"}}
+FWD_TRAFFIC = {"8k_r8": {"bytes_per_head": (729.829376e6 + 135.572992e6) / 2, "src": "df4df3a8e7828aae"}}
 FWD_SOURCES = ("clear_fwd.cuh", "clear_sched.cuh", "clear_common.cuh", "sm100_ptx.cuh")
 
 
@@ -285,6 +285,84 @@ def time_forward_config(L, wl: Workload, peak: float, stream, seed: int, calls: 
             "l2": "flushed between calls" if small else "inputs larger than L2"}
 
 
+def _median_call_ms(fn, stream, calls=10, flush=None):
+    for _ in range(2):
+        fn()
+    torch.cuda.synchronize()
+    per = []
+    for _ in range(calls):
+        if flush is not None:
+            flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        per.append(a.elapsed_time(b))
+    return statistics.median(per)
+
+
+def time_mixed_batch(L, peak, stream, seed):
+    """One clear_attn_fwd_varlen launch over FLUX-shaped items of three resolutions (32^2, 64^2 and
+    128^2 token grids, 512 text tokens each, r=16), against the same items as separate calls."""
+    items = [(512, 64, 64), (512, 64, 64), (512, 128, 128), (512, 32, 32)]
+    heads, d, r = 24, 128, 16
+    total, starts = L.varlen_tokens(items)
+    gen = torch.Generator(device="cpu").manual_seed(seed)
+    q, k, v = (torch.randn((heads, total, d), generator=gen).to(torch.bfloat16).cuda() for _ in range(3))
+    ws = torch.empty(L.varlen_workspace_size(heads, d, r, items), dtype=torch.uint8, device="cuda")
+    o = torch.empty_like(q)
+    lse = torch.empty((heads, total), dtype=torch.float32, device="cuda")
+    useful = sum(L.pair_counts(L.make_params(1, heads, nt, H, W, d, r))[0] * 4 * d for nt, H, W in items)
+    per_item = [tuple(t[:, s:s + nt + H * W].unsqueeze(0).contiguous() for t in (q, k, v))
+                for (nt, H, W), s in zip(items, starts)]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def batch():
+        L.clear_attn_fwd_varlen(q, k, v, items, r, o=o, lse=lse, workspace=ws, stream=stream)
+
+    def separate():
+        for (nt, H, W), (qi, ki, vi) in zip(items, per_item):
+            L.clear_attn_fwd(qi, ki, vi, nt, H, W, r, stream=stream)
+
+    ms_b = _median_call_ms(batch, stream, flush=flush)
+    ms_s = _median_call_ms(separate, stream, flush=flush)
+    if L.clear_attn_check() != 0:
+        raise RuntimeError("device error timing the mixed batch")
+    return {"items": [list(t) for t in items], "heads": heads, "r": r, "ms_per_call": ms_b,
+            "useful_tflops": useful / (ms_b * 1e-3) / 1e12, "frac_of_peak": useful / (ms_b * 1e-3) / 1e12 / peak,
+            "separate_calls_ms": ms_s, "l2": "flushed between calls"}
+
+
+def time_patch_parallel(L, stream, seed):
+    """Patch-parallel split of the FLUX 2048^2 call (128 x 128 grid, r=16) into 2 and 4 row stripes,
+    every stripe's kernels run in turn on this one GPU (the halo exchange and text-row all-gather
+    between GPUs are not timed: one GPU), with the text-row difference between the exact merge and
+    the paper's Eq. 7 patch average."""
+    from local_circular_window_b200 import patch_parallel as pp
+    wl = WORKLOADS["flux2048_r16"]
+    q, k, v = make_inputs(wl, seed=seed, device="cuda")
+    ref_o, _ = L.clear_attn_fwd(q, k, v, wl.n_text, wl.H, wl.W, wl.r)
+    out = {"workload": wl.name, "single_call_ms": _median_call_ms(
+        lambda: L.clear_attn_fwd(q, k, v, wl.n_text, wl.H, wl.W, wl.r, stream=stream), stream)}
+    for stripes in (2, 4):
+        res = {}
+        for mode in ("exact", "eq7"):
+            o, _ = pp.forward_by_stripes(q, k, v, wl.n_text, wl.H, wl.W, wl.r, stripes, mode=mode)
+            res[mode] = o
+            out[f"{stripes}_stripes_{mode}_ms"] = _median_call_ms(
+                lambda: pp.forward_by_stripes(q, k, v, wl.n_text, wl.H, wl.W, wl.r, stripes, mode=mode), stream)
+        nt = wl.n_text
+        out[f"{stripes}_stripes_exact_vs_single_max_abs"] = float((res["exact"].float() - ref_o.float()).abs().max())
+        out[f"{stripes}_stripes_eq7_vs_exact_text_max_abs"] = float(
+            (res["eq7"][:, :, :nt].float() - res["exact"][:, :, :nt].float()).abs().max())
+        out[f"{stripes}_stripes_eq7_vs_exact_text_mean_abs"] = float(
+            (res["eq7"][:, :, :nt].float() - res["exact"][:, :, :nt].float()).abs().mean())
+    if L.clear_attn_check() != 0:
+        raise RuntimeError("device error timing the patch-parallel split")
+    return out
+
+
 def run_clear(args):
     world, rank, local = _dist()
     torch.cuda.set_device(local)
@@ -399,6 +477,14 @@ def run_clear(args):
         configs["clocks"] = cfg_clk.summary()
         torch.cuda.empty_cache()
 
+    # The NEXT rows built on the same kernels: a mixed-resolution batch in one launch, and the
+    # patch-parallel split (each stripe's work on this GPU in turn).
+    extras = None
+    if not args.no_configs and rank == 0:
+        extras = {"mixed_batch": time_mixed_batch(L, peak, stream, seed=4000),
+                  "patch_parallel": time_patch_parallel(L, stream, seed=4001)}
+        torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         sec, cores, sample = oracle_call_seconds(wl, args.cpu_budget)
@@ -422,7 +508,7 @@ def run_clear(args):
                          "frac": achieved / peak, "traffic": _fwd_traffic(wl),
                          "peak_source": f"{peak_kind} bf16 dense (burst; kernel timed alone)",
                          "kernel": "clear_fwd_kernel + clear_fwd_combine_kernel (one call, CUDA events)"},
-            "e2e": e2e, "cpu_baseline": cpu, "bwd": bwd, "configs": configs, "clocks": clocks,
+            "e2e": e2e, "cpu_baseline": cpu, "bwd": bwd, "configs": configs, "extras": extras, "clocks": clocks,
             "gpu_launches": 2 * args.steps,
         }
         print(json.dumps(line), flush=True)

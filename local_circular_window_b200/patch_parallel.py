@@ -1,4 +1,8 @@
-"""Patch-parallel CLEAR inference: the image grid split into row stripes, one per rank (GPU).
+"""Patch-parallel CLEAR inference: heads split over ranks, or the image grid split into row stripes,
+one per rank (GPU).
+
+Head sharding needs no exchange at all: heads are independent problems, so each rank runs the
+forward on its own heads (head_parallel_forward gathers the outputs if asked).
 
 CLEAR's window has radius r, so an image query reaches r - 1 grid rows up and down: a rank that owns
 rows [lo, hi) needs, besides the text tokens every rank holds, only r - 1 rows of keys from each
@@ -25,6 +29,45 @@ from dataclasses import dataclass
 import torch
 
 from . import _binding as B
+
+
+def head_bounds(heads: int, world: int):
+    """Heads [lo, hi) of each rank: a balanced split of the heads over `world` ranks."""
+    base, extra = divmod(heads, world)
+    out, lo = [], 0
+    for p in range(world):
+        hi = lo + base + (1 if p < extra else 0)
+        out.append((lo, hi))
+        lo = hi
+    return out
+
+
+def head_parallel_forward(q, k, v, n_text: int, H: int, W: int, r: int, group=None, window: str = "circle",
+                          gather: bool = True, local_forward=None):
+    """Forward of this rank's heads. q, k, v: [B, heads_r, T, d], the heads head_bounds assigns to this
+    rank. Returns (o, lse) of those heads, or, with gather, of all heads on every rank (an all-gather
+    of the outputs; the forward itself exchanges nothing)."""
+    import torch.distributed as dist
+
+    world = dist.get_world_size(group)
+    fwd = local_forward or (lambda q_, k_, v_: B.clear_attn_fwd(q_, k_, v_, n_text, H, W, r, window=window))
+    o, lse = fwd(q, k, v)
+    if not gather:
+        return o, lse
+    counts = [torch.zeros(1, dtype=torch.int64, device=o.device) for _ in range(world)]
+    dist.all_gather(counts, torch.tensor([o.shape[1]], dtype=torch.int64, device=o.device), group)
+    counts = [int(c.item()) for c in counts]
+    m = max(counts)
+    pad_o = o.new_zeros((o.shape[0], m) + tuple(o.shape[2:]))
+    pad_l = lse.new_zeros((lse.shape[0], m) + tuple(lse.shape[2:]))
+    pad_o[:, :o.shape[1]] = o
+    pad_l[:, :lse.shape[1]] = lse
+    os_ = [torch.empty_like(pad_o) for _ in range(world)]
+    ls_ = [torch.empty_like(pad_l) for _ in range(world)]
+    dist.all_gather(os_, pad_o, group)
+    dist.all_gather(ls_, pad_l, group)
+    return (torch.cat([t[:, :c] for t, c in zip(os_, counts)], dim=1),
+            torch.cat([t[:, :c] for t, c in zip(ls_, counts)], dim=1))
 
 
 def stripe_bounds(H: int, world: int):

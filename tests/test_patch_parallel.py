@@ -140,3 +140,35 @@ def test_stripe_bounds_balanced_and_contiguous():
             assert b == _bounds(H, world)
             sizes = [hi - lo for lo, hi in b]
             assert max(sizes) - min(sizes) <= 1 and sum(sizes) == H
+
+
+def _head_rank_main(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from local_circular_window_b200 import patch_parallel as pp
+        n_text, H, W, r, heads = 4, 7, 6, 3, 5
+        wl = Workload("hp", 1, heads, n_text, H, W, 16, r)
+        q, k, v = (t.double() for t in make_inputs(wl, seed=12, dtype=torch.float32))
+        lo, hi = pp.head_bounds(heads, world)[rank]
+
+        def fwd(q_, k_, v_):
+            O, Lse = oracle.clear_attention_forward(q_, k_, v_, n_text, H, W, r)
+            return torch.from_numpy(O), torch.from_numpy(Lse)
+
+        o, lse = pp.head_parallel_forward(q[:, lo:hi], k[:, lo:hi], v[:, lo:hi], n_text, H, W, r, local_forward=fwd)
+        out[rank] = (o.numpy(), lse.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_head_sharded_ranks_gather_the_full_result(world):
+    out = mp.get_context("spawn").Manager().dict()
+    mp.spawn(_head_rank_main, args=(world, _free_port(), out), nprocs=world, join=True)
+    wl = Workload("hp", 1, 5, 4, 7, 6, 16, 3)
+    q, k, v = make_inputs(wl, seed=12, dtype=torch.float32)
+    O, Lse = oracle.clear_attention_forward(q, k, v, 4, 7, 6, 3)
+    for rank in range(world):
+        o, lse = out[rank]
+        assert o.shape == O.shape and np.abs(o - O).max() < 1e-12 and np.abs(lse - Lse).max() < 1e-12
