@@ -80,3 +80,14 @@ def make_random(shape, seed: int, dtype=torch.bfloat16, device="cpu"):
     gen.manual_seed(seed)
     t = torch.randn(shape, generator=gen, dtype=torch.float32, device=dev)
     return t.to(dtype) if dtype != torch.float32 else t
+
+
+def quantize_e4m3(t: torch.Tensor):
+    """Encode t [B, heads, T, d] as OCP FP8 E4M3 codes with one scale per (batch, head): the scale
+    maps the head's largest magnitude to 448 (the format's largest finite value) and the codes are
+    t / scale rounded to nearest-even by torch's float8_e4m3fn cast. Returns (codes uint8, scale
+    float32 [B, heads]); decode(codes) * scale approximates t."""
+    amax = t.detach().float().abs().amax(dim=(2, 3)).clamp_min(1e-12)
+    scale = amax / 448.0
+    codes = (t.float() / scale[:, :, None, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes, scale

@@ -14,4 +14,6 @@ from .clear_attention import (  # noqa: F401
     useful_flops_fwd,
     clear_attention_stripe,
     clear_text_rows_patch_average,
+    e4m3_decode,
+    clear_attention_forward_fp8,
 )

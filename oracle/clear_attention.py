@@ -42,6 +42,14 @@ Revs Pre-Trained Diffusion Transformers Up"):
    gives one stripe's rows (image rows of its own grid rows, text rows over the keys it is given),
    and `clear_text_rows_patch_average` the patch-wise average of Eq. 7 for the text rows.
 
+8. FP8 score products (not on the pages; a variant for inference): q and k arrive as 8-bit
+   floating-point codes in the OCP FP8 E4M3 format with a dequantization scale per (batch, head),
+   v stays bf16. `e4m3_decode` writes the format out (sign bit, 4 exponent bits with bias 7,
+   3 mantissa bits; exponent field 0 holds subnormals m * 2^-9; the all-ones exponent and mantissa
+   is NaN, the format has no infinities) and `clear_attention_forward_fp8` runs the plain forward
+   above on q = decode(q8) * s_q and k = decode(k8) * s_k: the scores are those of the dequantized
+   inputs, the rest is unchanged.
+
 Readings where the pages leave a step open (each listed with its reason in the design notes):
 strict "<" in the radius test; image tokens in row-major order t = n_text + y*W + x; windows are
 clipped at the grid border (border queries see fewer keys); text queries attend to every token
@@ -321,3 +329,34 @@ def clear_text_rows_patch_average(q, k, v, n_text: int, H: int, W: int, row_boun
                 P, _ = _masked_softmax_rows(S, np.ones_like(S, dtype=bool))
                 O[b, h] += P @ v[b, h, cols]
     return O / n
+
+
+# ----------------------------------------------------------------------------------------------
+# FP8 (E4M3) score products
+# ----------------------------------------------------------------------------------------------
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Value of each OCP FP8 E4M3 code (uint8 array) as float64: (-1)^s * 2^(e-7) * (1 + m/8) for
+    exponent field e in 1..15, (-1)^s * 2^-6 * (m/8) for e = 0 (subnormals, including +-0), and
+    NaN for the codes with e = 15 and m = 7 (0x7F, 0xFF)."""
+    c = np.asarray(codes, dtype=np.int64)
+    sign = np.where((c >> 7) & 1, -1.0, 1.0)
+    e = (c >> 3) & 15
+    m = (c & 7).astype(np.float64)
+    normal = sign * np.ldexp(1.0 + m / 8.0, (e - 7).astype(np.int64))
+    sub = sign * np.ldexp(m / 8.0, -6)
+    v = np.where(e == 0, sub, normal)
+    return np.where((e == 15) & (m == 7), np.nan, v)
+
+
+def clear_attention_forward_fp8(q8, k8, v, s_q, s_k, n_text: int, H: int, W: int, r: int, scale=None,
+                                window: str = "circle"):
+    """CLEAR forward with E4M3 query and key codes. q8, k8: uint8 codes [B, heads, T, d]; v: values
+    [B, heads, T, d]; s_q, s_k: dequantization scales [B, heads]. Returns (O, LSE) in float64 of
+    the plain forward on q = decode(q8) * s_q, k = decode(k8) * s_k."""
+    q8 = q8.detach().cpu().numpy() if hasattr(q8, "detach") else np.asarray(q8)
+    k8 = k8.detach().cpu().numpy() if hasattr(k8, "detach") else np.asarray(k8)
+    sq = _as_f64(s_q)[:, :, None, None]
+    sk = _as_f64(s_k)[:, :, None, None]
+    return clear_attention_forward(e4m3_decode(q8) * sq, e4m3_decode(k8) * sk, v, n_text, H, W, r, scale=scale,
+                                   window=window)
