@@ -181,6 +181,23 @@ CLEAR_API clear_status_t clear_attn_text_merge(const clear_attn_params_t* params
                                                void* stream);
 
 /*
+ * Forward with FP8 score products: q and k as OCP FP8 E4M3 codes (one byte per element), v in
+ * bf16. The scores are the products of the decoded codes, scaled by qk_descale[b * heads + h]
+ * (= s_q * s_k, the two inputs' dequantization scales) and by 1/sqrt(d); everything after the
+ * scores (mask, softmax, P rounded to bf16, P V, O and LSE) is as in clear_attn_fwd (the CLEAR mask of
+ * the pith.science review of "CLEAR: Conv-Like Linearization Revs Pre-Trained Diffusion
+ * Transformers Up", "Core claim"; the paper has no FP8 path). The score products run as
+ * tcgen05.mma kind::f8f6f4 at twice the bf16 rate on half the q and k bytes.
+ *   q8, k8: uint8 [B, heads, T, d] contiguous, d = 128 (other d: CLEAR_ERR_UNSUPPORTED);
+ *   v, o: bf16 [B, heads, T, d]; lse: fp32 [B, heads, T]; qk_descale: device fp32 [B * heads];
+ *   workspace: clear_attn_fwd_workspace_size bytes (same as the bf16 forward).
+ * Otherwise as clear_attn_fwd.
+ */
+CLEAR_API clear_status_t clear_attn_fwd_fp8(const clear_attn_params_t* params, const void* q8, const void* k8,
+                                            const void* v, const float* qk_descale, void* o, float* lse,
+                                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Mixed-resolution batch forward: n_items problems of their own (n_text, H, W) in ONE launch (their
  * pairs form one work list), e.g. a batch holding 1024^2 and 2048^2 images at once. Each item is the
  * CLEAR forward of clear_attn_fwd (pith.science review of "CLEAR: Conv-Like Linearization Revs

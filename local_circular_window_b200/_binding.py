@@ -79,6 +79,8 @@ _lib.clear_attn_fwd_stripe_workspace_size.restype = ctypes.c_size_t
 _lib.clear_attn_fwd_stripe_workspace_size.argtypes = [_P, _S, ctypes.POINTER(_i)]
 _lib.clear_attn_fwd_stripe.restype = _i
 _lib.clear_attn_fwd_stripe.argtypes = [_P, _S, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+_lib.clear_attn_fwd_fp8.restype = _i
+_lib.clear_attn_fwd_fp8.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 _lib.clear_attn_fwd_varlen_workspace_size.restype = ctypes.c_size_t
 _lib.clear_attn_fwd_varlen_workspace_size.argtypes = [_P, _i, ctypes.POINTER(_i), ctypes.POINTER(_i)]
 _lib.clear_attn_fwd_varlen.restype = _i
@@ -308,6 +310,36 @@ def clear_attn_fwd_stripe(q, k, v, n_text: int, H: int, W: int, r: int, stripe: 
                                         _stream_ptr(stream))
     if status != CLEAR_OK:
         raise ClearError(status, "clear_attn_fwd_stripe")
+    return o, lse
+
+
+def clear_attn_fwd_fp8(q8, k8, v, qk_descale, n_text: int, H: int, W: int, r: int, o=None, lse=None, workspace=None,
+                       stream=None, window="circle"):
+    """Forward with E4M3 score products through clear_attn_fwd_fp8. q8, k8: contiguous CUDA uint8
+    E4M3 codes [B, heads, T, d] (d = 128); v: bf16 like q8; qk_descale: CUDA float32 [B, heads]
+    (s_q * s_k per head). Returns (o, lse)."""
+    B, heads, T, d = q8.shape
+    if T != n_text + H * W:
+        raise ValueError("T must equal n_text + H * W")
+    for name, t in (("q8", q8), ("k8", k8)):
+        if not (t.is_cuda and t.dtype == torch.uint8 and t.is_contiguous() and tuple(t.shape) == (B, heads, T, d)):
+            raise ValueError(f"{name} must be a contiguous CUDA uint8 tensor of shape {(B, heads, T, d)}")
+    _check_qkv("v", v, q8.shape)
+    if not (qk_descale.is_cuda and qk_descale.dtype == torch.float32 and qk_descale.is_contiguous()
+            and qk_descale.numel() == B * heads):
+        raise ValueError("qk_descale must be a contiguous CUDA float32 tensor of B * heads values")
+    p = make_params(B, heads, n_text, H, W, d, r, window)
+    if o is None:
+        o = torch.empty(q8.shape, dtype=torch.bfloat16, device=q8.device)
+    if lse is None:
+        lse = torch.empty((B, heads, T), dtype=torch.float32, device=q8.device)
+    if workspace is None:
+        n = fwd_workspace_size(p)
+        workspace = torch.empty(max(16, n), dtype=torch.uint8, device=q8.device)
+    status = _lib.clear_attn_fwd_fp8(ctypes.byref(p), _ptr(q8), _ptr(k8), _ptr(v), _ptr(qk_descale), _ptr(o), _ptr(lse),
+                                     _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    if status != CLEAR_OK:
+        raise ClearError(status, "clear_attn_fwd_fp8")
     return o, lse
 
 

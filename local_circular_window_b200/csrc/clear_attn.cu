@@ -296,6 +296,73 @@ clear_status_t launch_fwd(const Geom& g, const QKVMaps& m, void* o, const Tensor
   return CLEAR_OK;
 }
 
+// E4M3 q or k (one byte per element, contiguous [B, heads, T, d] with d = 128): linear view
+// (d, T, B*heads) with lin_rows-token boxes and image view (d, W, H, B*heads) with img_rows x 16
+// boxes, each box one 128-byte row block (128-byte swizzle), as the bf16 maps but with one block.
+bool make_e4m3_maps(CUtensorMap* lin, CUtensorMap* img, const void* base, const Geom& g, int lin_rows, int img_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)g.d, (cuuint64_t)g.T, (cuuint64_t)g.BH};
+  cuuint64_t strides[2] = {(cuuint64_t)g.d, (cuuint64_t)g.T * g.d};
+  cuuint32_t box[3] = {(cuuint32_t)g.d, (cuuint32_t)lin_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  if (enc(lin, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  const char* ib = static_cast<const char*>(base) + (size_t)g.n_text * g.d;
+  cuuint64_t idims[4] = {(cuuint64_t)g.d, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.BH};
+  cuuint64_t istrides[3] = {(cuuint64_t)g.d, (cuuint64_t)g.W * g.d, (cuuint64_t)g.T * g.d};
+  cuuint32_t ibox[4] = {(cuuint32_t)g.d, (cuuint32_t)kKW, (cuuint32_t)img_rows, 1};
+  cuuint32_t iestr[4] = {1, 1, 1, 1};
+  return enc(img, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<char*>(ib), idims, istrides, ibox, iestr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The forward with E4M3 q, k (score products of kind::f8f6f4) and bf16 v; contiguous tensors.
+clear_status_t launch_fwd_f8(const Geom& g, const void* q8, const void* k8, const void* v, const float* qk_descale,
+                             void* o, float* lse, void* ws, int num_sms, cudaStream_t stream) {
+  constexpr int D = 128;
+  using L = FwdLayout<D, true>;
+  QKVMaps m;
+  const TensorStrides cs = contiguous_strides(g);
+  if (!make_e4m3_maps(&m.q_lin, &m.q_img, q8, g, kTile, kQH) || !make_e4m3_maps(&m.k_lin, &m.k_img, k8, g, kFChunk, kFKH) ||
+      !make_fwd_tensor_maps(&m.v_lin, &m.v_img, v, cs, g, kFChunk, kFKH, false))
+    return CLEAR_ERR_CUDA;
+  const int smem_bytes = L::alloc_bytes(hw_table_size(g.r, g.H));
+  if (smem_bytes > 232448) return CLEAR_ERR_UNSUPPORTED;
+  FwdParams p{};
+  p.g = g;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.o_sb = cs.sb;
+  p.o_sh = cs.sh;
+  p.o_st = cs.st;
+  p.lse = lse;
+  const FwdWorkspace wl = fwd_workspace_layout(g);
+  p.opart = g.n_text ? reinterpret_cast<float*>(static_cast<char*>(ws) + wl.opart_off) : nullptr;
+  p.ml = g.n_text ? reinterpret_cast<float2*>(static_cast<char*>(ws) + wl.ml_off) : nullptr;
+  p.wide_o = (reinterpret_cast<uintptr_t>(o) & 31u) == 0;
+  p.wide_part = (reinterpret_cast<uintptr_t>(p.opart) & 31u) == 0;
+  p.n_work = g.n_txt_pairs + g.n_img_pairs;
+  p.qk_descale = qk_descale;
+  if (cudaFuncSetAttribute(clear_fwd_kernel<D, false, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem_bytes) != cudaSuccess)
+    return CLEAR_ERR_CUDA;
+  const long long grid = p.n_work < num_sms ? p.n_work : num_sms;
+  clear_fwd_kernel<D, false, false, true><<<(unsigned)grid, kFwdThreads, smem_bytes, stream>>>(
+      m.q_lin, m.q_img, m.k_lin, m.k_img, m.v_lin, m.v_img, p);
+  if (cudaGetLastError() != cudaSuccess) return CLEAR_ERR_CUDA;
+  if (g.n_text > 0) {
+    const long long rows = (long long)g.BH * g.n_text;
+    const int wpb = 8;
+    clear_fwd_combine_kernel<D, false><<<(unsigned)((rows + wpb - 1) / wpb), wpb * 32, 0, stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return CLEAR_ERR_CUDA;
+  }
+  return CLEAR_OK;
+}
+
 // Device address of g_noalloc_scratch on the current device. The symbol's name is only a host-side
 // stand-in; the address is looked up with that device current and kept once the lookup succeeded.
 // A failed lookup (e.g. the module could not be loaded because device memory was exhausted, or a
@@ -696,6 +763,23 @@ clear_status_t clear_attn_fwd_stripe(const clear_attn_params_t* params, const cl
   const TensorStrides cs = contiguous_strides(c.g);
   const TensorStrides st4[4] = {cs, cs, cs, cs};
   return run_fwd(c.g, st4, q, k, v, o, lse, workspace, static_cast<cudaStream_t>(stream));
+}
+
+clear_status_t clear_attn_fwd_fp8(const clear_attn_params_t* params, const void* q8, const void* k8, const void* v,
+                                  const float* qk_descale, void* o, float* lse, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  const Checked c = check_params(params);
+  if (c.st != CLEAR_OK) return c.st;
+  if (params->d != 128) return CLEAR_ERR_UNSUPPORTED;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !qk_descale ||
+      (reinterpret_cast<uintptr_t>(qk_descale) & 3u) != 0)
+    return CLEAR_ERR_INVALID_ARG;
+  const size_t need = fwd_workspace_layout(c.g).total;
+  if (need > 0 && (workspace_bytes < need || !aligned16(workspace))) return CLEAR_ERR_WORKSPACE;
+  int num_sms = 0;
+  const clear_status_t st = check_device(&num_sms);
+  if (st != CLEAR_OK) return st;
+  return launch_fwd_f8(c.g, q8, k8, v, qk_descale, o, lse, workspace, num_sms, static_cast<cudaStream_t>(stream));
 }
 
 size_t clear_attn_fwd_varlen_workspace_size(const clear_attn_params_t* params, int n_items, const int* item_shapes,

@@ -76,6 +76,9 @@ struct FwdParams {
   const CUtensorMap* item_maps;
   const long long* wbound;
   int n_items;
+  // FP8 score products (the kernel's kF8 parameter): s_q * s_k of each (batch, head), the
+  // dequantization of the E4M3 codes' products, folded into the score scale.
+  const float* qk_descale;
 };
 
 // Item of pair w of a mixed-resolution batch, and w's index among the item's own pairs.
@@ -127,15 +130,17 @@ __device__ __forceinline__ void st_global_v8(void* ptr, uint32_t a0, uint32_t a1
                : "memory");
 }
 
-template <int D>
+// kF8: q and k tiles hold E4M3 codes (one byte per element; one 128-byte row block at d = 128).
+template <int D, bool kF8 = false>
 struct FwdLayout {
-  static constexpr int kQTileBytes = kTile * D * 2;      // one 128-row bf16 query tile
-  static constexpr int kKVTileBytes = kFChunk * D * 2;   // one 64-key bf16 tile
+  static constexpr int kQTileBytes = kTile * D * (kF8 ? 1 : 2);     // one 128-row query tile
+  static constexpr int kKTileBytes = kFChunk * D * (kF8 ? 1 : 2);   // one 64-key k tile
+  static constexpr int kVTileBytes = kFChunk * D * 2;               // one 64-key bf16 v tile
   static constexpr int kKVBlock = kFChunk * 128;         // 64 rows x 64 elements (128B-swizzled)
   static constexpr int kQ = 0;                           // Q_A, Q_B
   static constexpr int kK = kQ + 2 * kQTileBytes;
-  static constexpr int kV = kK + kKStages * kKVTileBytes;
-  static constexpr int kBars = kV + kVStages * kKVTileBytes;
+  static constexpr int kV = kK + kKStages * kKTileBytes;
+  static constexpr int kBars = kV + kVStages * kVTileBytes;
   // barrier indices
   static constexpr int bQFull = 0, bQEmpty = 1;
   static constexpr int bKFull = 2;                       // + slot
@@ -209,13 +214,13 @@ __device__ __forceinline__ void load_q128(uint8_t* dst, const CUtensorMap* lin, 
   }
 }
 
-template <int D, bool kSplit, bool kVar>
+template <int D, bool kSplit, bool kVar, bool kF8 = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_constant__ CUtensorMap tm_q_img,
                  const __grid_constant__ CUtensorMap tm_k_lin, const __grid_constant__ CUtensorMap tm_k_img,
                  const __grid_constant__ CUtensorMap tm_v_lin, const __grid_constant__ CUtensorMap tm_v_img,
                  const FwdParams p) {
-  using L = FwdLayout<D>;
+  using L = FwdLayout<D, kF8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
@@ -310,7 +315,16 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
           const int t0 = kVar ? gq.t0 : 0;  // the item's first token in the packed batch
           const PairItem it = decode_pair(gq, lw);
           mbar_arrive_expect_tx(&bars[L::bQFull], (it.validB ? 2 : 1) * L::kQTileBytes);
-          if (it.is_text) {
+          if constexpr (kF8) {  // one 128-byte row block per tile
+            uint8_t* qa = smem + L::kQ;
+            if (it.is_text) {
+              tma_load_3d(qa, &tm_q_lin, &bars[L::bQFull], 0, it.q0, it.bh);
+              if (it.validB) tma_load_3d(qa + L::kQTileBytes, &tm_q_lin, &bars[L::bQFull], 0, it.q0 + kTile, it.bh);
+            } else {
+              tma_load_4d(qa, &tm_q_img, &bars[L::bQFull], 0, it.x0, it.q0, it.bh);
+              if (it.validB) tma_load_4d(qa + L::kQTileBytes, &tm_q_img, &bars[L::bQFull], 0, it.x0, it.q0 + kQH, it.bh);
+            }
+          } else if (it.is_text) {
             load_q128<D, kSplit>(smem + L::kQ, &tm_q_lin, qimg, &bars[L::bQFull], kLinear, t0 + it.q0, 0, it.bh, g.heads);
             if (it.validB)
               load_q128<D, kSplit>(smem + L::kQ + L::kQTileBytes, &tm_q_lin, qimg, &bars[L::bQFull], kLinear,
@@ -332,8 +346,14 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
             // Linear tiles carry item-local tokens; bits 16+ of the first word hold the batch item.
             ring[Gk % kTileRing] = make_int4(tcur.kind | (tcur.flags << 4) | (next_in_pair ? 0 : (1 << 12)) | (ik << 16),
                                              tcur.a, tcur.b, itk.bh);
-            mbar_arrive_expect_tx(&bars[L::bKFull + ks], L::kKVTileBytes);
-            load_kv64<D, kSplit>(smem + L::kK + ks * L::kKVTileBytes, &tm_k_lin,
+            mbar_arrive_expect_tx(&bars[L::bKFull + ks], L::kKTileBytes);
+            if constexpr (kF8) {  // one 128-byte row block per tile
+              if (tcur.kind == kLinear)
+                tma_load_3d(smem + L::kK + ks * L::kKTileBytes, &tm_k_lin, &bars[L::bKFull + ks], 0, tcur.a, itk.bh);
+              else
+                tma_load_4d(smem + L::kK + ks * L::kKTileBytes, &tm_k_img, &bars[L::bKFull + ks], 0, tcur.b, tcur.a, itk.bh);
+            } else
+            load_kv64<D, kSplit>(smem + L::kK + ks * L::kKTileBytes, &tm_k_lin,
                                  kVar ? p.item_maps + 3 * ik + 1 : &tm_k_img, &bars[L::bKFull + ks], tcur.kind,
                                  tcur.kind == kLinear && kVar ? p.items[ik].t0 + tcur.a : tcur.a, tcur.b, itk.bh, g.heads);
             ++Gk;
@@ -353,8 +373,8 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
           if (mbar_test(&bars[L::bVEmpty + vs], ((Gv / kVStages) & 1) ^ 1)) {
             const int4 e = ring[Gv % kTileRing];
             const int iv = e.x >> 16;
-            mbar_arrive_expect_tx(&bars[L::bVFull + vs], L::kKVTileBytes);
-            load_kv64<D, kSplit>(smem + L::kV + vs * L::kKVTileBytes, &tm_v_lin,
+            mbar_arrive_expect_tx(&bars[L::bVFull + vs], L::kVTileBytes);
+            load_kv64<D, kSplit>(smem + L::kV + vs * L::kVTileBytes, &tm_v_lin,
                                  kVar ? p.item_maps + 3 * iv + 2 : &tm_v_img, &bars[L::bVFull + vs], e.x & 15,
                                  (e.x & 15) == kLinear && kVar ? p.items[iv].t0 + e.y : e.y, e.z, e.w, g.heads);
             ++Gv;
@@ -411,7 +431,7 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
             const bool vr = mbar_test(&bars[L::bVFull + vs], (Gp / kVStages) & 1);
             if (pr && vr) {
               tc_fence_after();
-              const uint64_t vd = vdesc0 + (uint64_t)((vs * L::kKVTileBytes) >> 4);
+              const uint64_t vd = vdesc0 + (uint64_t)((vs * L::kVTileBytes) >> 4);
               const uint32_t s_tm = tmem + L::s_col(h, b);
               const bool first = hF & 1;
               #pragma unroll
@@ -471,12 +491,21 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
                 mbar_arrive(&bars[L::bMsgFull + 2 * h + ms]);
                 ++nmsg;
                 tc_fence_after();
-                const uint64_t kd = kdesc0 + (uint64_t)((ks * L::kKVTileBytes) >> 4);
-                #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                  const uint32_t qoff = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-                  const uint32_t koff = ((kk >> 2) * L::kKVBlock + (kk & 3) * 32) >> 4;
-                  umma_ss(tmem + L::s_col(h, b), qdesc + qoff, kd + koff, idesc_qk, kk > 0);
+                const uint64_t kd = kdesc0 + (uint64_t)((ks * L::kKTileBytes) >> 4);
+                if constexpr (kF8) {
+                  // 32 one-byte elements per step, all inside the tile's single 128-byte row block
+                  constexpr uint32_t idesc_f8 = idesc_e4m3_f32(128, kFChunk);
+                  #pragma unroll
+                  for (int kk = 0; kk < D / 32; ++kk)
+                    umma_ss_f8(tmem + L::s_col(h, b), qdesc + (uint32_t)((kk * 32) >> 4), kd + (uint32_t)((kk * 32) >> 4),
+                               idesc_f8, kk > 0);
+                } else {
+                  #pragma unroll
+                  for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t qoff = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+                    const uint32_t koff = ((kk >> 2) * L::kKVBlock + (kk & 3) * 32) >> 4;
+                    umma_ss(tmem + L::s_col(h, b), qdesc + qoff, kd + koff, idesc_qk, kk > 0);
+                  }
                 }
                 umma_commit(&bars[L::bSFull + 2 * h + b]);
                 umma_commit(&bars[L::bKEmpty + ks]);
@@ -534,7 +563,7 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
     const uint32_t o_tm = tmem + lane_base + L::o_col(half);
     const int full_bit = half == 0 ? kFullA : kFullB;
     uint32_t nq = 0, n_out = 0, nmsg = 0;
-    const float sl2 = p.scale_log2;
+    float sl2 = p.scale_log2;  // with kF8, times the pair's s_q * s_k (set at each pair's first tile)
     // Per-pair state, set up at the pair's first tile. gs: the pair's geometry (its batch item's in a
     // mixed-resolution batch).
     Geom gv = g;
@@ -642,6 +671,7 @@ clear_fwd_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_cons
         long long lw = blockIdx.x + (long long)(mv.w >> 8) * stride;
         if constexpr (kVar) gv = p.items[locate_pair(p, lw, &lw)];
         it = decode_pair(gs, lw);
+        if constexpr (kF8) sl2 = p.scale_log2 * __ldg(p.qk_descale + it.bh);
         if (it.is_text) {
           tq = it.q0 + half * kTile + row;
           row_valid = tq < gs.n_text;
