@@ -29,7 +29,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from clear_inputs import WORKLOADS, Workload, make_inputs  # noqa: E402
+from clear_inputs import WORKLOADS, Workload, make_inputs, quantize_e4m3  # noqa: E402
 
 METRIC = "CLEAR attn useful TFLOP/s & ms/call (bf16, 512² grid, r=8); % of TC peak"
 FALLBACK_BF16_TFLOPS = 1590.0
@@ -334,6 +334,34 @@ def time_mixed_batch(L, peak, stream, seed):
             "separate_calls_ms": ms_s, "l2": "flushed between calls"}
 
 
+def time_fp8_forward(L, peak, stream, seed):
+    """The forward with E4M3 score products (clear_attn_fwd_fp8) on the headline workload and on
+    8K r=32, against the bf16 forward on the same inputs (same calls, CUDA events)."""
+    out = {}
+    for name in ("8k_r8", "8k_r32"):
+        wl = WORKLOADS[name]
+        q, k, v = make_inputs(wl, seed=seed, device="cuda")
+        q8, sq = quantize_e4m3(q)
+        k8, sk = quantize_e4m3(k)
+        desc = (sq * sk).float().contiguous()
+        del q, k
+        o = torch.empty_like(v)
+        lse = torch.empty((wl.B, wl.heads, wl.T), dtype=torch.float32, device="cuda")
+        p = L.make_params(wl.B, wl.heads, wl.n_text, wl.H, wl.W, wl.d, wl.r)
+        ws = torch.empty(max(16, L.fwd_workspace_size(p)), dtype=torch.uint8, device="cuda")
+        ms = _median_call_ms(lambda: L.clear_attn_fwd_fp8(q8, k8, v, desc, wl.n_text, wl.H, wl.W, wl.r, o=o, lse=lse,
+                                                          workspace=ws, stream=stream), stream)
+        useful, _ = _flops(L, wl)
+        out[name] = {"ms_per_call": ms, "useful_tflops": useful / (ms * 1e-3) / 1e12,
+                     "frac_of_bf16_peak": useful / (ms * 1e-3) / 1e12 / peak}
+        del q8, k8, v, o, lse, ws
+        torch.cuda.empty_cache()
+    if L.clear_attn_check() != 0:
+        raise RuntimeError("device error timing the FP8 forward")
+    out["inputs"] = "q, k E4M3 codes with one scale per (batch, head); v bf16; inputs larger than L2"
+    return out
+
+
 def time_patch_parallel(L, stream, seed):
     """Patch-parallel split of the FLUX 2048^2 call (128 x 128 grid, r=16) into 2 and 4 row stripes,
     every stripe's kernels run in turn on this one GPU (the halo exchange and text-row all-gather
@@ -482,7 +510,8 @@ def run_clear(args):
     extras = None
     if not args.no_configs and rank == 0:
         extras = {"mixed_batch": time_mixed_batch(L, peak, stream, seed=4000),
-                  "patch_parallel": time_patch_parallel(L, stream, seed=4001)}
+                  "patch_parallel": time_patch_parallel(L, stream, seed=4001),
+                  "fp8_scores": time_fp8_forward(L, peak, stream, seed=4002)}
         torch.cuda.empty_cache()
 
     cpu = None
