@@ -50,6 +50,15 @@ Revs Pre-Trained Diffusion Transformers Up"):
    above on q = decode(q8) * s_q and k = decode(k8) * s_k: the scores are those of the dequantized
    inputs, the rest is unchanged.
 
+9. Rotary position embedding applied to q and k before the scores (a fused-prologue variant): the
+   review lists an NTK-aware RoPE scale factor of 10 among the free parameters ["Assumptions &
+   free parameters"] and the paper cites RoFormer (rotary embedding: each pair of adjacent head
+   dims (2i, 2i+1) rotated by position * base^(-2i/d)) and NTK-aware scaled RoPE (the base raised
+   to theta * alpha^(d/(d-2)) for a scale factor alpha). Read for the token grid as axial 2D RoPE:
+   the first half of the head dims rotated by the grid row y, the second half by the column x,
+   each half with its own d/2 dims in the formulas above; text tokens are not rotated.
+   `rope_2d`, `clear_attention_forward_rope`.
+
 Readings where the pages leave a step open (each listed with its reason in the design notes):
 strict "<" in the radius test; image tokens in row-major order t = n_text + y*W + x; windows are
 clipped at the grid border (border queries see fewer keys); text queries attend to every token
@@ -360,3 +369,43 @@ def clear_attention_forward_fp8(q8, k8, v, s_q, s_k, n_text: int, H: int, W: int
     sk = _as_f64(s_k)[:, :, None, None]
     return clear_attention_forward(e4m3_decode(q8) * sq, e4m3_decode(k8) * sk, v, n_text, H, W, r, scale=scale,
                                    window=window)
+
+
+# ----------------------------------------------------------------------------------------------
+# Rotary position embedding (axial 2D, interleaved pairs, NTK-aware base)
+# ----------------------------------------------------------------------------------------------
+
+def rope_inv_freq(d_axis: int, theta: float = 10000.0, ntk: float = 1.0) -> np.ndarray:
+    """Rotation rate of each dim pair of one axis: base^(-2i/d_axis), i = 0 .. d_axis/2 - 1, with
+    the NTK-aware base theta * ntk^(d_axis / (d_axis - 2))."""
+    base = theta * ntk ** (d_axis / (d_axis - 2.0))
+    return base ** (-np.arange(0, d_axis, 2, dtype=np.float64) / d_axis)
+
+
+def rope_2d(x, n_text: int, H: int, W: int, theta: float = 10000.0, ntk: float = 1.0) -> np.ndarray:
+    """Axial 2D rotary embedding of x [..., T, d] (float64 copy): image token (y, x) has dims
+    [0, d/2) rotated by y and dims [d/2, d) by x, pair (2i, 2i+1) of an axis by angle
+    position * rope_inv_freq(d/2)[i]: (a, b) -> (a cos - b sin, a sin + b cos). Text tokens are
+    unchanged."""
+    x = _as_f64(x).copy()
+    d = x.shape[-1]
+    assert d % 4 == 0
+    da = d // 2
+    inv = rope_inv_freq(da, theta, ntk)
+    y_pos, x_pos, is_text = token_coords(n_text, H, W)
+    img = ~is_text
+    for axis, pos in ((0, y_pos), (1, x_pos)):
+        ang = pos[img][:, None] * inv[None, :]          # [N, da/2]
+        c, s_ = np.cos(ang), np.sin(ang)
+        a = x[..., img, axis * da + 0:axis * da + da:2].copy()
+        b = x[..., img, axis * da + 1:axis * da + da:2].copy()
+        x[..., img, axis * da + 0:axis * da + da:2] = a * c - b * s_
+        x[..., img, axis * da + 1:axis * da + da:2] = a * s_ + b * c
+    return x
+
+
+def clear_attention_forward_rope(q, k, v, n_text: int, H: int, W: int, r: int, theta: float = 10000.0,
+                                 ntk: float = 1.0, scale=None, window: str = "circle"):
+    """The plain forward on rope_2d(q) and rope_2d(k) (v unchanged). Returns (O, LSE) in float64."""
+    return clear_attention_forward(rope_2d(q, n_text, H, W, theta, ntk), rope_2d(k, n_text, H, W, theta, ntk), v,
+                                   n_text, H, W, r, scale=scale, window=window)
