@@ -362,6 +362,42 @@ def time_fp8_forward(L, peak, stream, seed):
     return out
 
 
+def time_rope_forward(L, peak, hbm, stream, seed):
+    """The forward on rotary-embedded q and k (clear_attn_fwd_rope, NTK factor 10) on the headline
+    workload and on F2048 r=16, against the plain forward on the same inputs. The rotation pass is
+    HBM-bound: it reads q and k and writes their rotated copies once, 4 * B*heads*T*d bf16 bytes;
+    its time is the difference of the two medians."""
+    out = {}
+    for name in ("8k_r8", "flux2048_r16"):
+        wl = WORKLOADS[name]
+        q, k, v = make_inputs(wl, seed=seed, device="cuda")
+        o = torch.empty_like(v)
+        lse = torch.empty((wl.B, wl.heads, wl.T), dtype=torch.float32, device="cuda")
+        p = L.make_params(wl.B, wl.heads, wl.n_text, wl.H, wl.W, wl.d, wl.r)
+        ws = torch.empty(L.rope_workspace_size(p), dtype=torch.uint8, device="cuda")
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if q_bytes(wl) < (128 << 20) else None
+        ms_rope = _median_call_ms(lambda: L.clear_attn_fwd_rope(q, k, v, wl.n_text, wl.H, wl.W, wl.r, ntk=10.0, o=o,
+                                                                lse=lse, workspace=ws, stream=stream),
+                                  stream, flush=flush)
+        ms_plain = _median_call_ms(lambda: L.clear_attn_fwd(q, k, v, wl.n_text, wl.H, wl.W, wl.r, o=o, lse=lse,
+                                                            workspace=ws, stream=stream), stream, flush=flush)
+        useful, _ = _flops(L, wl)
+        rot_bytes = 4 * q_bytes(wl)
+        rot_ms = max(ms_rope - ms_plain, 1e-6)
+        out[name] = {"ms_per_call": ms_rope, "plain_forward_ms": ms_plain, "rotation_ms": rot_ms,
+                     "rotation_gbs": rot_bytes / (rot_ms * 1e-3) / 1e9,
+                     "rotation_frac_of_hbm": rot_bytes / (rot_ms * 1e-3) / 1e9 / hbm if hbm else None,
+                     "rotation_bytes": rot_bytes,
+                     "useful_tflops": useful / (ms_rope * 1e-3) / 1e12,
+                     "frac_of_peak": useful / (ms_rope * 1e-3) / 1e12 / peak}
+        del q, k, v, o, lse, ws, flush
+        torch.cuda.empty_cache()
+    if L.clear_attn_check() != 0:
+        raise RuntimeError("device error timing the RoPE forward")
+    out["l2"] = "flushed between calls below 128 MB of q, else inputs larger than L2"
+    return out
+
+
 def time_patch_parallel(L, stream, seed):
     """Patch-parallel split of the FLUX 2048^2 call (128 x 128 grid, r=16) into 2 and 4 row stripes,
     every stripe's kernels run in turn on this one GPU (the halo exchange and text-row all-gather
@@ -511,7 +547,8 @@ def run_clear(args):
     if not args.no_configs and rank == 0:
         extras = {"mixed_batch": time_mixed_batch(L, peak, stream, seed=4000),
                   "patch_parallel": time_patch_parallel(L, stream, seed=4001),
-                  "fp8_scores": time_fp8_forward(L, peak, stream, seed=4002)}
+                  "fp8_scores": time_fp8_forward(L, peak, stream, seed=4002),
+                  "rope": time_rope_forward(L, peak, hbm, stream, seed=4003)}
         torch.cuda.empty_cache()
 
     cpu = None

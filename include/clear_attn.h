@@ -197,6 +197,36 @@ CLEAR_API clear_status_t clear_attn_fwd_fp8(const clear_attn_params_t* params, c
                                             const void* v, const float* qk_descale, void* o, float* lse,
                                             void* workspace, size_t workspace_bytes, void* stream);
 
+/* Rotary position embedding applied by clear_attn_fwd_rope. */
+typedef struct {
+  float theta;  /* RoPE base, > 1 (10000 in RoFormer) */
+  float ntk;    /* NTK-aware scale factor alpha > 0 (1: plain RoPE; the review lists 10 for CLEAR) */
+} clear_attn_rope_t;
+
+/* Workspace bytes of clear_attn_fwd_rope: the forward's, the (cos, sin) table, the rotated q and k
+ * (2 * B * heads * T * d bf16 values). */
+CLEAR_API size_t clear_attn_fwd_rope_workspace_size(const clear_attn_params_t* params, clear_status_t* status);
+
+/*
+ * The forward on rotary-embedded q and k: one streaming pass rotates q and k (HBM-bound, each
+ * element read and written once, rounded to bf16 once) into the workspace, then the CLEAR forward
+ * of clear_attn_fwd runs on the rotated copies; v is used as given. The rotary embedding is axial
+ * 2D with interleaved pairs (RoFormer's rotary embedding and NTK-aware scaled RoPE, both cited by
+ * the paper; the pith.science review of "CLEAR: Conv-Like Linearization Revs Pre-Trained Diffusion
+ * Transformers Up" lists the NTK scale factor 10): image token (y, x) has head dims [0, d/2)
+ * rotated by y and [d/2, d) by x, pair (2i, 2i+1) of an axis by the angle
+ * position * base^(-2i/(d/2)), base = theta * ntk^((d/2)/(d/2 - 2)), (a, b) -> (a cos - b sin,
+ * a sin + b cos); text tokens are not rotated. The (cos, sin) table is evaluated on the device in
+ * double and rounded to fp32. Tensors as clear_attn_fwd (contiguous; d = 64 or 128); the inputs are
+ * not modified. workspace: clear_attn_fwd_rope_workspace_size bytes, 256-byte aligned, written on
+ * `stream` (calls that overlap on the GPU need their own workspaces); no host synchronisation, so
+ * the call can be captured in a CUDA graph. CLEAR_ERR_INVALID_ARG for theta <= 1, ntk <= 0 or
+ * non-finite values; otherwise as clear_attn_fwd.
+ */
+CLEAR_API clear_status_t clear_attn_fwd_rope(const clear_attn_params_t* params, const clear_attn_rope_t* rope,
+                                             const void* q, const void* k, const void* v, void* o, float* lse,
+                                             void* workspace, size_t workspace_bytes, void* stream);
+
 /*
  * Mixed-resolution batch forward: n_items problems of their own (n_text, H, W) in ONE launch (their
  * pairs form one work list), e.g. a batch holding 1024^2 and 2048^2 images at once. Each item is the

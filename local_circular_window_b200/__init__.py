@@ -13,7 +13,7 @@ _EXPORTS = {
     "device_diag", "forward_shape", "ClearStripe", "make_stripe", "clear_attn_fwd_stripe", "clear_attn_text_merge",
     "fwd_host_workspace_size", "fwd_workspace_size", "header_functions", "item_tiles", "lib", "make_params",
     "pair_counts", "selftest_expiry", "status_string", "version", "clear_attn_fwd_varlen", "varlen_workspace_size",
-    "varlen_tokens", "clear_attn_fwd_fp8",
+    "varlen_tokens", "clear_attn_fwd_fp8", "clear_attn_fwd_rope", "rope_workspace_size", "ClearRope",
 }
 
 

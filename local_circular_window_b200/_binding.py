@@ -79,6 +79,14 @@ _lib.clear_attn_fwd_stripe_workspace_size.restype = ctypes.c_size_t
 _lib.clear_attn_fwd_stripe_workspace_size.argtypes = [_P, _S, ctypes.POINTER(_i)]
 _lib.clear_attn_fwd_stripe.restype = _i
 _lib.clear_attn_fwd_stripe.argtypes = [_P, _S, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+class ClearRope(ctypes.Structure):
+    _fields_ = [("theta", ctypes.c_float), ("ntk", ctypes.c_float)]
+
+
+_lib.clear_attn_fwd_rope_workspace_size.restype = ctypes.c_size_t
+_lib.clear_attn_fwd_rope_workspace_size.argtypes = [_P, ctypes.POINTER(_i)]
+_lib.clear_attn_fwd_rope.restype = _i
+_lib.clear_attn_fwd_rope.argtypes = [_P, ctypes.POINTER(ClearRope), _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 _lib.clear_attn_fwd_fp8.restype = _i
 _lib.clear_attn_fwd_fp8.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 _lib.clear_attn_fwd_varlen_workspace_size.restype = ctypes.c_size_t
@@ -340,6 +348,39 @@ def clear_attn_fwd_fp8(q8, k8, v, qk_descale, n_text: int, H: int, W: int, r: in
                                      _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_ptr(stream))
     if status != CLEAR_OK:
         raise ClearError(status, "clear_attn_fwd_fp8")
+    return o, lse
+
+
+def rope_workspace_size(p: ClearParams) -> int:
+    st = _i(0)
+    n = _lib.clear_attn_fwd_rope_workspace_size(ctypes.byref(p), ctypes.byref(st))
+    if st.value != CLEAR_OK:
+        raise ClearError(st.value, "clear_attn_fwd_rope_workspace_size")
+    return n
+
+
+def clear_attn_fwd_rope(q, k, v, n_text: int, H: int, W: int, r: int, theta: float = 10000.0, ntk: float = 1.0,
+                        o=None, lse=None, workspace=None, stream=None, window="circle"):
+    """Forward on rotary-embedded q and k through clear_attn_fwd_rope: one streaming pass rotates q
+    and k (axial 2D RoPE with the NTK-aware base) into the workspace, then the forward runs on the
+    rotated copies; the inputs are not modified. Tensors as clear_attn_fwd. Returns (o, lse)."""
+    B, heads, T, d = q.shape
+    if T != n_text + H * W:
+        raise ValueError("T must equal n_text + H * W")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_qkv(name, t, q.shape)
+    p = make_params(B, heads, n_text, H, W, d, r, window)
+    rope = ClearRope(theta, ntk)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, heads, T), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(rope_workspace_size(p), dtype=torch.uint8, device=q.device)
+    status = _lib.clear_attn_fwd_rope(ctypes.byref(p), ctypes.byref(rope), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                      _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    if status != CLEAR_OK:
+        raise ClearError(status, "clear_attn_fwd_rope")
     return o, lse
 
 

@@ -14,6 +14,7 @@
 #include "clear_attn.h"
 #include "clear_bwd.cuh"
 #include "clear_fwd.cuh"
+#include "clear_rope.cuh"
 #include "clear_sched.cuh"
 
 using namespace clear;
@@ -361,6 +362,87 @@ clear_status_t launch_fwd_f8(const Geom& g, const void* q8, const void* k8, cons
     if (cudaGetLastError() != cudaSuccess) return CLEAR_ERR_CUDA;
   }
   return CLEAR_OK;
+}
+
+// Rotary embedding: one (cos, sin) table for both axes, [max(H, W) positions][d/4 pairs]; pair i of
+// an axis turns by position * base^(-2i/(d/2)) with the NTK-aware base theta * ntk^((d/2)/(d/2 - 2)).
+struct RopeTable {
+  int n = 0;
+  size_t bytes = 0;
+};
+
+RopeTable rope_table_shape(const Geom& g) {
+  RopeTable t;
+  t.n = g.H > g.W ? g.H : g.W;
+  t.bytes = (size_t)t.n * (g.d / 4) * sizeof(float2);
+  return t;
+}
+
+// Workspace of the rotary forward: the forward's own, the table, the rotated q, the rotated k.
+struct RopeWorkspace {
+  size_t tab_off, q_off, k_off, total;
+};
+
+RopeWorkspace rope_workspace_layout(const Geom& g) {
+  RopeWorkspace w;
+  const size_t qk = (size_t)g.BH * g.T * g.d * sizeof(__nv_bfloat16);
+  w.tab_off = align256(fwd_workspace_layout(g).total);
+  w.q_off = w.tab_off + align256(rope_table_shape(g).bytes);
+  w.k_off = w.q_off + align256(qk);
+  w.total = w.k_off + align256(qk);
+  return w;
+}
+
+size_t rope_workspace_bytes(const Geom& g) { return rope_workspace_layout(g).total; }
+
+// Launch shape of the rotation: a grid-stride loop over every chunk, kRopeUnroll chunks in flight
+// per thread, as many blocks as are resident at once on the device (no tail wave).
+template <int D>
+unsigned rope_grid(long long chunks, int num_sms) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, clear_rope_kernel<D>, kRopeThreads, 0) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  const long long per_block = (long long)kRopeThreads * kRopeUnroll;
+  const long long need = (2 * chunks + per_block - 1) / per_block;
+  const long long cap = (long long)num_sms * per_sm;
+  return (unsigned)(need < cap ? need : cap);
+}
+
+clear_status_t launch_rope(const Geom& g, const clear_attn_rope_t& rope, const void* q, const void* k, void* ws,
+                           int num_sms, cudaStream_t stream) {
+  const RopeWorkspace wl = rope_workspace_layout(g);
+  char* base = static_cast<char*>(ws);
+  RopeTableParams tp{};
+  tp.tab = reinterpret_cast<float2*>(base + wl.tab_off);
+  tp.n = rope_table_shape(g).n;
+  tp.np = g.d / 4;
+  const int da = g.d / 2;
+  const double rope_base = (double)rope.theta * std::pow((double)rope.ntk, (double)da / (da - 2.0));
+  for (int i = 0; i < tp.np; ++i) tp.inv_freq[i] = std::pow(rope_base, -2.0 * i / da);
+  clear_rope_table_kernel<<<(unsigned)((tp.n * tp.np + kRopeThreads - 1) / kRopeThreads), kRopeThreads, 0, stream>>>(
+      tp);
+  if (cudaGetLastError() != cudaSuccess) return CLEAR_ERR_CUDA;
+  RopeParams p{};
+  p.src[0] = static_cast<const uint4*>(q);
+  p.src[1] = static_cast<const uint4*>(k);
+  p.dst[0] = reinterpret_cast<uint4*>(base + wl.q_off);
+  p.dst[1] = reinterpret_cast<uint4*>(base + wl.k_off);
+  p.tab = reinterpret_cast<const float4*>(base + wl.tab_off);
+  p.chunks = (long long)g.BH * g.T * (g.d / 8);
+  p.T = g.T;
+  p.n_text = g.n_text;
+  p.W = g.W;
+  if (p.chunks == 0) return CLEAR_OK;
+  if (g.d == 128)
+    clear_rope_kernel<128><<<rope_grid<128>(p.chunks, num_sms), kRopeThreads, 0, stream>>>(p);
+  else
+    clear_rope_kernel<64><<<rope_grid<64>(p.chunks, num_sms), kRopeThreads, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? CLEAR_OK : CLEAR_ERR_CUDA;
+}
+
+bool rope_ok(const clear_attn_rope_t* rope) {
+  return rope && std::isfinite(rope->theta) && rope->theta > 1.f && std::isfinite(rope->ntk) && rope->ntk > 0.f;
 }
 
 // Device address of g_noalloc_scratch on the current device. The symbol's name is only a host-side
@@ -780,6 +862,36 @@ clear_status_t clear_attn_fwd_fp8(const clear_attn_params_t* params, const void*
   const clear_status_t st = check_device(&num_sms);
   if (st != CLEAR_OK) return st;
   return launch_fwd_f8(c.g, q8, k8, v, qk_descale, o, lse, workspace, num_sms, static_cast<cudaStream_t>(stream));
+}
+
+size_t clear_attn_fwd_rope_workspace_size(const clear_attn_params_t* params, clear_status_t* status) {
+  const Checked c = check_params(params);
+  if (status) *status = c.st;
+  if (c.st != CLEAR_OK) return 0;
+  return rope_workspace_bytes(c.g);
+}
+
+clear_status_t clear_attn_fwd_rope(const clear_attn_params_t* params, const clear_attn_rope_t* rope, const void* q,
+                                   const void* k, const void* v, void* o, float* lse, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  const Checked c = check_params(params);
+  if (c.st != CLEAR_OK) return c.st;
+  if (!rope_ok(rope)) return CLEAR_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return CLEAR_ERR_INVALID_ARG;
+  if (workspace_bytes < rope_workspace_bytes(c.g) || !workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return CLEAR_ERR_WORKSPACE;
+  int num_sms = 0;
+  const clear_status_t st = check_device(&num_sms);
+  if (st != CLEAR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const clear_status_t rs = launch_rope(c.g, *rope, q, k, workspace, num_sms, s);
+  if (rs != CLEAR_OK) return rs;
+  const RopeWorkspace wl = rope_workspace_layout(c.g);
+  const TensorStrides cs = contiguous_strides(c.g);
+  const TensorStrides st4[4] = {cs, cs, cs, cs};
+  char* base = static_cast<char*>(workspace);
+  return run_fwd(c.g, st4, base + wl.q_off, base + wl.k_off, v, o, lse, workspace, s);
 }
 
 size_t clear_attn_fwd_varlen_workspace_size(const clear_attn_params_t* params, int n_items, const int* item_shapes,

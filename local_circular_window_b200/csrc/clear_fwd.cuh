@@ -154,8 +154,10 @@ struct FwdLayout {
   static constexpr int bODone = bMsgEmpty + 4;           // + half: last P V of the half's pair done
   static constexpr int bOReady = bODone + 2;             // + half: every P V done (one phase per tile)
   static constexpr int kNumBars = bOReady + 2;
-  static constexpr int kMsg = kBars + kNumBars * 8;      // int4[2][2] mailbox: {kind, a, b, flags | ordinal << 8}
+  static constexpr int kMsg = (kBars + kNumBars * 8 + 15) & ~15;  // int4[2][2] mailbox: {kind, a, b, flags | ordinal << 8}
   static constexpr int kRing = kMsg + 64;                // int4[kTileRing]: {kind | flags << 4 | last << 12, a, b, bh}
+  static_assert(kMsg % 16 == 0 && kRing % 16 == 0, "int4 mailbox and ring need 16-byte alignment");
+  static_assert(kQ % 1024 == 0 && kK % 1024 == 0 && kV % 1024 == 0, "swizzled tiles need 1024-byte alignment");
   static constexpr int kMisc = kRing + kTileRing * 16;
   static constexpr int kWTab = kMisc + 16;               // int[kMaxRTable] (tile enumeration)
   static constexpr int kHwTab = kWTab + kMaxRTable * 4;  // int16[hw_table_size(r, H)] (masks)

@@ -50,7 +50,7 @@ Revs Pre-Trained Diffusion Transformers Up"):
    above on q = decode(q8) * s_q and k = decode(k8) * s_k: the scores are those of the dequantized
    inputs, the rest is unchanged.
 
-9. Rotary position embedding applied to q and k before the scores (a fused-prologue variant): the
+9. Rotary position embedding applied to q and k before the scores (an optional first step): the
    review lists an NTK-aware RoPE scale factor of 10 among the free parameters ["Assumptions &
    free parameters"] and the paper cites RoFormer (rotary embedding: each pair of adjacent head
    dims (2i, 2i+1) rotated by position * base^(-2i/d)) and NTK-aware scaled RoPE (the base raised
