@@ -518,15 +518,16 @@ struct DkvLayout {
   static constexpr int kQStride = 2 * kTileBytes;
   static constexpr int kVec = kQ + 2 * kQStride;         // float lse2/dvec [2][2][128]
   static constexpr int kBars = kVec + 4 * kTile * 4;
-  static constexpr int bKVFull = 0, bKVEmpty = 1, bQFull = 2 /* + buf */, bQEmpty = 4 /* + buf */, bSFull = 6,
-                       bPFull = 7, bAccDone = 8;
-  static constexpr int kNumBars = 9;
+  static constexpr int bKVFull = 0, bKVEmpty = 1, bQFull = 2 /* + buf */, bQEmpty = 4 /* + buf */,
+                       bSFull = 6 /* + half */, bPFull = 8 /* + half */, bAccDone = 10;
+  static constexpr int kNumBars = 11;
   static constexpr int kMisc = kBars + kNumBars * 8;
   static constexpr int kWTab = kMisc + 16;
   static constexpr int kTotal = kWTab + kMaxRTable * 4;
   static constexpr int kAlloc = kTotal + 1024;
-  // TMEM: S^T (P^T as bf16 pairs over its first 64 columns once the softmax has read it), dP^T
-  // (dS^T likewise), and the dV, dK accumulators.
+  // TMEM: S^T of the partner tile's two 64-query halves at columns 0 and 64 (P^T of half h as bf16
+  // pairs over the first 32 columns of its S^T once the softmax has read it), dP^T likewise at 128
+  // and 192 (dS^T over them), and the dV, dK accumulators.
   static constexpr uint32_t kTmemS = 0, kTmemDP = 128, kTmemDV = 256, kTmemDK = 256 + D, kTmemCols = 512;
 };
 
@@ -534,7 +535,9 @@ struct DkvLayout {
 // mask is symmetric, so they are the key tiles KeyIter lists for a query tile at the same place):
 // S^T = K Q^T and dP^T = V dO^T into TMEM, P^T = 2^(S^T c - lse2) and dS^T = P^T (dP^T - D)
 // written back over them as bf16, then dV += P^T dO and dK += dS^T Q with the A operand read from
-// TMEM. Partner Q / dO tiles are double-buffered.
+// TMEM. Partner Q / dO tiles are double-buffered. Each partner tile is taken as two halves of 64
+// queries with barriers of their own, so that the tensor pipe works on one half (dV, dK of half a,
+// then S^T, dP^T of the next tile's half a) while the softmax turns the other into P^T, dS^T.
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_constant__ CUtensorMap tm_q_img,
@@ -561,8 +564,10 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
       mbar_init(&bars[L::bQFull + b], 1);
       mbar_init(&bars[L::bQEmpty + b], 1);
     }
-    mbar_init(&bars[L::bSFull], 1);
-    mbar_init(&bars[L::bPFull], 256);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&bars[L::bSFull + h], 1);
+      mbar_init(&bars[L::bPFull + h], 256);
+    }
     mbar_init(&bars[L::bAccDone], 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -615,41 +620,65 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
   } else if (warp == 9) {
     regs_dec<kBwdRegsLow>();
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);  // one half: 64 partner queries
       constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t k_addr = smem_u32(smem + L::kK);
       const uint32_t v_addr = smem_u32(smem + L::kV);
-      uint32_t kv_full_ph = 0, p_full_ph = 0, c = 0;
+      constexpr uint32_t kHalfRows = 64 * 128;  // bytes of 64 rows in each 64-column block of a tile
+      uint32_t kv_full_ph = 0, p_full_ph[2] = {0, 0}, c = 0;
+      // S^T and dP^T of half h of partner tile cc. They overwrite that half's P^T and dS^T of the
+      // tile before, whose readers (dV, dK of the half) were issued before, by this thread, and
+      // run first.
+      auto scores = [&](uint32_t cc, int h) {
+        const uint32_t qb = cc & 1;
+        const uint32_t q_addr = smem_u32(smem + L::kQ + qb * L::kQStride) + h * kHalfRows;
+        const uint32_t do_addr = smem_u32(smem + L::kDO + qb * L::kQStride) + h * kHalfRows;
+        mma_kmajor<D>(tmem + L::kTmemS + 64 * h, k_addr, q_addr, idesc_s);    // S^T = K Q^T
+        mma_kmajor<D>(tmem + L::kTmemDP + 64 * h, v_addr, do_addr, idesc_s);  // dP^T = V dO^T
+        umma_commit(&bars[L::bSFull + h]);
+      };
+      // dV += P^T dO and dK += dS^T Q over the 64 partner queries of half h (four K16 steps each).
+      auto accumulate = [&](uint32_t cc, int h, bool first) {
+        const uint32_t qb = cc & 1;
+        const uint64_t do_desc = smem_desc_sw128(smem_u32(smem + L::kDO + qb * L::kQStride), kHalfBytes, 1024);
+        const uint64_t q_desc = smem_desc_sw128(smem_u32(smem + L::kQ + qb * L::kQStride), kHalfBytes, 1024);
+        #pragma unroll
+        for (int j = 0; j < 4; ++j)
+          umma_ts(tmem + L::kTmemDV, tmem + L::kTmemS + 64 * h + 8 * j,
+                  do_desc + (uint64_t)(((4 * h + j) * 2048) >> 4), idesc_acc, (first && j == 0) ? 0u : 1u);
+        #pragma unroll
+        for (int j = 0; j < 4; ++j)
+          umma_ts(tmem + L::kTmemDK, tmem + L::kTmemDP + 64 * h + 8 * j,
+                  q_desc + (uint64_t)(((4 * h + j) * 2048) >> 4), idesc_acc, (first && j == 0) ? 0u : 1u);
+      };
       for (long long w = blockIdx.x; w < p.n_work; w += gridDim.x) {
         const WorkItem it = decode_work(g, w);
         const int n = count_key_tiles(g, it);
         if (!mbar_wait(&bars[L::bKVFull], kv_full_ph, abort_flag, kDevTimeoutMma)) goto mma_done;
         kv_full_ph ^= 1;
+        if (n > 0) {
+          if (!mbar_wait(&bars[L::bQFull + (c & 1)], (c >> 1) & 1, abort_flag, kDevTimeoutMma)) goto mma_done;
+          tc_fence_after();
+          scores(c, 0);
+          scores(c, 1);
+        }
         for (int i = 0; i < n; ++i, ++c) {
-          const uint32_t qb = c & 1;
-          const uint32_t q_addr = smem_u32(smem + L::kQ + qb * L::kQStride);
-          const uint32_t do_addr = smem_u32(smem + L::kDO + qb * L::kQStride);
-          if (!mbar_wait(&bars[L::bQFull + qb], (c >> 1) & 1, abort_flag, kDevTimeoutMma)) goto mma_done;
-          tc_fence_after();
-          // S^T and dP^T overwrite the previous tile's P^T and dS^T: the products reading those
-          // were issued before, by this thread, and run first.
-          mma_kmajor<D>(tmem + L::kTmemS, k_addr, q_addr, idesc_s);    // S^T = K Q^T
-          mma_kmajor<D>(tmem + L::kTmemDP, v_addr, do_addr, idesc_s);  // dP^T = V dO^T
-          umma_commit(&bars[L::bSFull]);
-          if (!mbar_wait(&bars[L::bPFull], p_full_ph, abort_flag, kDevTimeoutMma)) goto mma_done;
-          p_full_ph ^= 1;
-          tc_fence_after();
-          const uint64_t do_desc = smem_desc_sw128(do_addr, kHalfBytes, 1024);
-          const uint64_t q_desc = smem_desc_sw128(q_addr, kHalfBytes, 1024);
-          #pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk)  // dV += P^T dO
-            umma_ts(tmem + L::kTmemDV, tmem + L::kTmemS + kk * 8, do_desc + (uint64_t)((kk * 2048) >> 4), idesc_acc,
-                    (i > 0 || kk > 0) ? 1u : 0u);
-          #pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk)  // dK += dS^T Q
-            umma_ts(tmem + L::kTmemDK, tmem + L::kTmemDP + kk * 8, q_desc + (uint64_t)((kk * 2048) >> 4), idesc_acc,
-                    (i > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&bars[L::bQEmpty + qb]);
+          const bool more = i + 1 < n;
+          for (int h = 0; h < 2; ++h) {
+            if (!mbar_wait(&bars[L::bPFull + h], p_full_ph[h], abort_flag, kDevTimeoutMma)) goto mma_done;
+            p_full_ph[h] ^= 1;
+            tc_fence_after();
+            accumulate(c, h, i == 0 && h == 0);
+            if (h == 1) umma_commit(&bars[L::bQEmpty + (c & 1)]);  // last reads of this Q / dO buffer issued
+            if (more) {
+              if (h == 0) {
+                if (!mbar_wait(&bars[L::bQFull + ((c + 1) & 1)], ((c + 1) >> 1) & 1, abort_flag, kDevTimeoutMma))
+                  goto mma_done;
+                tc_fence_after();
+              }
+              scores(c + 1, h);
+            }
+          }
         }
         umma_commit(&bars[L::bAccDone]);
         umma_commit(&bars[L::bKVEmpty]);
@@ -663,7 +692,7 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
     const int row = threadIdx.x & 127;       // key row of the stationary tile = TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     constexpr int kHalfD = D / 2;            // output columns of this warpgroup
-    uint32_t s_full_ph = 0, acc_ph = 0;
+    uint32_t s_full_ph[2] = {0, 0}, acc_ph = 0;
     const float sl2 = p.scale_log2;
     uint32_t tile_counter = 0;
     for (long long w = blockIdx.x; w < p.n_work; w += gridDim.x) {
@@ -703,25 +732,21 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
           lse_s[c] = ok ? p.l2vec[qrow] : INFINITY;
           dv_s[c] = ok ? p.dvec[qrow] : 0.f;
         }
-        if (!mbar_wait(&bars[L::bSFull], s_full_ph, abort_flag, kDevTimeoutSoftmax)) goto softmax_done;
-        s_full_ph ^= 1;
-        tc_fence_after();
-        uint32_t sr[2][32], dr[2][32];
-        tmem_ld32(tmem + lane_base + L::kTmemS + 64 * wg, sr[0]);
-        tmem_ld32(tmem + lane_base + L::kTmemS + 64 * wg + 32, sr[1]);
-        tmem_ld32(tmem + lane_base + L::kTmemDP + 64 * wg, dr[0]);
-        tmem_ld32(tmem + lane_base + L::kTmemDP + 64 * wg + 32, dr[1]);
-        tmem_wait_ld();
-        // Every thread has read its S^T / dP^T columns (P^T / dS^T overwrite columns of the other
-        // warpgroup's half) and warpgroup 0 has stored the partner statistics.
-        tc_fence_before();
-        named_bar_sync(1, 256);
-        tc_fence_after();
-        // P^T = 2^(s c - lse2) on kept pairs, dS^T = P^T (dP^T - D), as bf16 pairs.
-        uint32_t pw[32], dw[32];
-        #pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          const int gch = 2 * wg + ch;  // 32-column chunk of the tile
+        for (int h = 0; h < 2; ++h) {  // the tile's two 64-query halves
+          if (!mbar_wait(&bars[L::bSFull + h], s_full_ph[h], abort_flag, kDevTimeoutSoftmax)) goto softmax_done;
+          s_full_ph[h] ^= 1;
+          tc_fence_after();
+          const int gch = 2 * h + wg;  // this warpgroup's 32-column chunk of the tile
+          uint32_t sr[32], dr[32];
+          tmem_ld32(tmem + lane_base + L::kTmemS + 32 * gch, sr);
+          tmem_ld32(tmem + lane_base + L::kTmemDP + 32 * gch, dr);
+          tmem_wait_ld();
+          // Every thread has read its S^T / dP^T columns (warpgroup 1's P^T / dS^T overwrite
+          // columns warpgroup 0 reads) and warpgroup 0 has stored the partner statistics.
+          tc_fence_before();
+          named_bar_sync(1, 256);
+          tc_fence_after();
+          // P^T = 2^(s c - lse2) on kept pairs, dS^T = P^T (dP^T - D), as bf16 pairs.
           uint32_t keep = 0xffffffffu;
           if (t.flags != kFull) {
             if (t.kind == kLinear) {
@@ -732,24 +757,25 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
                      (rect_row_bits(g, wtab, yk, xk, t.a + 2 * gch + 1, t.b) << 16);
             }
           }
+          uint32_t pw[16], dw[16];
           #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const int c = gch * 32 + e;
-            const float x0 = ((keep >> e) & 1u) ? __uint_as_float(sr[ch][e]) : -INFINITY;
-            const float x1 = ((keep >> (e + 1)) & 1u) ? __uint_as_float(sr[ch][e + 1]) : -INFINITY;
+            const float x0 = ((keep >> e) & 1u) ? __uint_as_float(sr[e]) : -INFINITY;
+            const float x1 = ((keep >> (e + 1)) & 1u) ? __uint_as_float(sr[e + 1]) : -INFINITY;
             const float p0 = ex2_approx(fmaf(x0, sl2, -lse_s[c]));
             const float p1 = ex2_approx(fmaf(x1, sl2, -lse_s[c + 1]));
-            const float d0 = p0 * (__uint_as_float(dr[ch][e]) - dv_s[c]);
-            const float d1 = p1 * (__uint_as_float(dr[ch][e + 1]) - dv_s[c + 1]);
-            pw[ch * 16 + e / 2] = pack_bf16x2(p0, p1);
-            dw[ch * 16 + e / 2] = pack_bf16x2(d0, d1);
+            const float d0 = p0 * (__uint_as_float(dr[e]) - dv_s[c]);
+            const float d1 = p1 * (__uint_as_float(dr[e + 1]) - dv_s[c + 1]);
+            pw[e / 2] = pack_bf16x2(p0, p1);
+            dw[e / 2] = pack_bf16x2(d0, d1);
           }
+          tmem_st16(tmem + lane_base + L::kTmemS + 64 * h + 16 * wg, pw);
+          tmem_st16(tmem + lane_base + L::kTmemDP + 64 * h + 16 * wg, dw);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&bars[L::bPFull + h]);
         }
-        tmem_st32(tmem + lane_base + L::kTmemS + 32 * wg, pw);
-        tmem_st32(tmem + lane_base + L::kTmemDP + 32 * wg, dw);
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&bars[L::bPFull]);
       }
       if (!mbar_wait(&bars[L::bAccDone], acc_ph, abort_flag, kDevTimeoutSoftmax)) goto softmax_done;
       acc_ph ^= 1;
