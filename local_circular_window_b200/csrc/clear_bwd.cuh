@@ -225,8 +225,9 @@ struct DqLayout {
   static constexpr int kBars = kDS + kTile * kTile * 2;
   static constexpr int bQFull = 0, bQEmpty = 1, bSdpFull = 2, bSdpFree = 3, bDsFull = 4, bDsEmpty = 5,
                        bAccDone = 6;
-  static constexpr int bKFull = 7, bVFull = bKFull + NST, bKVEmpty = bVFull + NST;
-  static constexpr int kNumBars = bKVEmpty + NST;
+  // K and V ring slots are released separately: V after dP (its only reader), K after dQ.
+  static constexpr int bKFull = 7, bVFull = bKFull + NST, bKEmpty = bVFull + NST, bVEmpty = bKEmpty + NST;
+  static constexpr int kNumBars = bVEmpty + NST;
   static constexpr int kMisc = kBars + kNumBars * 8;
   static constexpr int kWTab = kMisc + 16;
   static constexpr int kTotal = kWTab + kMaxRTable * 4;
@@ -263,7 +264,8 @@ clear_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_c
     for (int s = 0; s < NST; ++s) {
       mbar_init(&bars[L::bKFull + s], 1);
       mbar_init(&bars[L::bVFull + s], 1);
-      mbar_init(&bars[L::bKVEmpty + s], 1);
+      mbar_init(&bars[L::bKEmpty + s], 1);
+      mbar_init(&bars[L::bVEmpty + s], 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -300,18 +302,22 @@ clear_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_c
         ki.init(g, it);
         KeyTile t;
         while (ki.next(&t)) {
-          if (!mbar_wait(&bars[L::bKVEmpty + stage], ring_ph ^ 1, abort_flag, kDevTimeoutTmaEmpty)) goto producer_done;
-          mbar_arrive_expect_tx(&bars[L::bKFull + stage], L::kTileBytes);
-          load_tile<D>(smem + L::kK + stage * L::kTileBytes, &tm_k_lin, &tm_k_img, &bars[L::bKFull + stage], t.kind,
-                       t.a, t.b, it.bh);
+          // V first: its slot frees as soon as dP of the tile before has run, so only K's load
+          // waits for the dQ product.
+          if (!mbar_wait(&bars[L::bVEmpty + stage], ring_ph ^ 1, abort_flag, kDevTimeoutTmaEmpty)) goto producer_done;
           mbar_arrive_expect_tx(&bars[L::bVFull + stage], L::kTileBytes);
           load_tile<D>(smem + L::kV + stage * L::kTileBytes, &tm_v_lin, &tm_v_img, &bars[L::bVFull + stage], t.kind,
+                       t.a, t.b, it.bh);
+          if (!mbar_wait(&bars[L::bKEmpty + stage], ring_ph ^ 1, abort_flag, kDevTimeoutTmaEmpty)) goto producer_done;
+          mbar_arrive_expect_tx(&bars[L::bKFull + stage], L::kTileBytes);
+          load_tile<D>(smem + L::kK + stage * L::kTileBytes, &tm_k_lin, &tm_k_img, &bars[L::bKFull + stage], t.kind,
                        t.a, t.b, it.bh);
           if (++stage == NST) { stage = 0; ring_ph ^= 1; }
         }
       }
       for (int s = 0; s < NST; ++s) {
-        if (!mbar_wait(&bars[L::bKVEmpty + stage], ring_ph ^ 1, abort_flag, kDevTimeoutTmaEmpty)) break;
+        if (!mbar_wait(&bars[L::bVEmpty + stage], ring_ph ^ 1, abort_flag, kDevTimeoutTmaEmpty)) break;
+        if (!mbar_wait(&bars[L::bKEmpty + stage], ring_ph ^ 1, abort_flag, kDevTimeoutTmaEmpty)) break;
         if (++stage == NST) { stage = 0; ring_ph ^= 1; }
       }
     producer_done:;
@@ -328,16 +334,19 @@ clear_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_c
       static_assert(NST == 2, "S and dP of the next key tile are issued while dQ still reads this one's K");
       int stage = 0;
       uint32_t ring_ph = 0, q_full_ph = 0, ds_full_ph = 0, sdp_free_ph = 0;
-      // S = Q K^T and dP = dO V^T of key tile j into TMEM (K/V ring slot `stage`), once the softmax
-      // has read the previous pair.
+      // dP = dO V^T and S = Q K^T of key tile j into TMEM (K/V ring slot `stage`), once the softmax
+      // has read the previous pair. dP goes first: V arrives earlier than K (its slot is released
+      // after dP, K's after dQ), and K's load overlaps dP's issue.
       auto issue_sdp = [&](int j, int n) -> bool {
         if (!mbar_wait(&bars[L::bSdpFree], sdp_free_ph ^ 1, abort_flag, kDevTimeoutMma)) return false;
         sdp_free_ph ^= 1;
-        if (!mbar_wait(&bars[L::bKFull + stage], ring_ph, abort_flag, kDevTimeoutMma)) return false;
         if (!mbar_wait(&bars[L::bVFull + stage], ring_ph, abort_flag, kDevTimeoutMma)) return false;
         tc_fence_after();
-        mma_kmajor<D>(tmem + L::kTmemS, q_addr, smem_u32(smem + L::kK + stage * L::kTileBytes), idesc_s);
         mma_kmajor<D>(tmem + L::kTmemDP, do_addr, smem_u32(smem + L::kV + stage * L::kTileBytes), idesc_s);
+        umma_commit(&bars[L::bVEmpty + stage]);
+        if (!mbar_wait(&bars[L::bKFull + stage], ring_ph, abort_flag, kDevTimeoutMma)) return false;
+        tc_fence_after();
+        mma_kmajor<D>(tmem + L::kTmemS, q_addr, smem_u32(smem + L::kK + stage * L::kTileBytes), idesc_s);
         umma_commit(&bars[L::bSdpFull]);
         if (j == n - 1) umma_commit(&bars[L::bQEmpty]);  // Q and dO: last reads issued
         return true;
@@ -361,7 +370,7 @@ clear_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_c
           mma_a_kmajor_b_mnmajor<D>(tmem + L::kTmemAcc, ds_addr, smem_u32(smem + L::kK + cur * L::kTileBytes), idesc_dq,
                                     j > 0);
           umma_commit(&bars[L::bDsEmpty]);
-          umma_commit(&bars[L::bKVEmpty + cur]);
+          umma_commit(&bars[L::bKEmpty + cur]);
           if (j == n - 1) umma_commit(&bars[L::bAccDone]);
         }
       }
