@@ -436,8 +436,15 @@ clear_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_c
             }
           }
         }
-        #pragma unroll
-        for (int c = 0; c < kC; ++c) s[c] = ex2_approx(fmaf(s[c], sl2, -lse2));
+        {
+          const uint64_t sl2x2 = f32x2_pack(sl2, sl2), nlse2 = f32x2_pack(-lse2, -lse2);
+          #pragma unroll
+          for (int c = 0; c < kC; c += 2) {  // P = 2^(s c - lse2) on packed pairs (same results as scalar fp32)
+            const uint64_t x = f32x2_fma(f32x2_pack(s[c], s[c + 1]), sl2x2, nlse2);
+            s[c] = ex2_approx(f32x2_lo(x));
+            s[c + 1] = ex2_approx(f32x2_hi(x));
+          }
+        }
         float dp[kC];
         {
           uint32_t dr[2][32];
@@ -449,8 +456,15 @@ clear_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_c
         }
         tc_fence_before();
         mbar_arrive(&bars[L::bSdpFree]);
-        #pragma unroll
-        for (int c = 0; c < kC; ++c) s[c] = s[c] * (dp[c] - dd);  // dS
+        {
+          const uint64_t ndd2 = f32x2_pack(-dd, -dd);
+          #pragma unroll
+          for (int c = 0; c < kC; c += 2) {  // dS = P (dP - D)
+            const uint64_t ds = f32x2_mul(f32x2_pack(s[c], s[c + 1]), f32x2_add(f32x2_pack(dp[c], dp[c + 1]), ndd2));
+            s[c] = f32x2_lo(ds);
+            s[c + 1] = f32x2_hi(ds);
+          }
+        }
         if (ds_pending) {
           if (!mbar_wait(&bars[L::bDsEmpty], ds_empty_ph, abort_flag, kDevTimeoutSoftmax)) goto softmax_done;
           ds_empty_ph ^= 1;
@@ -767,17 +781,20 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
             }
           }
           uint32_t pw[16], dw[16];
+          const uint64_t sl2x2 = f32x2_pack(sl2, sl2);
           #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
+          for (int e = 0; e < 32; e += 2) {  // packed pairs: the same results as scalar fp32
             const int c = gch * 32 + e;
             const float x0 = ((keep >> e) & 1u) ? __uint_as_float(sr[e]) : -INFINITY;
             const float x1 = ((keep >> (e + 1)) & 1u) ? __uint_as_float(sr[e + 1]) : -INFINITY;
-            const float p0 = ex2_approx(fmaf(x0, sl2, -lse_s[c]));
-            const float p1 = ex2_approx(fmaf(x1, sl2, -lse_s[c + 1]));
-            const float d0 = p0 * (__uint_as_float(dr[e]) - dv_s[c]);
-            const float d1 = p1 * (__uint_as_float(dr[e + 1]) - dv_s[c + 1]);
+            const uint64_t x = f32x2_fma(f32x2_pack(x0, x1), sl2x2, f32x2_pack(-lse_s[c], -lse_s[c + 1]));
+            const float p0 = ex2_approx(f32x2_lo(x));
+            const float p1 = ex2_approx(f32x2_hi(x));
+            const uint64_t d = f32x2_mul(f32x2_pack(p0, p1),
+                                         f32x2_add(f32x2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])),
+                                                   f32x2_pack(-dv_s[c], -dv_s[c + 1])));
             pw[e / 2] = pack_bf16x2(p0, p1);
-            dw[e / 2] = pack_bf16x2(d0, d1);
+            dw[e / 2] = pack_bf16x2(f32x2_lo(d), f32x2_hi(d));
           }
           tmem_st16(tmem + lane_base + L::kTmemS + 64 * h + 16 * wg, pw);
           tmem_st16(tmem + lane_base + L::kTmemDP + 64 * h + 16 * wg, dw);
