@@ -96,6 +96,7 @@ Checked check_stripe(const clear_attn_params_t* p, const clear_attn_stripe_t* s)
   const int tk_lo = p->n_text + s->key_row0 * p->W, tk_hi = p->n_text + s->key_row1 * p->W;
   set_text_key_ranges(&c.g, s->text_keys, tk_lo, tk_hi);
   set_forward_work(&c.g, s->q_row0, s->q_row1);
+  balance_forward_splits(&c.g);
   c.st = CLEAR_OK;
   return c;
 }
@@ -477,7 +478,7 @@ clear_status_t noalloc_geom(Geom* g) {
   if (g->n_text == 0) return CLEAR_OK;
   for (int cap = g->fS; cap >= 1; --cap) {
     Geom t = *g;
-    choose_splits(t.fnC, 2 * kSplitTargetChunks, cap, &t.fS, &t.fcps);
+    choose_splits(t.fnC, t.ftarget, cap, &t.fS, &t.fcps);
     t.n_txt_pairs = (long long)t.BH * t.nTq2 * t.fS;
     if (fwd_workspace_layout(t).total <= kNoAllocScratchBytes) {
       *g = t;

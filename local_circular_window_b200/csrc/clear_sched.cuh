@@ -81,6 +81,7 @@ struct Geom {
   int fnC;           // 64-key chunks a text query row visits (both key ranges below)
   int fnTk;          // 64-key chunks over the text tokens
   int fS, fcps;      // forward text splits and 64-key chunks per split
+  int ftarget;       // chunks per forward text split aimed at (balance_forward_splits)
   long long n_txt_pairs, n_img_pairs;
   // Stripe mode (patch-parallel inference; the defaults are the whole problem): image query rows
   // are rows [qy0, qy1) of the grid only, and text query rows see the keys of token ranges
@@ -165,10 +166,13 @@ CLEAR_HD void set_forward_work(Geom* g, int qy0, int qy1) {
   g->qy1 = qy1;
   g->nqy2 = cdiv(qy1 - qy0, 2 * kQH);
   g->nQ2 = g->nqy2 * g->nqx;
-  choose_splits(g->fnC, 2 * kSplitTargetChunks, kMaxSplits, &g->fS, &g->fcps);
+  g->ftarget = 2 * kSplitTargetChunks;
+  choose_splits(g->fnC, g->ftarget, kMaxSplits, &g->fS, &g->fcps);
   g->n_txt_pairs = (long long)g->BH * g->nTq2 * g->fS;
   g->n_img_pairs = (long long)g->BH * g->nQ2;
 }
+
+CLEAR_HD void balance_forward_splits(Geom* g);
 
 CLEAR_HD Geom make_geom(int B, int heads, int n_text, int H, int W, int d, int r, int window = kCircle) {
   Geom g;
@@ -189,6 +193,7 @@ CLEAR_HD Geom make_geom(int B, int heads, int n_text, int H, int W, int d, int r
   g.fnTk = cdiv(n_text, kFChunk);
   set_text_key_ranges(&g, 1, n_text, g.T);
   set_forward_work(&g, 0, H);
+  balance_forward_splits(&g);
   g.t0 = 0;
   g.tok_total = g.T;
   g.part_row0 = 0;
@@ -501,6 +506,70 @@ CLEAR_HD void count_pair_tiles(const Geom& g, const PairItem& it, const int* tab
   *n_union = nu;
   *n_a = na;
   *n_b = nb;
+}
+
+// Text split count of the forward, chosen with a model of the static round-robin assignment
+// (pair item w runs on CTA w mod kFwdModelSMs, one CTA per SM): an item costs the (key tile,
+// half) products it issues plus a fixed cost per item (kFwdTextItemCost, kFwdImageItemCost; fitted
+// to timings of split counts 1 to 7 on FLUX-shaped 64 x 64 and 128 x 128 grids, where the model
+// then picks the measured best each time), and the split count with the smallest busiest CTA wins
+// (the smaller count on ties). Candidates run from the plain rule (splits of at most
+// 2 * kSplitTargetChunks chunks) up to 8 splits, never above kMaxSplits. With more than 64 image
+// pairs per SM the plain rule is kept: the items are then many and small enough to balance.
+constexpr int kFwdModelSMs = 148;
+constexpr int kFwdTextItemCost = 16;
+constexpr int kFwdImageItemCost = 24;
+
+CLEAR_HD long long forward_makespan(const Geom& g, int S, const int* img_cost, int n_img_cost) {
+  const int cps = cdiv(g.fnC, S);
+  S = cdiv(g.fnC, cps);
+  const long long n = (long long)g.BH * (g.nTq2 * S + n_img_cost);
+  const int G = n < kFwdModelSMs ? (int)n : kFwdModelSMs;
+  long long load[kFwdModelSMs] = {};
+  int bin = 0;
+  for (int pr = 0; pr < g.BH * g.nTq2; ++pr)  // text pairs, then their splits, as decode_pair orders them
+    for (int sp = 0; sp < S; ++sp) {
+      load[bin] += 2 * (imin(g.fnC, (sp + 1) * cps) - sp * cps) + kFwdTextItemCost;
+      if (++bin == G) bin = 0;
+    }
+  for (int bh = 0; bh < g.BH; ++bh)
+    for (int i = 0; i < n_img_cost; ++i) {
+      load[bin] += img_cost[i] + kFwdImageItemCost;
+      if (++bin == G) bin = 0;
+    }
+  long long mx = 0;
+  for (int i = 0; i < G; ++i) mx = load[i] > mx ? load[i] : mx;
+  return mx;
+}
+
+CLEAR_HD void balance_forward_splits(Geom* g) {
+  g->ftarget = 2 * kSplitTargetChunks;
+  choose_splits(g->fnC, g->ftarget, kMaxSplits, &g->fS, &g->fcps);
+  g->n_txt_pairs = (long long)g->BH * g->nTq2 * g->fS;
+  constexpr int kMaxModelPairs = 64 * kFwdModelSMs;
+  if (g->n_text == 0 || g->nQ2 == 0 || (long long)g->BH * g->nQ2 > kMaxModelPairs || g->fS >= 8) return;
+#ifndef __CUDA_ARCH__
+  // (key tile, half) products of each image pair of head 0; every head has the same.
+  static thread_local int cost[kMaxModelPairs];
+  for (int blk = 0; blk < g->nQ2; ++blk) {
+    const PairItem it = decode_pair(*g, g->n_txt_pairs + blk);
+    PairKeyIter ki;
+    ki.init(*g, it, nullptr, 0);
+    KeyTile t;
+    int c = 0;
+    while (ki.next(&t)) c += ((t.flags & kNeedA) ? 1 : 0) + ((t.flags & kNeedB) ? 1 : 0);
+    cost[blk] = c;
+  }
+  int best_s = g->fS;
+  long long best = forward_makespan(*g, g->fS, cost, g->nQ2);
+  for (int s = g->fS + 1; s <= imin(8, kMaxSplits); ++s) {
+    const long long m = forward_makespan(*g, s, cost, g->nQ2);
+    if (m < best) { best = m; best_s = s; }
+  }
+  g->ftarget = cdiv(g->fnC, best_s);
+  choose_splits(g->fnC, g->ftarget, kMaxSplits, &g->fS, &g->fcps);
+  g->n_txt_pairs = (long long)g->BH * g->nTq2 * g->fS;
+#endif
 }
 
 }  // namespace clear
