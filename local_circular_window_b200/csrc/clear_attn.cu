@@ -646,10 +646,17 @@ clear_status_t plan_varlen(const clear_attn_params_t* p, int n_items, const int*
   const int r = p->window == kShifted ? p->r : (p->r < rmax_full ? p->r : rmax_full);
   if (hw_table_size(r, max_h) > kMaxHwTable) return CLEAR_ERR_UNSUPPORTED;
   v->items.resize(n_items);
+  // Text splits by the plain rule: the launch deals every item's pairs round-robin as one list, so
+  // there are many items per SM and the split-balancing model (made for one item alone) only adds
+  // partial writes; measured on five FLUX-shaped mixes, the plain rule was as fast or 0.2-5 % faster.
+  for (int i = 0; i < n_items; ++i) {
+    v->items[i] = make_geom(1, p->heads, shapes[3 * i], shapes[3 * i + 1], shapes[3 * i + 2], p->d, r, p->window);
+    plain_forward_splits(&v->items[i]);
+  }
   v->wbound.assign(2 * (size_t)n_items + 1, 0);
   long long t0 = 0, part = 0, crow = 0, wt = 0;
   for (int i = 0; i < n_items; ++i) {
-    Geom g = make_geom(1, p->heads, shapes[3 * i], shapes[3 * i + 1], shapes[3 * i + 2], p->d, r, p->window);
+    Geom g = v->items[i];
     g.t0 = (int)t0;
     g.tok_total = tok;
     g.part_row0 = part;

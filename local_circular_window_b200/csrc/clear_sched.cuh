@@ -542,24 +542,34 @@ CLEAR_HD long long forward_makespan(const Geom& g, int S, const int* img_cost, i
   return mx;
 }
 
-CLEAR_HD void balance_forward_splits(Geom* g) {
-  g->ftarget = 2 * kSplitTargetChunks;
-  choose_splits(g->fnC, g->ftarget, kMaxSplits, &g->fS, &g->fcps);
-  g->n_txt_pairs = (long long)g->BH * g->nTq2 * g->fS;
-  constexpr int kMaxModelPairs = 64 * kFwdModelSMs;
-  if (g->n_text == 0 || g->nQ2 == 0 || (long long)g->BH * g->nQ2 > kMaxModelPairs || g->fS >= 8) return;
-#ifndef __CUDA_ARCH__
-  // (key tile, half) products of each image pair of head 0; every head has the same.
-  static thread_local int cost[kMaxModelPairs];
-  for (int blk = 0; blk < g->nQ2; ++blk) {
-    const PairItem it = decode_pair(*g, g->n_txt_pairs + blk);
+constexpr int kMaxModelPairs = 64 * kFwdModelSMs;
+
+// (key tile, half) products of each image pair of head 0, g.nQ2 entries; every head has the same.
+CLEAR_HD void image_pair_costs(const Geom& g, int* cost) {
+  for (int blk = 0; blk < g.nQ2; ++blk) {
+    const PairItem it = decode_pair(g, g.n_txt_pairs + blk);
     PairKeyIter ki;
-    ki.init(*g, it, nullptr, 0);
+    ki.init(g, it, nullptr, 0);
     KeyTile t;
     int c = 0;
     while (ki.next(&t)) c += ((t.flags & kNeedA) ? 1 : 0) + ((t.flags & kNeedB) ? 1 : 0);
     cost[blk] = c;
   }
+}
+
+// The plain rule: splits of at most 2 * kSplitTargetChunks chunks.
+CLEAR_HD void plain_forward_splits(Geom* g) {
+  g->ftarget = 2 * kSplitTargetChunks;
+  choose_splits(g->fnC, g->ftarget, kMaxSplits, &g->fS, &g->fcps);
+  g->n_txt_pairs = (long long)g->BH * g->nTq2 * g->fS;
+}
+
+CLEAR_HD void balance_forward_splits(Geom* g) {
+  plain_forward_splits(g);
+  if (g->n_text == 0 || g->nQ2 == 0 || (long long)g->BH * g->nQ2 > kMaxModelPairs || g->fS >= 8) return;
+#ifndef __CUDA_ARCH__
+  static thread_local int cost[kMaxModelPairs];
+  image_pair_costs(*g, cost);
   int best_s = g->fS;
   long long best = forward_makespan(*g, g->fS, cost, g->nQ2);
   for (int s = g->fS + 1; s <= imin(8, kMaxSplits); ++s) {

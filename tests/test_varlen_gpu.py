@@ -1,7 +1,9 @@
 """Mixed-resolution batches (clear_attn_fwd_varlen): items of their own (n_text, H, W) packed along
-the token axis run in one forward launch. Each item must equal clear_attn_fwd on that item alone
-(bit for bit: the same tiles, splits and arithmetic), and small items are checked against the
-oracle as well."""
+the token axis run in one forward launch. Each item's image rows must equal clear_attn_fwd on that
+item alone bit for bit (the same tiles and arithmetic). Its text rows are split-KV partials merged
+in a fixed order, and the batch may split them differently from the single call (a single call
+chooses its split count for its own load balance, the batch by the plain rule), so they are held to
+the single call within the bf16 bar. Small items are checked against the oracle as well."""
 import numpy as np
 import pytest
 import torch
@@ -10,6 +12,15 @@ import local_circular_window_b200 as L
 import oracle
 from clear_inputs import make_random
 from gpu_util import LSE_ABS, assert_close
+
+
+def _same_item(o, lse, oi, li, n_text, what):
+    """Image rows bit for bit; text rows within the bf16 bar (their split merge may differ)."""
+    assert torch.equal(o[..., n_text:, :], oi[..., n_text:, :]), what
+    assert torch.equal(lse[..., n_text:], li[..., n_text:]), what
+    if n_text:
+        assert_close(o[..., :n_text, :].float().cpu().numpy(), oi[..., :n_text, :].float().cpu().numpy(), f"{what} text")
+        assert (lse[..., :n_text] - li[..., :n_text]).abs().max().item() <= LSE_ABS, what
 
 
 def _packed(items, heads, d, seed):
@@ -43,8 +54,7 @@ def test_mixed_batch_equals_items_alone(items, heads, d, r, window):
         qi, ki, vi = (_item(t, s, n_text, H, W) for t in (q, k, v))
         oi, li = L.clear_attn_fwd(qi, ki, vi, n_text, H, W, r, window=window)
         torch.cuda.synchronize()
-        assert torch.equal(o[:, s:s + T], oi[0]), (n_text, H, W)
-        assert torch.equal(lse[:, s:s + T], li[0]), (n_text, H, W)
+        _same_item(o[:, s:s + T], lse[:, s:s + T], oi[0], li[0], n_text, (n_text, H, W))
         if T <= 2000:
             O, Lse = oracle.clear_attention_forward(qi, ki, vi, n_text, H, W, r, window=window)
             assert_close(o[:, s:s + T].float().cpu().numpy(), O[0], f"item {(n_text, H, W)}")
@@ -59,7 +69,7 @@ def test_single_item_batch_is_the_plain_call():
     oi, li = L.clear_attn_fwd(q.unsqueeze(0), k.unsqueeze(0), v.unsqueeze(0), 300, 33, 47, 6)
     torch.cuda.synchronize()
     assert L.clear_attn_check() == 0
-    assert torch.equal(o, oi[0]) and torch.equal(lse, li[0])
+    _same_item(o, lse, oi[0], li[0], 300, "single item")
 
 
 @pytest.mark.gpu
@@ -75,4 +85,4 @@ def test_many_small_items():
         T = n_text + H * W
         oi, li = L.clear_attn_fwd(*(_item(t, s, n_text, H, W) for t in (q, k, v)), n_text, H, W, 3)
         torch.cuda.synchronize()
-        assert torch.equal(o[:, s:s + T], oi[0]) and torch.equal(lse[:, s:s + T], li[0]), (n_text, H, W)
+        _same_item(o[:, s:s + T], lse[:, s:s + T], oi[0], li[0], n_text, (n_text, H, W))
