@@ -327,13 +327,11 @@ clear_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_c
     regs_dec<kBwdRegsLow>();
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
-      constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t q_addr = smem_u32(smem + L::kQ);
       const uint32_t do_addr = smem_u32(smem + L::kDO);
-      const uint32_t ds_addr = smem_u32(smem + L::kDS);
       static_assert(NST == 2, "S and dP of the next key tile are issued while dQ still reads this one's K");
       int stage = 0;
-      uint32_t ring_ph = 0, q_full_ph = 0, ds_full_ph = 0, sdp_free_ph = 0;
+      uint32_t ring_ph = 0, q_full_ph = 0, sdp_free_ph = 0;
       // dP = dO V^T and S = Q K^T of key tile j into TMEM (K/V ring slot `stage`), once the softmax
       // has read the previous pair. dP goes first: V arrives earlier than K (its slot is released
       // after dP, K's after dQ), and K's load overlaps dP's issue.
@@ -351,30 +349,49 @@ clear_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid_c
         if (j == n - 1) umma_commit(&bars[L::bQEmpty]);  // Q and dO: last reads issued
         return true;
       };
+      // This thread issues the score products (S, dP) of every tile; warp 10 issues the dQ
+      // products, so that the two streams' issue costs overlap (a thread is held ~80 cycles per
+      // tcgen05.mma, and the two share no TMEM columns: dQ reads dS and K from shared memory).
       for (long long w = blockIdx.x; w < p.n_work; w += gridDim.x) {
         const WorkItem it = decode_work(g, w);
         const int n = count_key_tiles(g, it);
         if (!mbar_wait(&bars[L::bQFull], q_full_ph, abort_flag, kDevTimeoutMma)) goto mma_done;
         q_full_ph ^= 1;
         tc_fence_after();
-        if (!issue_sdp(0, n)) goto mma_done;
         for (int j = 0; j < n; ++j) {
-          const int cur = stage;
+          if (!issue_sdp(j, n)) goto mma_done;
           if (++stage == NST) { stage = 0; ring_ph ^= 1; }
-          // S and dP of tile j + 1 run while the softmax turns tile j into dS.
-          if (j + 1 < n && !issue_sdp(j + 1, n)) goto mma_done;
-          // dQ += dS K
-          if (!mbar_wait(&bars[L::bDsFull], ds_full_ph, abort_flag, kDevTimeoutMma)) goto mma_done;
-          ds_full_ph ^= 1;
-          tc_fence_after();
-          mma_a_kmajor_b_mnmajor<D>(tmem + L::kTmemAcc, ds_addr, smem_u32(smem + L::kK + cur * L::kTileBytes), idesc_dq,
-                                    j > 0);
-          umma_commit(&bars[L::bDsEmpty]);
-          umma_commit(&bars[L::bKEmpty + cur]);
-          if (j == n - 1) umma_commit(&bars[L::bAccDone]);
         }
       }
     mma_done:;
+    }
+    __syncwarp();
+  } else if (warp == 10) {
+    regs_dec<kBwdRegsLow>();
+    if (lane == 0) {
+      constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t ds_addr = smem_u32(smem + L::kDS);
+      int stage = 0;
+      uint32_t ring_ph = 0, ds_full_ph = 0;
+      for (long long w = blockIdx.x; w < p.n_work; w += gridDim.x) {
+        const WorkItem it = decode_work(g, w);
+        const int n = count_key_tiles(g, it);
+        for (int j = 0; j < n; ++j) {
+          // dQ += dS K, once the softmax has stored dS of tile j. K's slot cannot have been
+          // reloaded (that waits for this product), so its full barrier still shows tile j's load.
+          if (!mbar_wait(&bars[L::bDsFull], ds_full_ph, abort_flag, kDevTimeoutMma)) goto dq_done;
+          ds_full_ph ^= 1;
+          if (!mbar_wait(&bars[L::bKFull + stage], ring_ph, abort_flag, kDevTimeoutMma)) goto dq_done;
+          tc_fence_after();
+          mma_a_kmajor_b_mnmajor<D>(tmem + L::kTmemAcc, ds_addr, smem_u32(smem + L::kK + stage * L::kTileBytes),
+                                    idesc_dq, j > 0);
+          umma_commit(&bars[L::bDsEmpty]);
+          umma_commit(&bars[L::bKEmpty + stage]);
+          if (j == n - 1) umma_commit(&bars[L::bAccDone]);
+          if (++stage == NST) { stage = 0; ring_ph ^= 1; }
+        }
+      }
+    dq_done:;
     }
     __syncwarp();
   } else if (warp < 8) {
