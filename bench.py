@@ -39,7 +39,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # dram__bytes_write.sum) on the 8K r=8 shape cut to 2 heads (the full 24-head launch is too large
 # to capture), per head; heads are independent, so a full launch moves heads x this. Valid only
 # for the kernel sources it was taken on (hash below); any change to them reports null.
-FWD_TRAFFIC = {"8k_r8": {"bytes_per_head": (728.778240e6 + 136.499712e6) / 2, "src": "ab9fa34c283b1c53"}}
+FWD_TRAFFIC = {"8k_r8": {"bytes_per_head": (729.469184e6 + 136.059136e6) / 2, "src": "08feca85a1acbfa9"}}
 FWD_SOURCES = ("clear_fwd.cuh", "clear_sched.cuh", "clear_common.cuh", "sm100_ptx.cuh")
 
 
