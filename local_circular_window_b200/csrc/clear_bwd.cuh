@@ -556,7 +556,7 @@ struct DkvLayout {
   static constexpr int kQ = kV + kTileBytes;             // + buf * kQStride
   static constexpr int kDO = kQ + kTileBytes;            // + buf * kQStride
   static constexpr int kQStride = 2 * kTileBytes;
-  static constexpr int kVec = kQ + 2 * kQStride;         // float lse2/dvec [2][2][128]
+  static constexpr int kVec = kQ + 2 * kQStride;         // float [tile parity][warpgroup][lse2 | D][64]
   static constexpr int kBars = kVec + 4 * kTile * 4;
   static constexpr int bKVFull = 0, bKVEmpty = 1, bQFull = 2 /* + buf */, bQEmpty = 4 /* + buf */,
                        bSFull = 6 /* + half */, bPFull = 8 /* + half */, bAccDone = 10;
@@ -565,9 +565,9 @@ struct DkvLayout {
   static constexpr int kWTab = kMisc + 16;
   static constexpr int kTotal = kWTab + kMaxRTable * 4;
   static constexpr int kAlloc = kTotal + 1024;
-  // TMEM: S^T of the partner tile's two 64-query halves at columns 0 and 64 (P^T of half h as bf16
-  // pairs over the first 32 columns of its S^T once the softmax has read it), dP^T likewise at 128
-  // and 192 (dS^T over them), and the dV, dK accumulators.
+  // TMEM: S^T of the partner tile's two 64-query halves at columns 0 and 64, dP^T likewise at 128
+  // and 192, and the dV, dK accumulators. Each warpgroup reads a 32-column chunk of each half and
+  // writes its P^T (dS^T) as bf16 pairs over the first 16 columns of that same chunk.
   static constexpr uint32_t kTmemS = 0, kTmemDP = 128, kTmemDV = 256, kTmemDK = 256 + D, kTmemCols = 512;
 };
 
@@ -678,17 +678,19 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
         umma_commit(&bars[L::bSFull + h]);
       };
       // dV += P^T dO and dK += dS^T Q over the 64 partner queries of half h (four K16 steps each).
+      // Step j's 16 queries are packed (8 columns) at the start of their warpgroup's 32-column chunk:
+      // column 64 h + 32 (j / 2) + 8 (j % 2) of the S^T (P^T) and dP^T (dS^T) regions.
       auto accumulate = [&](uint32_t cc, int h, bool first) {
         const uint32_t qb = cc & 1;
         const uint64_t do_desc = smem_desc_sw128(smem_u32(smem + L::kDO + qb * L::kQStride), kHalfBytes, 1024);
         const uint64_t q_desc = smem_desc_sw128(smem_u32(smem + L::kQ + qb * L::kQStride), kHalfBytes, 1024);
         #pragma unroll
         for (int j = 0; j < 4; ++j)
-          umma_ts(tmem + L::kTmemDV, tmem + L::kTmemS + 64 * h + 8 * j,
+          umma_ts(tmem + L::kTmemDV, tmem + L::kTmemS + 64 * h + 32 * (j >> 1) + 8 * (j & 1),
                   do_desc + (uint64_t)(((4 * h + j) * 2048) >> 4), idesc_acc, (first && j == 0) ? 0u : 1u);
         #pragma unroll
         for (int j = 0; j < 4; ++j)
-          umma_ts(tmem + L::kTmemDK, tmem + L::kTmemDP + 64 * h + 8 * j,
+          umma_ts(tmem + L::kTmemDK, tmem + L::kTmemDP + 64 * h + 32 * (j >> 1) + 8 * (j & 1),
                   q_desc + (uint64_t)(((4 * h + j) * 2048) >> 4), idesc_acc, (first && j == 0) ? 0u : 1u);
       };
       for (long long w = blockIdx.x; w < p.n_work; w += gridDim.x) {
@@ -753,12 +755,15 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
       ki.init(g, it);
       KeyTile t;
       while (ki.next(&t)) {
-        // Row statistics of the 128 partner queries into smem (column c <- thread c of warpgroup 0).
-        float* lse_s = vec + (tile_counter & 1) * 2 * kTile;
-        float* dv_s = lse_s + kTile;
+        // Row statistics of this warpgroup's 64 partner columns (its 32-column chunk of each half)
+        // into its own block, [lse2 | D][64] per tile parity: thread r stores lse2 of local column r
+        // (r < 64) or D of local column r - 64. Only this warpgroup reads them.
+        float* lse_s = vec + ((tile_counter & 1) * 2 + wg) * 2 * 64;
+        float* dv_s = lse_s + 64;
         ++tile_counter;
-        if (wg == 0) {
-          const int c = row;
+        {
+          const int cl = row & 63;
+          const int c = cl < 32 ? 32 * wg + cl : 32 + 32 * wg + cl;  // the tile's column
           bool ok;
           size_t qrow;
           if (t.kind == kLinear) {
@@ -769,9 +774,12 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
             ok = yq < g.H && xq < g.W && yq >= 0 && xq >= 0;
             qrow = ok ? (size_t)it.bh * g.T + g.n_text + (size_t)yq * g.W + xq : 0;
           }
-          lse_s[c] = ok ? p.l2vec[qrow] : INFINITY;
-          dv_s[c] = ok ? p.dvec[qrow] : 0.f;
+          if (row < 64)
+            lse_s[cl] = ok ? p.l2vec[qrow] : INFINITY;
+          else
+            dv_s[cl] = ok ? p.dvec[qrow] : 0.f;
         }
+        named_bar_sync(1 + wg, 128);
         for (int h = 0; h < 2; ++h) {  // the tile's two 64-query halves
           if (!mbar_wait(&bars[L::bSFull + h], s_full_ph[h], abort_flag, kDevTimeoutSoftmax)) goto softmax_done;
           s_full_ph[h] ^= 1;
@@ -781,12 +789,9 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
           tmem_ld32(tmem + lane_base + L::kTmemS + 32 * gch, sr);
           tmem_ld32(tmem + lane_base + L::kTmemDP + 32 * gch, dr);
           tmem_wait_ld();
-          // Every thread has read its S^T / dP^T columns (warpgroup 1's P^T / dS^T overwrite
-          // columns warpgroup 0 reads) and warpgroup 0 has stored the partner statistics.
-          tc_fence_before();
-          named_bar_sync(1, 256);
-          tc_fence_after();
-          // P^T = 2^(s c - lse2) on kept pairs, dS^T = P^T (dP^T - D), as bf16 pairs.
+          // P^T = 2^(s c - lse2) on kept pairs, dS^T = P^T (dP^T - D), as bf16 pairs, written over
+          // the first 16 columns of this warpgroup's own chunk (each thread only touches its own
+          // TMEM lane, so the two warpgroups never wait for each other).
           uint32_t keep = 0xffffffffu;
           if (t.flags != kFull) {
             if (t.kind == kLinear) {
@@ -801,7 +806,7 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
           const uint64_t sl2x2 = f32x2_pack(sl2, sl2);
           #pragma unroll
           for (int e = 0; e < 32; e += 2) {  // packed pairs: the same results as scalar fp32
-            const int c = gch * 32 + e;
+            const int c = h * 32 + e;  // local column
             const float x0 = ((keep >> e) & 1u) ? __uint_as_float(sr[e]) : -INFINITY;
             const float x1 = ((keep >> (e + 1)) & 1u) ? __uint_as_float(sr[e + 1]) : -INFINITY;
             const uint64_t x = f32x2_fma(f32x2_pack(x0, x1), sl2x2, f32x2_pack(-lse_s[c], -lse_s[c + 1]));
@@ -813,8 +818,8 @@ clear_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q_lin, const __grid
             pw[e / 2] = pack_bf16x2(p0, p1);
             dw[e / 2] = pack_bf16x2(f32x2_lo(d), f32x2_hi(d));
           }
-          tmem_st16(tmem + lane_base + L::kTmemS + 64 * h + 16 * wg, pw);
-          tmem_st16(tmem + lane_base + L::kTmemDP + 64 * h + 16 * wg, dw);
+          tmem_st16(tmem + lane_base + L::kTmemS + 32 * gch, pw);
+          tmem_st16(tmem + lane_base + L::kTmemDP + 32 * gch, dw);
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(&bars[L::bPFull + h]);
