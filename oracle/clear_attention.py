@@ -382,11 +382,13 @@ def rope_inv_freq(d_axis: int, theta: float = 10000.0, ntk: float = 1.0) -> np.n
     return base ** (-np.arange(0, d_axis, 2, dtype=np.float64) / d_axis)
 
 
-def rope_2d(x, n_text: int, H: int, W: int, theta: float = 10000.0, ntk: float = 1.0) -> np.ndarray:
+def rope_2d(x, n_text: int, H: int, W: int, theta: float = 10000.0, ntk: float = 1.0,
+            inverse: bool = False) -> np.ndarray:
     """Axial 2D rotary embedding of x [..., T, d] (float64 copy): image token (y, x) has dims
     [0, d/2) rotated by y and dims [d/2, d) by x, pair (2i, 2i+1) of an axis by angle
     position * rope_inv_freq(d/2)[i]: (a, b) -> (a cos - b sin, a sin + b cos). Text tokens are
-    unchanged."""
+    unchanged. inverse=True turns every pair by the negated angle: each 2x2 rotation is orthogonal,
+    so that is its transpose and its inverse (what carries a gradient back through the embedding)."""
     x = _as_f64(x).copy()
     d = x.shape[-1]
     assert d % 4 == 0
@@ -396,6 +398,8 @@ def rope_2d(x, n_text: int, H: int, W: int, theta: float = 10000.0, ntk: float =
     img = ~is_text
     for axis, pos in ((0, y_pos), (1, x_pos)):
         ang = pos[img][:, None] * inv[None, :]          # [N, da/2]
+        if inverse:
+            ang = -ang
         c, s_ = np.cos(ang), np.sin(ang)
         a = x[..., img, axis * da + 0:axis * da + da:2].copy()
         b = x[..., img, axis * da + 1:axis * da + da:2].copy()

@@ -91,3 +91,18 @@ def test_rope_forward_is_the_plain_forward_of_rotated_inputs():
     assert np.abs(O - O2).max() < 1e-12 and np.abs(L - L2).max() < 1e-12
     O3, _ = oracle.clear_attention_forward(q, k, v, 4, 5, 6, 3)
     assert np.abs(O - O3).max() > 1e-3
+
+
+def test_inverse_rotation_is_the_transpose():
+    # The inverse turns every pair back: it undoes the rotation both ways, and it is the transpose,
+    # <R x, y> = <x, R^T y> over every token.
+    wl = Workload("ri", 1, 2, 3, 5, 7, 16, 3)
+    x, y, _ = make_inputs(wl, seed=4, dtype=torch.float32)
+    xd, yd = x.double().numpy(), y.double().numpy()
+    rx = oracle.rope_2d(x, 3, 5, 7, ntk=10.0)
+    assert np.abs(oracle.rope_2d(rx, 3, 5, 7, ntk=10.0, inverse=True) - xd).max() < 1e-12
+    assert np.abs(oracle.rope_2d(oracle.rope_2d(x, 3, 5, 7, ntk=10.0, inverse=True), 3, 5, 7, ntk=10.0) - xd).max() < 1e-12
+    ry_t = oracle.rope_2d(y, 3, 5, 7, ntk=10.0, inverse=True)
+    assert np.abs((rx * yd).sum(-1) - (xd * ry_t).sum(-1)).max() < 1e-12
+    # and it is not the identity: an image token moves
+    assert np.abs(ry_t[:, :, 3:] - yd[:, :, 3:]).max() > 0.1
