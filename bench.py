@@ -364,9 +364,9 @@ def time_fp8_forward(L, peak, stream, seed):
 
 def time_rope_forward(L, peak, hbm, stream, seed):
     """The forward on rotary-embedded q and k (clear_attn_fwd_rope, NTK factor 10) on the headline
-    workload and on F2048 r=16, against the plain forward on the same inputs. The rotation pass is
-    HBM-bound: it reads q and k and writes their rotated copies once, 4 * B*heads*T*d bf16 bytes;
-    its time is the difference of the two medians."""
+    workload and on F2048 r=16, the plain forward on the same inputs, and the rotation pass alone
+    (clear_attn_rope, CUDA events around the call): it is HBM-bound, reading q and k and writing
+    their rotated copies once, 4 * B*heads*T*d bf16 bytes."""
     out = {}
     for name in ("8k_r8", "flux2048_r16"):
         wl = WORKLOADS[name]
@@ -375,22 +375,25 @@ def time_rope_forward(L, peak, hbm, stream, seed):
         lse = torch.empty((wl.B, wl.heads, wl.T), dtype=torch.float32, device="cuda")
         p = L.make_params(wl.B, wl.heads, wl.n_text, wl.H, wl.W, wl.d, wl.r)
         ws = torch.empty(L.rope_workspace_size(p), dtype=torch.uint8, device="cuda")
+        qr, kr = torch.empty_like(q), torch.empty_like(k)
+        rws = torch.empty(L.rope_rotate_workspace_size(p), dtype=torch.uint8, device="cuda")
         flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if q_bytes(wl) < (128 << 20) else None
         ms_rope = _median_call_ms(lambda: L.clear_attn_fwd_rope(q, k, v, wl.n_text, wl.H, wl.W, wl.r, ntk=10.0, o=o,
                                                                 lse=lse, workspace=ws, stream=stream),
                                   stream, flush=flush)
         ms_plain = _median_call_ms(lambda: L.clear_attn_fwd(q, k, v, wl.n_text, wl.H, wl.W, wl.r, o=o, lse=lse,
                                                             workspace=ws, stream=stream), stream, flush=flush)
+        rot_ms = _median_call_ms(lambda: L.clear_attn_rope(q, k, wl.n_text, wl.H, wl.W, ntk=10.0, q_out=qr, k_out=kr,
+                                                           workspace=rws, stream=stream), stream, calls=20, flush=flush)
         useful, _ = _flops(L, wl)
         rot_bytes = 4 * q_bytes(wl)
-        rot_ms = max(ms_rope - ms_plain, 1e-6)
         out[name] = {"ms_per_call": ms_rope, "plain_forward_ms": ms_plain, "rotation_ms": rot_ms,
                      "rotation_gbs": rot_bytes / (rot_ms * 1e-3) / 1e9,
                      "rotation_frac_of_hbm": rot_bytes / (rot_ms * 1e-3) / 1e9 / hbm if hbm else None,
                      "rotation_bytes": rot_bytes,
                      "useful_tflops": useful / (ms_rope * 1e-3) / 1e12,
                      "frac_of_peak": useful / (ms_rope * 1e-3) / 1e12 / peak}
-        del q, k, v, o, lse, ws, flush
+        del q, k, v, o, lse, ws, qr, kr, rws, flush
         torch.cuda.empty_cache()
     if L.clear_attn_check() != 0:
         raise RuntimeError("device error timing the RoPE forward")

@@ -227,6 +227,26 @@ CLEAR_API clear_status_t clear_attn_fwd_rope(const clear_attn_params_t* params, 
                                              const void* q, const void* k, const void* v, void* o, float* lse,
                                              void* workspace, size_t workspace_bytes, void* stream);
 
+/* Workspace bytes of clear_attn_rope: the (cos, sin) table, max(H, W) * d/4 fp32 pairs, rounded up to
+ * 256 bytes. */
+CLEAR_API size_t clear_attn_rope_workspace_size(const clear_attn_params_t* params, clear_status_t* status);
+
+/*
+ * The rotary embedding of clear_attn_fwd_rope on its own: q and k (bf16 [B, heads, T, d],
+ * contiguous, d = 64 or 128) rotated into q_out and k_out, each element read and written once and
+ * rounded to bf16 once; text tokens are copied unchanged. inverse = 1 turns every pair by the
+ * negated angle, the transpose of the rotation (each 2x2 rotation is orthogonal): rotating the
+ * gradients of the rotated q and k back with it gives the gradients of q and k, so a training step
+ * can rotate once, run clear_attn_fwd and clear_attn_bwd on the rotated tensors, and rotate dQ, dK
+ * back. q_out may be q and k_out may be k (in place). workspace: clear_attn_rope_workspace_size
+ * bytes, 256-byte aligned, written on `stream`. CLEAR_ERR_INVALID_ARG for theta <= 1, ntk <= 0,
+ * non-finite values, inverse other than 0 or 1, or misaligned pointers; CLEAR_ERR_WORKSPACE for a
+ * small or misaligned workspace; otherwise as clear_attn_fwd.
+ */
+CLEAR_API clear_status_t clear_attn_rope(const clear_attn_params_t* params, const clear_attn_rope_t* rope, int inverse,
+                                         const void* q, const void* k, void* q_out, void* k_out, void* workspace,
+                                         size_t workspace_bytes, void* stream);
+
 /*
  * Mixed-resolution batch forward: n_items problems of their own (n_text, H, W) in ONE launch (their
  * pairs form one work list), e.g. a batch holding 1024^2 and 2048^2 images at once. Each item is the

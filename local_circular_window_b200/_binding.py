@@ -87,6 +87,10 @@ _lib.clear_attn_fwd_rope_workspace_size.restype = ctypes.c_size_t
 _lib.clear_attn_fwd_rope_workspace_size.argtypes = [_P, ctypes.POINTER(_i)]
 _lib.clear_attn_fwd_rope.restype = _i
 _lib.clear_attn_fwd_rope.argtypes = [_P, ctypes.POINTER(ClearRope), _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+_lib.clear_attn_rope_workspace_size.restype = ctypes.c_size_t
+_lib.clear_attn_rope_workspace_size.argtypes = [_P, ctypes.POINTER(_i)]
+_lib.clear_attn_rope.restype = _i
+_lib.clear_attn_rope.argtypes = [_P, ctypes.POINTER(ClearRope), _i, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 _lib.clear_attn_fwd_fp8.restype = _i
 _lib.clear_attn_fwd_fp8.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 _lib.clear_attn_fwd_varlen_workspace_size.restype = ctypes.c_size_t
@@ -535,3 +539,38 @@ def _check_host(name, t, shape, dtype):
     # Page-locking is checked by the library (CLEAR_ERR_INVALID_ARG if missing).
     if not (t.device.type == "cpu" and t.dtype == dtype and t.is_contiguous() and tuple(t.shape) == tuple(shape)):
         raise ValueError(f"{name} must be a contiguous CPU {dtype} tensor of shape {tuple(shape)}")
+
+
+def rope_rotate_workspace_size(p: ClearParams) -> int:
+    st = _i(0)
+    n = _lib.clear_attn_rope_workspace_size(ctypes.byref(p), ctypes.byref(st))
+    if st.value != CLEAR_OK:
+        raise ClearError(st.value, "clear_attn_rope_workspace_size")
+    return n
+
+
+def clear_attn_rope(q, k, n_text: int, H: int, W: int, theta: float = 10000.0, ntk: float = 1.0, inverse: bool = False,
+                    q_out=None, k_out=None, workspace=None, stream=None):
+    """The rotary embedding alone through clear_attn_rope: q and k (bf16 [B, heads, T, d]) rotated by
+    axial 2D RoPE with the NTK-aware base (inverse=True: by the negated angles, the transpose) into
+    q_out and k_out (new tensors by default; q_out=q, k_out=k rotates in place). Returns
+    (q_out, k_out)."""
+    B, heads, T, d = q.shape
+    if T != n_text + H * W:
+        raise ValueError("T must equal n_text + H * W")
+    for name, t in (("q", q), ("k", k)):
+        _check_qkv(name, t, q.shape)
+    p = make_params(B, heads, n_text, H, W, d, 1)
+    rope = ClearRope(theta, ntk)
+    q_out = torch.empty_like(q) if q_out is None else q_out
+    k_out = torch.empty_like(k) if k_out is None else k_out
+    for name, t in (("q_out", q_out), ("k_out", k_out)):
+        _check_qkv(name, t, q.shape)
+    if workspace is None:
+        workspace = torch.empty(rope_rotate_workspace_size(p), dtype=torch.uint8, device=q.device)
+    status = _lib.clear_attn_rope(ctypes.byref(p), ctypes.byref(rope), 1 if inverse else 0, _ptr(q), _ptr(k), _ptr(q_out),
+                                  _ptr(k_out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                  _stream_ptr(stream))
+    if status != CLEAR_OK:
+        raise ClearError(status, "clear_attn_rope")
+    return q_out, k_out

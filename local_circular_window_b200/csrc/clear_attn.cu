@@ -396,26 +396,31 @@ RopeWorkspace rope_workspace_layout(const Geom& g) {
 
 size_t rope_workspace_bytes(const Geom& g) { return rope_workspace_layout(g).total; }
 
-// Launch shape of the rotation: a grid-stride loop over every chunk, kRopeUnroll chunks in flight
-// per thread, as many blocks as are resident at once on the device (no tail wave).
+// The rotation streamed through shared memory: as many blocks as are resident at once (two per SM
+// at 96 KB of shared memory each), each walking its pieces of q and k round-robin.
 template <int D>
-unsigned rope_grid(long long chunks, int num_sms) {
+clear_status_t launch_rope_bulk(const RopeBulkParams& p, int num_sms, cudaStream_t stream) {
+  if (cudaFuncSetAttribute(clear_rope_bulk_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kRopeBulkSmem) !=
+      cudaSuccess)
+    return CLEAR_ERR_CUDA;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, clear_rope_kernel<D>, kRopeThreads, 0) != cudaSuccess ||
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, clear_rope_bulk_kernel<D>, kRopeBulkThreads,
+                                                    kRopeBulkSmem) != cudaSuccess ||
       per_sm < 1)
     per_sm = 1;
-  const long long per_block = (long long)kRopeThreads * kRopeUnroll;
-  const long long need = (2 * chunks + per_block - 1) / per_block;
   const long long cap = (long long)num_sms * per_sm;
-  return (unsigned)(need < cap ? need : cap);
+  const long long grid = 2 * p.pieces < cap ? 2 * p.pieces : cap;
+  clear_rope_bulk_kernel<D><<<(unsigned)grid, kRopeBulkThreads, kRopeBulkSmem, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? CLEAR_OK : CLEAR_ERR_CUDA;
 }
 
-clear_status_t launch_rope(const Geom& g, const clear_attn_rope_t& rope, const void* q, const void* k, void* ws,
-                           int num_sms, cudaStream_t stream) {
-  const RopeWorkspace wl = rope_workspace_layout(g);
-  char* base = static_cast<char*>(ws);
+// The (cos, sin) table into tab (rope_table_shape(g).bytes, 16-byte aligned), then q and k rotated
+// into q_out and k_out (which may be q and k themselves: every 16-byte chunk is read and written by
+// the same thread). inverse turns every pair back by the negated angle.
+clear_status_t launch_rope(const Geom& g, const clear_attn_rope_t& rope, bool inverse, const void* q, const void* k,
+                           void* q_out, void* k_out, void* tab, int num_sms, cudaStream_t stream) {
   RopeTableParams tp{};
-  tp.tab = reinterpret_cast<float2*>(base + wl.tab_off);
+  tp.tab = static_cast<float2*>(tab);
   tp.n = rope_table_shape(g).n;
   tp.np = g.d / 4;
   const int da = g.d / 2;
@@ -424,22 +429,20 @@ clear_status_t launch_rope(const Geom& g, const clear_attn_rope_t& rope, const v
   clear_rope_table_kernel<<<(unsigned)((tp.n * tp.np + kRopeThreads - 1) / kRopeThreads), kRopeThreads, 0, stream>>>(
       tp);
   if (cudaGetLastError() != cudaSuccess) return CLEAR_ERR_CUDA;
-  RopeParams p{};
-  p.src[0] = static_cast<const uint4*>(q);
-  p.src[1] = static_cast<const uint4*>(k);
-  p.dst[0] = reinterpret_cast<uint4*>(base + wl.q_off);
-  p.dst[1] = reinterpret_cast<uint4*>(base + wl.k_off);
-  p.tab = reinterpret_cast<const float4*>(base + wl.tab_off);
-  p.chunks = (long long)g.BH * g.T * (g.d / 8);
+  RopeBulkParams p{};
+  p.src[0] = static_cast<const uint8_t*>(q);
+  p.src[1] = static_cast<const uint8_t*>(k);
+  p.dst[0] = static_cast<uint8_t*>(q_out);
+  p.dst[1] = static_cast<uint8_t*>(k_out);
+  p.tab = static_cast<const float4*>(tab);
+  p.bytes = (long long)g.BH * g.T * g.d * 2;
+  p.pieces = (p.bytes + kRopePiece - 1) / kRopePiece;
   p.T = g.T;
   p.n_text = g.n_text;
   p.W = g.W;
-  if (p.chunks == 0) return CLEAR_OK;
-  if (g.d == 128)
-    clear_rope_kernel<128><<<rope_grid<128>(p.chunks, num_sms), kRopeThreads, 0, stream>>>(p);
-  else
-    clear_rope_kernel<64><<<rope_grid<64>(p.chunks, num_sms), kRopeThreads, 0, stream>>>(p);
-  return cudaGetLastError() == cudaSuccess ? CLEAR_OK : CLEAR_ERR_CUDA;
+  p.sin_sign = inverse ? -1.f : 1.f;
+  if (p.bytes == 0) return CLEAR_OK;
+  return g.d == 128 ? launch_rope_bulk<128>(p, num_sms, stream) : launch_rope_bulk<64>(p, num_sms, stream);
 }
 
 bool rope_ok(const clear_attn_rope_t* rope) {
@@ -893,13 +896,37 @@ clear_status_t clear_attn_fwd_rope(const clear_attn_params_t* params, const clea
   const clear_status_t st = check_device(&num_sms);
   if (st != CLEAR_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const clear_status_t rs = launch_rope(c.g, *rope, q, k, workspace, num_sms, s);
-  if (rs != CLEAR_OK) return rs;
   const RopeWorkspace wl = rope_workspace_layout(c.g);
+  char* base = static_cast<char*>(workspace);
+  const clear_status_t rs = launch_rope(c.g, *rope, false, q, k, base + wl.q_off, base + wl.k_off, base + wl.tab_off,
+                                        num_sms, s);
+  if (rs != CLEAR_OK) return rs;
   const TensorStrides cs = contiguous_strides(c.g);
   const TensorStrides st4[4] = {cs, cs, cs, cs};
-  char* base = static_cast<char*>(workspace);
   return run_fwd(c.g, st4, base + wl.q_off, base + wl.k_off, v, o, lse, workspace, s);
+}
+
+size_t clear_attn_rope_workspace_size(const clear_attn_params_t* params, clear_status_t* status) {
+  const Checked c = check_params(params);
+  if (status) *status = c.st;
+  if (c.st != CLEAR_OK) return 0;
+  return align256(rope_table_shape(c.g).bytes);
+}
+
+clear_status_t clear_attn_rope(const clear_attn_params_t* params, const clear_attn_rope_t* rope, int inverse,
+                               const void* q, const void* k, void* q_out, void* k_out, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  const Checked c = check_params(params);
+  if (c.st != CLEAR_OK) return c.st;
+  if (!rope_ok(rope) || (inverse != 0 && inverse != 1)) return CLEAR_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_out) || !aligned16(k_out)) return CLEAR_ERR_INVALID_ARG;
+  if (workspace_bytes < align256(rope_table_shape(c.g).bytes) || !workspace ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return CLEAR_ERR_WORKSPACE;
+  int num_sms = 0;
+  const clear_status_t st = check_device(&num_sms);
+  if (st != CLEAR_OK) return st;
+  return launch_rope(c.g, *rope, inverse != 0, q, k, q_out, k_out, workspace, num_sms, static_cast<cudaStream_t>(stream));
 }
 
 size_t clear_attn_fwd_varlen_workspace_size(const clear_attn_params_t* params, int n_items, const int* item_shapes,

@@ -211,3 +211,16 @@ def test_varlen_workspace_grows_with_text_rows():
     assert b > a > 0 and a % 256 == 0 and b % 256 == 0
     with pytest.raises(L.ClearError):
         L.varlen_workspace_size(2, 128, 4, [(1, 2, 2)] * 4097)
+
+
+def test_rope_rotation_workspace_size():
+    # The stand-alone rotation's workspace is its (cos, sin) table: max(H, W) positions x d/4 fp32
+    # pairs, rounded up to 256 bytes; bad parameters report their status.
+    for n_text, H, W, d in ((512, 64, 64, 128), (0, 13, 50, 64), (77, 24, 40, 128)):
+        p = L.make_params(1, 2, n_text, H, W, d, 1)
+        want = (max(H, W) * (d // 4) * 8 + 255) // 256 * 256
+        assert L.rope_rotate_workspace_size(p) == want
+    st = ctypes.c_int(0)
+    bad = L.make_params(1, 2, 4, 8, 8, 96, 1)  # d = 96 is not supported
+    assert L.lib().clear_attn_rope_workspace_size(ctypes.byref(bad), ctypes.byref(st)) == 0
+    assert st.value != 0

@@ -92,3 +92,70 @@ def test_rope_rejects_bad_parameters():
             L.clear_attn_fwd_rope(q, k, v, 4, 8, 8, 2, theta=theta, ntk=ntk)
         assert e.value.status == 1
     assert L.clear_attn_check() == 0
+
+
+# The rotation alone (clear_attn_rope): the exact rotation rounded to bf16. bf16 keeps 8 significant
+# bits, so rounding moves a value v by at most 2^-8 |v|; the fp32 arithmetic and table add at most
+# ~2^-20 of the operands (inputs are unit normal: an absolute 1e-5 covers it).
+def _assert_rotated(got, ref, what):
+    got = got.double().cpu().numpy()
+    err = np.abs(got - ref)
+    bound = 2.0 ** -8 * np.abs(ref) + 1e-5
+    assert (err <= bound).all(), f"{what}: worst excess {(err - bound).max():.3e}"
+
+
+ROT = [
+    (Workload("rot_ragged", 2, 3, 77, 24, 40, 128, 1), 10000.0, 10.0),
+    (Workload("rot_d64", 1, 2, 200, 13, 50, 64, 1), 500.0, 1.0),
+    (Workload("rot_no_text", 1, 2, 0, 19, 21, 128, 1), 10000.0, 2.0),
+]
+
+
+@pytest.mark.parametrize("wl,theta,ntk", ROT, ids=lambda c: c.name if hasattr(c, "name") else str(c))
+def test_rope_rotation_alone(wl, theta, ntk):
+    q, k, _ = gpu_inputs(wl, seed=73)
+    for inverse in (False, True):
+        qr, kr = L.clear_attn_rope(q, k, wl.n_text, wl.H, wl.W, theta=theta, ntk=ntk, inverse=inverse)
+        torch.cuda.synchronize()
+        for name, x, xr in (("q", q, qr), ("k", k, kr)):
+            ref = oracle.rope_2d(x.cpu(), wl.n_text, wl.H, wl.W, theta, ntk, inverse=inverse)
+            _assert_rotated(xr, ref, f"{wl.name} {name} inverse={inverse}")
+            assert torch.equal(xr[:, :, :wl.n_text], x[:, :, :wl.n_text])  # text tokens are copied
+    # in place equals out of place, and the inverse undoes the rotation up to two bf16 roundings
+    q2, k2 = q.clone(), k.clone()
+    L.clear_attn_rope(q2, k2, wl.n_text, wl.H, wl.W, theta=theta, ntk=ntk, q_out=q2, k_out=k2)
+    qr, kr = L.clear_attn_rope(q, k, wl.n_text, wl.H, wl.W, theta=theta, ntk=ntk)
+    torch.cuda.synchronize()
+    assert torch.equal(q2, qr) and torch.equal(k2, kr)
+    qb, _ = L.clear_attn_rope(qr, kr, wl.n_text, wl.H, wl.W, theta=theta, ntk=ntk, inverse=True)
+    torch.cuda.synchronize()
+    back = qb.double().cpu().numpy()
+    x0 = q.double().cpu().numpy()
+    # each rounding moves a pair by at most 2^-8 of its norm, and the rotations keep norms
+    pair_norm = np.repeat(np.sqrt(x0[..., 0::2] ** 2 + x0[..., 1::2] ** 2), 2, axis=-1)
+    assert (np.abs(back - x0) <= 2.0 ** -7 * pair_norm * 1.01 + 1e-5).all()
+    assert L.clear_attn_check() == 0
+
+
+def test_rope_rotation_flux2048_heads():
+    wl = WORKLOADS["flux2048_r16"]
+    q, k, _ = gpu_inputs(wl, seed=74)
+    qr, kr = L.clear_attn_rope(q, k, wl.n_text, wl.H, wl.W, ntk=10.0)
+    torch.cuda.synchronize()
+    for h in (0, 23):
+        ref = oracle.rope_2d(q[0:1, h:h + 1].cpu(), wl.n_text, wl.H, wl.W, ntk=10.0)
+        _assert_rotated(qr[0:1, h:h + 1], ref, f"head {h}")
+
+
+def test_rope_rotation_rejects_bad_inverse():
+    import ctypes
+    wl = Workload("rot_bad", 1, 1, 4, 8, 8, 128, 1)
+    q, k, _ = gpu_inputs(wl, seed=75)
+    p = L.make_params(1, 1, 4, 8, 8, 128, 1)
+    rope = L.ClearRope(10000.0, 1.0)
+    ws = torch.empty(L.rope_rotate_workspace_size(p), dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(q)
+    vp = lambda t: ctypes.c_void_p(t.data_ptr())
+    st = L.lib().clear_attn_rope(ctypes.byref(p), ctypes.byref(rope), 2, vp(q), vp(k), vp(out), vp(out), vp(ws),
+                                 ctypes.c_size_t(ws.numel()), None)
+    assert L.status_string(st) == "CLEAR_ERR_INVALID_ARG"
