@@ -247,6 +247,24 @@ CLEAR_API clear_status_t clear_attn_rope(const clear_attn_params_t* params, cons
                                          const void* q, const void* k, void* q_out, void* k_out, void* workspace,
                                          size_t workspace_bytes, void* stream);
 
+/* Workspace bytes of clear_attn_bwd_rope: the backward's, the (cos, sin) table, the rotated q and k. */
+CLEAR_API size_t clear_attn_bwd_rope_workspace_size(const clear_attn_params_t* params, clear_status_t* status);
+
+/*
+ * The backward of clear_attn_fwd_rope: the gradients with respect to the unrotated q, k and v.
+ * q and k are rotated into the workspace as the forward saw them, clear_attn_bwd runs on the
+ * rotated tensors (o and lse are the ones clear_attn_fwd_rope returned), and dq, dk are then turned
+ * back by the inverse rotation, the transpose of the rotation (each 2x2 rotation is orthogonal),
+ * in place; dv needs no turn. Tensors as clear_attn_bwd (contiguous; d = 64 or 128; the shifted
+ * window is CLEAR_ERR_UNSUPPORTED as there). workspace: clear_attn_bwd_rope_workspace_size bytes,
+ * 256-byte aligned, written on `stream`. CLEAR_ERR_INVALID_ARG for the rotary parameters as in
+ * clear_attn_fwd_rope; otherwise as clear_attn_bwd.
+ */
+CLEAR_API clear_status_t clear_attn_bwd_rope(const clear_attn_params_t* params, const clear_attn_rope_t* rope,
+                                             const void* q, const void* k, const void* v, const void* o,
+                                             const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                                             void* workspace, size_t workspace_bytes, void* stream);
+
 /*
  * Mixed-resolution batch forward: n_items problems of their own (n_text, H, W) in ONE launch (their
  * pairs form one work list), e.g. a batch holding 1024^2 and 2048^2 images at once. Each item is the

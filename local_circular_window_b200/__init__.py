@@ -14,7 +14,7 @@ _EXPORTS = {
     "fwd_host_workspace_size", "fwd_workspace_size", "header_functions", "item_tiles", "lib", "make_params",
     "pair_counts", "selftest_expiry", "status_string", "version", "clear_attn_fwd_varlen", "varlen_workspace_size",
     "varlen_tokens", "clear_attn_fwd_fp8", "clear_attn_fwd_rope", "rope_workspace_size", "ClearRope",
-    "clear_attn_rope", "rope_rotate_workspace_size",
+    "clear_attn_rope", "rope_rotate_workspace_size", "clear_attn_bwd_rope",
 }
 
 

@@ -89,6 +89,11 @@ _lib.clear_attn_fwd_rope.restype = _i
 _lib.clear_attn_fwd_rope.argtypes = [_P, ctypes.POINTER(ClearRope), _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 _lib.clear_attn_rope_workspace_size.restype = ctypes.c_size_t
 _lib.clear_attn_rope_workspace_size.argtypes = [_P, ctypes.POINTER(_i)]
+_lib.clear_attn_bwd_rope_workspace_size.restype = ctypes.c_size_t
+_lib.clear_attn_bwd_rope_workspace_size.argtypes = [_P, ctypes.POINTER(_i)]
+_lib.clear_attn_bwd_rope.restype = _i
+_lib.clear_attn_bwd_rope.argtypes = [_P, ctypes.POINTER(ClearRope), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                     ctypes.c_size_t, _vp]
 _lib.clear_attn_rope.restype = _i
 _lib.clear_attn_rope.argtypes = [_P, ctypes.POINTER(ClearRope), _i, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 _lib.clear_attn_fwd_fp8.restype = _i
@@ -574,3 +579,31 @@ def clear_attn_rope(q, k, n_text: int, H: int, W: int, theta: float = 10000.0, n
     if status != CLEAR_OK:
         raise ClearError(status, "clear_attn_rope")
     return q_out, k_out
+
+
+def clear_attn_bwd_rope(q, k, v, o, lse, dO, n_text: int, H: int, W: int, r: int, theta: float = 10000.0,
+                        ntk: float = 1.0, dq=None, dk=None, dv=None, workspace=None, stream=None, window="circle"):
+    """Backward of clear_attn_fwd_rope through clear_attn_bwd_rope: gradients with respect to the
+    unrotated q, k and v (o and lse as clear_attn_fwd_rope returned them). Returns (dq, dk, dv)."""
+    B, heads, T, d = q.shape
+    if T != n_text + H * W:
+        raise ValueError("T must equal n_text + H * W")
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dO", dO)):
+        _check_qkv(name, t, q.shape)
+    p = make_params(B, heads, n_text, H, W, d, r, window)
+    rope = ClearRope(theta, ntk)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        st = _i(0)
+        n = _lib.clear_attn_bwd_rope_workspace_size(ctypes.byref(p), ctypes.byref(st))
+        if st.value != CLEAR_OK:
+            raise ClearError(st.value, "clear_attn_bwd_rope_workspace_size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+    st = _lib.clear_attn_bwd_rope(ctypes.byref(p), ctypes.byref(rope), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                  _ptr(dO), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    if st != CLEAR_OK:
+        raise ClearError(st, "clear_attn_bwd_rope")
+    return dq, dk, dv

@@ -1112,6 +1112,58 @@ clear_status_t clear_attn_bwd(const clear_attn_params_t* params, const void* q, 
                                        maps.v_img, do_lin, do_img, num_sms, s);
 }
 
+// Backward through the rotary embedding: [backward workspace][table][rotated q][rotated k].
+struct BwdRopeWorkspace {
+  size_t tab_off, q_off, k_off, total;
+};
+
+BwdRopeWorkspace bwd_rope_workspace_layout(const Geom& g) {
+  BwdRopeWorkspace w;
+  const size_t qk = (size_t)g.BH * g.T * g.d * sizeof(__nv_bfloat16);
+  w.tab_off = align256(bwd_workspace_layout(g).total);
+  w.q_off = w.tab_off + align256(rope_table_shape(g).bytes);
+  w.k_off = w.q_off + align256(qk);
+  w.total = w.k_off + align256(qk);
+  return w;
+}
+
+size_t clear_attn_bwd_rope_workspace_size(const clear_attn_params_t* params, clear_status_t* status) {
+  const Checked c = check_params(params);
+  if (status) *status = c.st;
+  if (c.st != CLEAR_OK) return 0;
+  return bwd_rope_workspace_layout(c.g).total;
+}
+
+clear_status_t clear_attn_bwd_rope(const clear_attn_params_t* params, const clear_attn_rope_t* rope, const void* q,
+                                   const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                                   void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  const Checked c = check_params(params);
+  if (c.st != CLEAR_OK) return c.st;
+  if (c.g.window == kShifted) return CLEAR_ERR_UNSUPPORTED;
+  if (!rope_ok(rope)) return CLEAR_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dO) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return CLEAR_ERR_INVALID_ARG;
+  const BwdRopeWorkspace wl = bwd_rope_workspace_layout(c.g);
+  if (workspace_bytes < wl.total || !workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return CLEAR_ERR_WORKSPACE;
+  int num_sms = 0;
+  const clear_status_t st = check_device(&num_sms);
+  if (st != CLEAR_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* base = static_cast<char*>(workspace);
+  // q, k rotated as the forward saw them; the backward on the rotated tensors; then dQ, dK carried
+  // back through the rotation by its transpose, in place.
+  clear_status_t rs = launch_rope(c.g, *rope, false, q, k, base + wl.q_off, base + wl.k_off, base + wl.tab_off,
+                                  num_sms, s);
+  if (rs != CLEAR_OK) return rs;
+  rs = clear_attn_bwd(params, base + wl.q_off, base + wl.k_off, v, o, lse, dO, dq, dk, dv, workspace, wl.tab_off,
+                      stream);
+  if (rs != CLEAR_OK) return rs;
+  return launch_rope(c.g, *rope, true, dq, dk, dq, dk, base + wl.tab_off, num_sms, s);
+}
+
 static thread_local int t_last_diag[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 
 clear_status_t clear_attn_check(void* stream) {

@@ -159,3 +159,31 @@ def test_rope_rotation_rejects_bad_inverse():
     st = L.lib().clear_attn_rope(ctypes.byref(p), ctypes.byref(rope), 2, vp(q), vp(k), vp(out), vp(out), vp(ws),
                                  ctypes.c_size_t(ws.numel()), None)
     assert L.status_string(st) == "CLEAR_ERR_INVALID_ARG"
+
+
+# The backward through the rotary embedding (clear_attn_bwd_rope): against the oracle's backward on
+# the rotated q and k as bf16 (the operands the kernels multiply), with dQ and dK turned back by the
+# oracle's inverse rotation in float64. The kernel rounds dQ and dK once more after turning them
+# back, inside the standard bf16 bar.
+BWD = [
+    (Workload("rbwd_ragged", 1, 2, 77, 24, 40, 128, 5), 10000.0, 10.0, "circle"),
+    (Workload("rbwd_d64_square", 1, 2, 30, 16, 20, 64, 4), 500.0, 2.0, "square"),
+]
+
+
+@pytest.mark.parametrize("wl,theta,ntk,window", BWD, ids=lambda c: c.name if hasattr(c, "name") else str(c))
+def test_rope_backward(wl, theta, ntk, window):
+    q, k, v, dO = gpu_inputs(wl, seed=76, grad=True)
+    o, lse = L.clear_attn_fwd_rope(q, k, v, wl.n_text, wl.H, wl.W, wl.r, theta=theta, ntk=ntk, window=window)
+    dq, dk, dv = L.clear_attn_bwd_rope(q, k, v, o, lse, dO, wl.n_text, wl.H, wl.W, wl.r, theta=theta, ntk=ntk,
+                                       window=window)
+    torch.cuda.synchronize()
+    assert L.clear_attn_check() == 0
+    qb = rotated_bf16(q.cpu(), wl.n_text, wl.H, wl.W, theta, ntk)
+    kb = rotated_bf16(k.cpu(), wl.n_text, wl.H, wl.W, theta, ntk)
+    rq, rk, rv = oracle.clear_attention_backward(qb, kb, v.cpu(), dO.cpu(), wl.n_text, wl.H, wl.W, wl.r, window=window)
+    rq = oracle.rope_2d(rq, wl.n_text, wl.H, wl.W, theta, ntk, inverse=True)
+    rk = oracle.rope_2d(rk, wl.n_text, wl.H, wl.W, theta, ntk, inverse=True)
+    assert_close(dq.float().cpu().numpy(), rq, f"{wl.name} dQ")
+    assert_close(dk.float().cpu().numpy(), rk, f"{wl.name} dK")
+    assert_close(dv.float().cpu().numpy(), rv, f"{wl.name} dV")
