@@ -10,16 +10,19 @@
 // Kernels (all deterministic, no floating-point atomics):
 //   preprocess  D and LSE * log2(e) per row                             (CUDA cores, HBM-bound)
 //   dq kernel   Q-stationary: per query tile, visit its 128-key tiles; S, dP -> TMEM,
-//               dS -> smem (bf16), dQ += dS K in TMEM; S and dP of the next key tile are issued
-//               before dQ of this one. Text query tiles are split over key chunks into fp32
-//               partials.
+//               dS -> smem (bf16), dQ += dS K in TMEM. One thread issues S and dP (the next key
+//               tile's while the softmax works on this one), another the dQ products; V's ring
+//               slot is released after dP, K's after dQ. Text query tiles are split over key
+//               chunks into fp32 partials.
 //   dkdv kernel KV-stationary: per key tile, visit the query tiles that keep it. The mask is
 //               symmetric, so the same tile enumeration with the roles of query and key swapped
-//               gives exactly those tiles. S^T, dP^T -> TMEM; P^T, dS^T written back over them
-//               (bf16); dV += P^T dO, dK += dS^T Q in TMEM with the A operand read from TMEM;
-//               partner Q / dO double-buffered. Text key tiles are split over query chunks into
-//               fp32 partials.
-// Both kernels split each tile's 128 columns over two softmax warpgroups (64 each).
+//               gives exactly those tiles. S^T, dP^T -> TMEM, per half of 64 partner queries;
+//               P^T, dS^T written back over them (bf16); dV += P^T dO, dK += dS^T Q in TMEM with
+//               the A operand read from TMEM, so one half's products overlap the other half's
+//               softmax; partner Q / dO double-buffered. Text key tiles are split over query
+//               chunks into fp32 partials.
+// Both kernels split each tile's 128 columns over two softmax warpgroups (64 each), which never
+// wait for each other.
 //   reduce      sums the split partials of the text rows in a fixed order and writes bf16.
 #pragma once
 #include <cuda_bf16.h>
