@@ -21,8 +21,8 @@
 //               the A operand read from TMEM, so one half's products overlap the other half's
 //               softmax; partner Q / dO double-buffered. Text key tiles are split over query
 //               chunks into fp32 partials.
-// Both kernels split each tile's 128 columns over two softmax warpgroups (64 each), which never
-// wait for each other.
+// Both kernels split each tile's 128 columns over two softmax warpgroups (64 each); in dkdv they
+// never wait for each other, in dq both arrive on the barriers that hand S / dP back and dS on.
 //   reduce      sums the split partials of the text rows in a fixed order and writes bf16.
 #pragma once
 #include <cuda_bf16.h>
